@@ -1,0 +1,258 @@
+/*
+ * CPU oracle for the STEPQuant packed-state decode step -- TEST INFRASTRUCTURE
+ * ONLY (see stepq_oracle.h): loaded by the tests, the smoke check and the
+ * benchmark's CPU-baseline leg, never by the product path.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fPIC -shared (oracle/build.py).
+ */
+#include "stepq_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---- IEEE binary16, round to nearest even, written from the format's
+ * definition: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits;
+ * normal numbers span [2^-14, 65504], subnormals are multiples of 2^-24. */
+uint16_t oracle_to_fp16(double x)
+{
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    if (isnan(x)) return 0x7E00u;
+    double a = fabs(x);
+    if (isinf(a)) return sign | 0x7C00u;
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);          /* a in [2^(e-1), 2^e) */
+    int ex = e - 1;
+    if (ex < -14) ex = -14; /* the subnormal range shares the quantum 2^-24 */
+    double quantum = ldexp(1.0, ex - 10);
+    double y = nearbyint(a / quantum) * quantum; /* exact scaling, ties to even */
+    if (y > 65504.0) return sign | 0x7C00u;
+    if (y < ldexp(1.0, -14)) return sign | (uint16_t)(y / ldexp(1.0, -24));
+    frexp(y, &e);
+    int E = e - 1; /* y in [2^E, 2^(E+1)) */
+    uint16_t frac = (uint16_t)((y / ldexp(1.0, E) - 1.0) * 1024.0);
+    return sign | (uint16_t)((E + 15) << 10) | frac;
+}
+
+double oracle_from_fp16(uint16_t h)
+{
+    int s = (h >> 15) & 1, E = (h >> 10) & 0x1F, f = h & 0x3FF;
+    double v;
+    if (E == 0) v = ldexp((double)f, -24);
+    else if (E == 31) v = f ? NAN : INFINITY;
+    else v = ldexp(1.0 + f / 1024.0, E - 15);
+    return s ? -v : v;
+}
+
+#define REAL float
+#define SFX(name) name##_f32
+#include "stepq_oracle_core.inc"
+#undef REAL
+#undef SFX
+
+#define REAL double
+#define SFX(name) name##_f64
+#include "stepq_oracle_core.inc"
+#undef REAL
+#undef SFX
+
+double oracle_column_error_f64(int dk, int dv, int j, const double *S, const uint8_t *bits,
+                               const float *rho, const double *r, double cj,
+                               const int32_t *code)
+{
+    double e = 0.0;
+    for (int i = 0; i < dk; i++) {
+        if (bits[i] == ORACLE_PIVOT_BITS) continue;
+        double d = S[i * dv + j] - r[i] * cj * (double)code[i * dv + j];
+        e += (double)rho[i] * d * d;
+    }
+    return e;
+}
+
+/* ---- the packed byte format ---------------------------------------------- */
+
+static size_t row_bytes(int dv, int b) { return (size_t)dv * (size_t)b / 8; }
+
+size_t oracle_item_bytes(int dk, int dv, const uint8_t *bits)
+{
+    size_t n = 4 * (size_t)dk + 4 * (size_t)dv;
+    for (int i = 0; i < dk; i++) n += row_bytes(dv, bits[i]);
+    return n;
+}
+
+static void put_f32(uint8_t *dst, float x) { memcpy(dst, &x, 4); } /* host is little-endian */
+static float get_f32(const uint8_t *src) { float x; memcpy(&x, src, 4); return x; }
+
+void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                      const int32_t *code, const float *piv, uint8_t *item)
+{
+    uint8_t *p = item;
+    for (int i = 0; i < dk; i++, p += 4) put_f32(p, r[i]);
+    for (int j = 0; j < dv; j++, p += 4) put_f32(p, c[j]);
+    for (int i = 0; i < dk; i++) {
+        int b = bits[i];
+        size_t nb = row_bytes(dv, b);
+        memset(p, 0, nb);
+        if (b == ORACLE_PIVOT_BITS) {
+            for (int j = 0; j < dv; j++) {
+                uint16_t h = oracle_to_fp16((double)piv[i * dv + j]);
+                p[2 * j] = (uint8_t)(h & 0xFF);
+                p[2 * j + 1] = (uint8_t)(h >> 8);
+            }
+        } else {
+            /* offset-binary code, bit t of column j at stream bit j*b + t */
+            for (int j = 0; j < dv; j++) {
+                uint32_t u = (uint32_t)(code[i * dv + j] + (1 << (b - 1)));
+                for (int t = 0; t < b; t++) {
+                    size_t bit = (size_t)j * b + t;
+                    p[bit / 8] |= (uint8_t)(((u >> t) & 1u) << (bit % 8));
+                }
+            }
+        }
+        p += nb;
+    }
+}
+
+void oracle_unpack_item(int dk, int dv, const uint8_t *bits, const uint8_t *item,
+                        float *r, float *c, int32_t *code, float *piv)
+{
+    const uint8_t *p = item;
+    for (int i = 0; i < dk; i++, p += 4) r[i] = get_f32(p);
+    for (int j = 0; j < dv; j++, p += 4) c[j] = get_f32(p);
+    for (int i = 0; i < dk; i++) {
+        int b = bits[i];
+        if (b == ORACLE_PIVOT_BITS) {
+            for (int j = 0; j < dv; j++) {
+                uint16_t h = (uint16_t)(p[2 * j] | (p[2 * j + 1] << 8));
+                piv[i * dv + j] = (float)oracle_from_fp16(h);
+                code[i * dv + j] = 0;
+            }
+        } else {
+            for (int j = 0; j < dv; j++) {
+                uint32_t u = 0;
+                for (int t = 0; t < b; t++) {
+                    size_t bit = (size_t)j * b + t;
+                    u |= (uint32_t)((p[bit / 8] >> (bit % 8)) & 1u) << t;
+                }
+                code[i * dv + j] = (int32_t)u - (1 << (b - 1));
+                piv[i * dv + j] = 0;
+            }
+        }
+        p += row_bytes(dv, b);
+    }
+}
+
+/* ---- batched drivers ------------------------------------------------------ */
+
+size_t oracle_pool_bytes(int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits)
+{
+    size_t tot = 0;
+    for (int s = 0; s < n; s++) tot += oracle_item_bytes(dk, dv, bits + (size_t)slot_head[s] * dk);
+    return tot;
+}
+
+typedef struct {
+    float *r, *c, *piv, *S, *arow;
+    int32_t *code;
+} scratch_t;
+
+static scratch_t scratch_new(int dk, int dv)
+{
+    scratch_t w;
+    w.r = (float *)malloc(sizeof(float) * dk);
+    w.c = (float *)malloc(sizeof(float) * dv);
+    w.piv = (float *)malloc(sizeof(float) * (size_t)dk * dv);
+    w.S = (float *)malloc(sizeof(float) * (size_t)dk * dv);
+    w.arow = (float *)malloc(sizeof(float) * dk);
+    w.code = (int32_t *)malloc(sizeof(int32_t) * (size_t)dk * dv);
+    return w;
+}
+
+static void scratch_free(scratch_t *w)
+{
+    free(w->r); free(w->c); free(w->piv); free(w->S); free(w->arow); free(w->code);
+}
+
+void oracle_pack_pool(int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits,
+                      const float *rho, int ls_iters, const float *S, uint8_t *pool)
+{
+    scratch_t w = scratch_new(dk, dv);
+    size_t off = 0;
+    for (int s = 0; s < n; s++) {
+        const uint8_t *bh = bits + (size_t)slot_head[s] * dk;
+        const float *rh = rho + (size_t)slot_head[s] * dk;
+        oracle_fit_quantise_f32(dk, dv, S + (size_t)s * dk * dv, bh, rh, ls_iters,
+                                ORACLE_PIVOT_FP16, w.r, w.c, w.code, w.piv, NULL, NULL);
+        oracle_pack_item(dk, dv, bh, w.r, w.c, w.code, w.piv, pool + off);
+        off += oracle_item_bytes(dk, dv, bh);
+    }
+    scratch_free(&w);
+}
+
+void oracle_unpack_pool(int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits,
+                        const uint8_t *pool, float *S)
+{
+    scratch_t w = scratch_new(dk, dv);
+    size_t off = 0;
+    for (int s = 0; s < n; s++) {
+        const uint8_t *bh = bits + (size_t)slot_head[s] * dk;
+        oracle_unpack_item(dk, dv, bh, pool + off, w.r, w.c, w.code, w.piv);
+        oracle_dequant_f32(dk, dv, bh, w.r, w.c, w.code, w.piv, S + (size_t)s * dk * dv);
+        off += oracle_item_bytes(dk, dv, bh);
+    }
+    scratch_free(&w);
+}
+
+void oracle_decode_step(int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits,
+                        const float *rho, int ls_iters, int kda, uint8_t *pool,
+                        const float *q, const float *k, const float *v, const float *alpha,
+                        const float *beta, float *out, float *S_new, float *tpre, float *lsgap)
+{
+    scratch_t w = scratch_new(dk, dv);
+    size_t off = 0;
+    for (int s = 0; s < n; s++) {
+        const uint8_t *bh = bits + (size_t)slot_head[s] * dk;
+        const float *rh = rho + (size_t)slot_head[s] * dk;
+        /* reconstruct the stored state */
+        oracle_unpack_item(dk, dv, bh, pool + off, w.r, w.c, w.code, w.piv);
+        oracle_dequant_f32(dk, dv, bh, w.r, w.c, w.code, w.piv, w.S);
+        /* gated Delta update + readout */
+        for (int i = 0; i < dk; i++) w.arow[i] = kda ? alpha[(size_t)s * dk + i] : alpha[s];
+        oracle_update_f32(dk, dv, w.S, w.arow, q + (size_t)s * dk, k + (size_t)s * dk,
+                          v + (size_t)s * dv, beta[s], out + (size_t)s * dv);
+        if (S_new) memcpy(S_new + (size_t)s * dk * dv, w.S, sizeof(float) * (size_t)dk * dv);
+        /* refit, requantise, write back */
+        oracle_fit_quantise_f32(dk, dv, w.S, bh, rh, ls_iters, ORACLE_PIVOT_FP16, w.r, w.c,
+                                w.code, w.piv, tpre ? tpre + (size_t)s * dk * dv : NULL,
+                                lsgap ? lsgap + (size_t)s * dv : NULL);
+        oracle_pack_item(dk, dv, bh, w.r, w.c, w.code, w.piv, pool + off);
+        off += oracle_item_bytes(dk, dv, bh);
+    }
+    scratch_free(&w);
+}
+
+void oracle_fp32_step(int n, int dk, int dv, int kda, float *S, const float *q, const float *k,
+                      const float *v, const float *alpha, const float *beta, float *out)
+{
+    float *arow = (float *)malloc(sizeof(float) * dk);
+    for (int s = 0; s < n; s++) {
+        for (int i = 0; i < dk; i++) arow[i] = kda ? alpha[(size_t)s * dk + i] : alpha[s];
+        oracle_update_f32(dk, dv, S + (size_t)s * dk * dv, arow, q + (size_t)s * dk,
+                          k + (size_t)s * dk, v + (size_t)s * dv, beta[s], out + (size_t)s * dv);
+    }
+    free(arow);
+}
+
+void oracle_fp64_step(int n, int dk, int dv, int kda, double *S, const double *q,
+                      const double *k, const double *v, const double *alpha,
+                      const double *beta, double *out)
+{
+    double *arow = (double *)malloc(sizeof(double) * dk);
+    for (int s = 0; s < n; s++) {
+        for (int i = 0; i < dk; i++) arow[i] = kda ? alpha[(size_t)s * dk + i] : alpha[s];
+        oracle_update_f64(dk, dv, S + (size_t)s * dk * dv, arow, q + (size_t)s * dk,
+                          k + (size_t)s * dk, v + (size_t)s * dv, beta[s], out + (size_t)s * dv);
+    }
+    free(arow);
+}

@@ -1,0 +1,145 @@
+/*
+ * CPU oracle for the STEPQuant packed-state gated Delta-rule decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path (the
+ * CUDA library and its Python binding) never calls it, and it shares no code
+ * with that path.
+ *
+ * Plain, slow, scalar nested loops written for a reader who checks them against
+ * the pages describing the method:
+ *   [P1] ai-feeds.com summary (Chinese), sections "方法" (method) and
+ *        "核心洞察" (insights);
+ *   [P2] ai.info summary "STEPQuant: When and Where Errors Matter in
+ *        Delta-Rule Recurrent State Quantization", sections "Key
+ *        Contributions", "Main Findings", "Methodology in Plain English";
+ *   [P4] ai-papers.net article, section "STEPQuantの仕組み" (mechanism);
+ *   [P5] ai-trend.me review, sections "방법" (method), "핵심 용어" (terms).
+ *
+ * Each function is compiled twice: with REAL = float (suffix _f32, the
+ * parity mode: every stored or element-wise quantity is fp32, sums are
+ * accumulated in fp64 and rounded once) and REAL = double (suffix _f64, for
+ * the invariant checks).
+ *
+ * Readings taken where the pages are silent (each restated at its function):
+ *   - state S is [dk x dv], key rows i, value columns j;
+ *   - update: S' = diag(alpha) S; v_old = S'^T k; S = S' + beta k (v - v_old)^T;
+ *     readout o = S^T q on the updated, unquantised state;
+ *   - stored form S_ij = r_i * c_j * code_ij, symmetric codes in [-Q_b, Q_b],
+ *     Q_b = 2^(b-1) - 1, kept offset-binary (u = code + 2^(b-1), never 0);
+ *   - row scale r_i = rms_i * rho_i^(-1/2) / Q_(b_i) (rms_i -> 1 if zero);
+ *   - column scale: init c_j = max_i |S_ij| / (r_i Q_(b_i)) (-> 1 if zero),
+ *     then ls_iters rounds of impact-weighted least squares for fixed codes,
+ *     weights rho_i r_i^2 on p_ij = S_ij / r_i;
+ *   - rounding half-to-even everywhere; pivot rows stored as IEEE binary16.
+ */
+#ifndef STEPQ_ORACLE_H
+#define STEPQ_ORACLE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ORACLE_PIVOT_BITS 16
+
+/* pivot storage: fp16 (the method), or exact REAL (debug: lets an all-pivot
+ * state be compared bit for bit with an unquantised recursion) */
+#define ORACLE_PIVOT_FP16 0
+#define ORACLE_PIVOT_EXACT 1
+
+/* ---- type-generic per-item functions (one (request, head) state) ---------- */
+
+/* Fit row and column scales to S and quantise it.
+ *   S      [dk*dv] row-major state to store.
+ *   bits   [dk] row widths: 2..8, or 16 for an FP16 pivot row.
+ *   rho    [dk] row-impact weights (> 0).
+ * Outputs: r [dk] (0 on pivot rows), c [dv] (0 if every row is a pivot),
+ *   code [dk*dv] signed codes (0 on pivot rows), piv [dk*dv] pivot values
+ *   (0 on quantised rows).
+ * Optional diagnostics (NULL to skip): tpre [dk*dv] the final pre-round values
+ *   p_ij / c_j; lsgap [dv] per column, the smallest relative distance of a
+ *   least-squares rounding decision from a rounding boundary (+inf if none). */
+void oracle_fit_quantise_f32(int dk, int dv, const float *S, const uint8_t *bits,
+                             const float *rho, int ls_iters, int pivot_mode,
+                             float *r, float *c, int32_t *code, float *piv,
+                             float *tpre, float *lsgap);
+void oracle_fit_quantise_f64(int dk, int dv, const double *S, const uint8_t *bits,
+                             const float *rho, int ls_iters, int pivot_mode,
+                             double *r, double *c, int32_t *code, double *piv,
+                             double *tpre, double *lsgap);
+
+/* Quantise S with given scales (final step of the fit, exposed for checks). */
+void oracle_quantise_f32(int dk, int dv, const float *S, const uint8_t *bits, const float *r,
+                         const float *c, int32_t *code, float *tpre);
+void oracle_quantise_f64(int dk, int dv, const double *S, const uint8_t *bits, const double *r,
+                         const double *c, int32_t *code, double *tpre);
+
+/* Dequantise: S_ij = (r_i * c_j) * code_ij on quantised rows, piv_ij on pivot rows. */
+void oracle_dequant_f32(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                        const int32_t *code, const float *piv, float *S);
+void oracle_dequant_f64(int dk, int dv, const uint8_t *bits, const double *r, const double *c,
+                        const int32_t *code, const double *piv, double *S);
+
+/* Gated Delta-rule update in place, then readout:
+ *   S'_ij = alpha_i S_ij; v_old_j = sum_i S'_ij k_i;
+ *   S_ij = S'_ij + (beta k_i)(v_j - v_old_j); o_j = sum_i S_ij q_i.
+ * alpha [dk] (Gated-DeltaNet passes one value repeated over the rows). */
+void oracle_update_f32(int dk, int dv, float *S, const float *alpha, const float *q,
+                       const float *k, const float *v, float beta, float *o);
+void oracle_update_f64(int dk, int dv, double *S, const double *alpha, const double *q,
+                       const double *k, const double *v, double beta, double *o);
+
+/* Weighted reconstruction error of one column j under scales r, c and codes:
+ * sum over quantised rows of rho_i (S_ij - r_i c_j code_ij)^2. */
+double oracle_column_error_f64(int dk, int dv, int j, const double *S, const uint8_t *bits,
+                               const float *rho, const double *r, double cj,
+                               const int32_t *code);
+
+/* ---- IEEE binary16 (round to nearest, ties to even) ----------------------- */
+uint16_t oracle_to_fp16(double x);
+double oracle_from_fp16(uint16_t h);
+
+/* ---- packed byte format (the pool) ---------------------------------------- *
+ * item = r[dk] fp32 | c[dv] fp32 | row 0 | ... | row dk-1
+ * quantised row i: dv * b_i / 8 bytes, a little-endian bit stream with the
+ *   offset-binary code of column j in bits [j b_i, (j+1) b_i);
+ * pivot row: dv binary16 values, little-endian.
+ * Requires dv * b_i % 8 == 0 for every row. */
+size_t oracle_item_bytes(int dk, int dv, const uint8_t *bits);
+void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                      const int32_t *code, const float *piv, uint8_t *item);
+void oracle_unpack_item(int dk, int dv, const uint8_t *bits, const uint8_t *item,
+                        float *r, float *c, int32_t *code, float *piv);
+
+/* ---- batched drivers over "slots" (a slot = one (request, head) state) ---- *
+ * slot_head[s] gives the head of slot s; bits/rho are per-head tables
+ * [H*dk].  The pool holds the slots' items back to back in slot order.
+ * alpha is [n*dk] when kda != 0, else [n]. */
+size_t oracle_pool_bytes(int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits);
+void oracle_pack_pool(int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits,
+                      const float *rho, int ls_iters, const float *S, uint8_t *pool);
+void oracle_unpack_pool(int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits,
+                        const uint8_t *pool, float *S);
+/* One decode step over every slot: dequantise, update, read out, refit,
+ * requantise, repack.  Optional diagnostics as in oracle_fit_quantise_f32
+ * (tpre [n*dk*dv], lsgap [n*dv]); S_new [n*dk*dv] receives the updated
+ * unquantised state. */
+void oracle_decode_step(int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits,
+                        const float *rho, int ls_iters, int kda, uint8_t *pool,
+                        const float *q, const float *k, const float *v, const float *alpha,
+                        const float *beta, float *out, float *S_new, float *tpre, float *lsgap);
+/* Unquantised fp32 recursion over slots (the fp32-state baseline). */
+void oracle_fp32_step(int n, int dk, int dv, int kda, float *S, const float *q, const float *k,
+                      const float *v, const float *alpha, const float *beta, float *out);
+/* Unquantised fp64 recursion over slots. */
+void oracle_fp64_step(int n, int dk, int dv, int kda, double *S, const double *q,
+                      const double *k, const double *v, const double *alpha,
+                      const double *beta, double *out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
