@@ -1,0 +1,353 @@
+"""Benchmark of the packed-state gated Delta-rule decode step on B200.
+
+One step = one fused decode step (reconstruct, gated Delta update, readout,
+scale refit, requantise, pack) over every (request, head) item of the
+serving-scale Gated-DeltaNet workload: batch 512, 48 heads, dk = dv = 128,
+4-bit nominal average (widths {3, 4, 6}, 1 % FP16 pivot heads), one
+least-squares round.  Inputs are seeded synthetic tensors (no model or
+dataset is involved); they are resident in HBM when the timed region starts.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  For N > 1 run under torch.distributed.run:
+every rank holds its own full workload (requests are independent; no
+collective on the data path), so scaling is weak and value is the sum over
+ranks of items processed divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_recurrent_state_sm_b200 import workload as W  # noqa: E402
+
+METRIC = "packed state updates/s (batch*head*step); achieved HBM GB/s vs B200 peak"
+UNIT = "state updates/s"
+CONFIG_INDEX = 3
+RING = 8  # distinct pre-generated input steps cycled through (8 x 38 MB > L2)
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=300)
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--config", type=int, default=CONFIG_INDEX)
+    return p.parse_args()
+
+
+def workload_name(cfg):
+    return (f"{cfg.name}: {'Gated-DeltaNet' if cfg.variant == W.GDN else 'KDA'} decode, batch {cfg.batch}, "
+            f"{cfg.heads} heads, dk=dv={cfg.dk}, widths {list(cfg.bits_choices)} avg {cfg.avg_bits:g} bits "
+            f"incl. {cfg.pivot_frac:.0%} FP16 pivots, ls_iters={cfg.ls_iters}")
+
+
+def algorithmic_bytes(cfg, bits):
+    """Bytes one decode step must move: packed state in and out, q, k, v, alpha,
+    beta in, readout out."""
+    state = int(W.head_item_bytes(bits, cfg.dv).sum()) * cfg.batch
+    n = cfg.items
+    alpha = n * (cfg.dk if cfg.variant == W.KDA else 1) * 4
+    inputs = n * (2 * cfg.dk + cfg.dv) * 4 + alpha + n * 4
+    out = n * cfg.dv * 4
+    return 2 * state + inputs + out, state
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "quantized_recurrent_state_sm_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(cfg_name):
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
+    valid only if the kernel sources are unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(cfg_name)
+    if not ent or ent.get("kernel_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock samples during the timed region (every 200 ms)."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1])); mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_rate(cfg, seconds):
+    """The CPU oracle as it stands (single thread) on a bounded sample of the
+    workload: the parity requests {0, 1, B/2, B-1} x all heads, consecutive
+    steps until `seconds` of CPU time have been spent.  Returns items/s."""
+    import oracle
+    req = W.parity_requests(cfg)
+    H = cfg.heads
+    slots = (np.asarray(req)[:, None] * H + np.arange(H)[None, :]).reshape(-1)
+    bits, rho = W.bit_table(cfg), W.rho(cfg)
+    kda = cfg.variant == W.KDA
+    pool = oracle.SlotPool(slots % H, bits, rho, ls_iters=cfg.ls_iters, kda=kda)
+    rng = np.random.default_rng(0)
+    pool.pack((rng.standard_normal((len(slots), 128, 128)) * 0.1).astype(np.float32))
+    n = len(slots)
+    items = 0
+    busy = 0.0
+    t = 0
+    while busy < seconds:
+        x = W.step_inputs(cfg, t, req)
+        args = (x["q"].reshape(n, -1), x["k"].reshape(n, -1), x["v"].reshape(n, -1),
+                x["alpha"].reshape(n, -1) if kda else x["alpha"].reshape(-1), x["beta"].reshape(-1))
+        t0 = time.perf_counter()
+        pool.step(*args)
+        busy += time.perf_counter() - t0
+        items += n
+        t += 1
+    return items / busy, {"kind": "oracle", "cores": 1,
+                          "sample": f"{n} items (requests {req} x {H} heads) x {t} steps of {cfg.name}, "
+                                    f"single-threaded C oracle, {busy:.1f} s"}
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rate, meta = cpu_oracle_rate(cfg, max(1.0, args.cpu_seconds))
+    per_step = args.steps * cfg.items / rate
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": cfg.items / rate * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": {"workload": workload_name(cfg)},
+        "cpu_baseline": dict(value=rate, unit=UNIT, **meta),
+        "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": f"the CPU oracle on a bounded sample; a full step would take {per_step / args.steps:.1f} s",
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    cfg = W.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from quantized_recurrent_state_sm_b200 import stepq
+
+    bits, rho = W.bit_table(cfg), W.rho(cfg)
+    B, H = cfg.batch, cfg.heads
+    pool = stepq.PackedStatePool(cfg.variant, B, H, bits, rho, cfg.ls_iters)
+    # input ring: RING pre-generated steps resident in HBM
+    ring = []
+    for t in range(RING):
+        x = W.step_inputs(cfg, t + 1000 * rank)
+        ring.append({k: torch.from_numpy(v).cuda() for k, v in x.items()})
+    out = torch.empty((B, H, cfg.dv), device="cuda")
+    # initial state: unquantised warm-up on the GPU (fp32 baseline kernel), then pack
+    S = torch.zeros((B, H, cfg.dk, cfg.dv), device="cuda")
+    for t in range(-cfg.warmup, 0):
+        d = ring[t % RING]
+        stepq.fp32_step(cfg.variant, S, d["q"], d["k"], d["v"], d["alpha"], d["beta"], out)
+    pool.pack(S)
+    torch.cuda.synchronize()
+
+    def step(i):
+        d = ring[i % RING]
+        pool.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"], out)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * cfg.items * args.steps / (ms * 1e-3)
+
+    # fp32-state baseline kernel on the same inputs (the packed/fp32 time ratio)
+    for i in range(3):
+        d = ring[i % RING]
+        stepq.fp32_step(cfg.variant, S, d["q"], d["k"], d["v"], d["alpha"], d["beta"], out)
+    torch.cuda.synchronize()
+    nf = max(10, args.steps // 20)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(nf):
+        d = ring[i % RING]
+        stepq.fp32_step(cfg.variant, S, d["q"], d["k"], d["v"], d["alpha"], d["beta"], out)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    fp32_ms = f0.elapsed_time(f1) / nf
+    del S
+
+    # end to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, the decode step, D2H of the readout, every step
+    host = []
+    for t in range(RING):
+        x = W.step_inputs(cfg, t + 1000 * rank)
+        host.append({k: torch.from_numpy(v).pin_memory() for k, v in x.items()})
+    dev_in = {k: torch.empty_like(v, device="cuda") for k, v in host[0].items()}
+    out_host = torch.empty((B, H, cfg.dv), dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * 4 for v in host[0].values())
+    d2h = out_host.numel() * 4
+
+    def e2e_step(i):
+        hx = host[i % RING]
+        for k in dev_in:
+            dev_in[k].copy_(hx[k], non_blocking=True)
+        pool.decode_step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"], dev_in["beta"], out)
+        out_host.copy_(out, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for i in range(args.e2e_steps):
+        e2e_step(i)
+    g1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = g0.elapsed_time(g1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * cfg.items * args.e2e_steps / (e2e_ms * 1e-3)
+
+    if rank == 0:
+        peaks, src = measured_peaks()
+        alg, state = algorithmic_bytes(cfg, bits)
+        achieved = alg / (ms_per_step * 1e-3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": workload_name(cfg), "batch": B, "heads": H, "dk": cfg.dk, "dv": cfg.dv,
+                       "packed_state_bytes": state, "per_gpu_items": cfg.items,
+                       "l2": "inputs larger than L2 (packed pool %.0f MB + %d-step input ring %.0f MB, no flush)"
+                             % (state / 1e6, RING, RING * h2d / 1e6)},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": recorded_traffic(cfg.name),
+                         "algorithmic_bytes_per_launch": alg, "peak_source": src,
+                         "kernel": "stepq fused decode step (k_item<0>)"},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": args.e2e_steps},
+            "gpu_launches": args.steps,
+            "fp32_state": {"ms_per_step": fp32_ms, "packed_speedup": fp32_ms / ms_per_step,
+                           "state_bytes": cfg.items * cfg.dk * cfg.dv * 4},
+            "clocks": clocks.summary(),
+        }
+        if not args.no_cpu_baseline:
+            rate, meta = cpu_oracle_rate(cfg, args.cpu_seconds)
+            line["cpu_baseline"] = dict(value=rate, unit=UNIT, **meta)
+        print(json.dumps(line), flush=True)
+    pool.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,177 @@
+/*
+ * stepq.h -- C ABI of the packed-state gated Delta-rule decode step (STEPQuant).
+ *
+ * The method (pages: ai.info summary "STEPQuant: When and Where Errors Matter
+ * in Delta-Rule Recurrent State Quantization", sections "Key Contributions" and
+ * "Methodology in Plain English"; ai-papers.net article, section
+ * "STEPQuantの仕組み"; ai-trend.me review, sections "방법" and "핵심 용어"):
+ * every concurrent request keeps one recurrent state S [dk x dv] per head.  The
+ * state is stored packed -- key-row scale x value-column scale x integer code,
+ * with a bit width per unit (a head for Gated-DeltaNet, a key row for KDA) and
+ * a few FP16 "pivot" units -- and one decode step reconstructs it, applies the
+ * gated Delta update, reads out o = S^T q, refits the scales and writes the
+ * packed state back.
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" are CUDA device pointers on the current device;
+ *     "host" pointers are read during the call only.  All device tensors are
+ *     contiguous fp32, 16-byte aligned, row-major in the shapes given.
+ *   - The caller owns every buffer passed in.  The library allocates no device
+ *     memory and never frees a caller buffer.
+ *   - Kernels are enqueued on the pool's stream (or the stream argument) and
+ *     the call returns without synchronising; results are ready when that
+ *     stream reaches the point of the call.
+ *   - Arguments are validated on the host before any launch; an invalid call
+ *     returns an error status and enqueues nothing.  A failed launch returns
+ *     STEPQ_ERR_CUDA.  No call throws or aborts.  stepq_last_error() returns a
+ *     one-line description of the last failure on the calling thread.
+ *   - Only dk = dv = 128 is implemented (other sizes: STEPQ_ERR_UNSUPPORTED).
+ */
+#ifndef STEPQ_H
+#define STEPQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols of the shared library (built with hidden default visibility). */
+#if defined(__GNUC__)
+#define STEPQ_API __attribute__((visibility("default")))
+#else
+#define STEPQ_API
+#endif
+
+typedef enum {
+    STEPQ_OK = 0,
+    STEPQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad table entry, misalignment */
+    STEPQ_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement */
+    STEPQ_ERR_CUDA = 3,        /* a CUDA call or kernel launch failed */
+    STEPQ_ERR_STATE = 4        /* the pool handle is not usable (e.g. destroyed) */
+} stepq_status;
+
+/* Gate kinds.  Gated-DeltaNet: one retention gate per (request, head), and the
+ * unit of bit allocation is the head.  KDA (Kimi Delta Attention): one gate per
+ * key row, and the unit of bit allocation is the key row (ai.info summary,
+ * "Future Directions"; ai-papers.net, "STEPQuantの仕組み"). */
+#define STEPQ_GDN 0
+#define STEPQ_KDA 1
+
+/* Row width meaning "FP16 pivot": the row is stored as dv binary16 values and
+ * takes no part in the scale fit (ai.info summary, "Key Contributions"). */
+#define STEPQ_PIVOT_BITS 16
+
+/* Largest batch * heads a pool may hold. */
+#define STEPQ_MAX_ITEMS (1 << 24)
+
+typedef struct {
+    int variant;  /* STEPQ_GDN or STEPQ_KDA */
+    int batch;    /* requests, >= 0 (0 gives an empty pool; every call is a no-op) */
+    int heads;    /* heads per request, >= 1 */
+    int dk, dv;   /* key and value dimension; 128 and 128 */
+    int ls_iters; /* least-squares rounds of the column-scale fit, 0..8 (1 is the default) */
+    /* host [heads * dk]: width of key row i of head h, in bits: 2..8, or 16 for
+     * an FP16 pivot row.  Gated-DeltaNet requires one width per head. */
+    const uint8_t *bits;
+    /* host [heads * dk]: calibrated row-impact weight of key row i of head h,
+     * finite and > 0 (pivot rows: ignored).  Fixed for all requests. */
+    const float *rho;
+} stepq_desc;
+
+typedef struct stepq_pool stepq_pool; /* opaque handle */
+
+/*
+ * Device bytes the caller must provide for a pool: the packed states of all
+ * batch * heads items followed by the library's small per-head tables.
+ * Returns 0 if the descriptor is invalid or unsupported.
+ *
+ * Packed state layout (offsets in bytes from the start of the buffer):
+ *   item (b, h) starts at b * R + P_h, R = sum over heads of the item sizes,
+ *   P_h = sum of the item sizes of heads 0..h-1;
+ *   item = r[dk] fp32 | c[dv] fp32 | row 0 | ... | row dk-1, where a row of
+ *   width b_i holds dv * b_i / 8 bytes: a little-endian bit stream with the
+ *   offset-binary code (code + 2^(b_i - 1), in 1 .. 2^b_i - 1) of value column
+ *   j in bits [j * b_i, (j + 1) * b_i); a pivot row holds dv binary16 values.
+ *   The stored element is r_i * c_j * code_ij (ai-papers.net,
+ *   "STEPQuantの仕組み"); pivot rows keep r_i = 0.
+ */
+STEPQ_API size_t stepq_pool_bytes(const stepq_desc *desc);
+
+/* Bytes of the packed states alone (the prefix of the pool buffer that holds
+ * the items); 0 if the descriptor is invalid. */
+STEPQ_API size_t stepq_state_bytes(const stepq_desc *desc);
+
+/*
+ * Create a pool over a caller-owned device buffer of at least
+ * stepq_pool_bytes(desc) bytes (16-byte aligned).  Copies the descriptor and
+ * the host tables, writes the derived per-head tables into the tail of the
+ * buffer, and synchronises the given stream once before returning (creation is
+ * not on the decode path).  The packed states are left uninitialised: call
+ * stepq_pack before the first decode step.  cuda_stream is a cudaStream_t
+ * (NULL = the legacy default stream); it can be changed with
+ * stepq_pool_set_stream.  On success *out receives the handle.
+ */
+STEPQ_API stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t bytes,
+                               void *cuda_stream, stepq_pool **out);
+
+/* Release the handle (host memory only; the device buffer stays the caller's).
+ * Passing NULL returns STEPQ_ERR_INVALID_ARG. */
+STEPQ_API stepq_status stepq_pool_destroy(stepq_pool *pool);
+
+/* Stream on which the pool's later calls enqueue their kernels. */
+STEPQ_API stepq_status stepq_pool_set_stream(stepq_pool *pool, void *cuda_stream);
+
+/*
+ * Fit and quantise full-precision states into the pool (the initial state of
+ * every item, or a restore from a checkpoint).  S: device fp32
+ * [batch, heads, dk, dv].  Per item: row scales from the row's root-mean-square
+ * magnitude and impact weight, column scales by least squares, codes by
+ * round-half-even with clamping -- the same fit the decode step performs after
+ * its update (ai.info summary, "Methodology in Plain English").
+ */
+STEPQ_API stepq_status stepq_pack(stepq_pool *pool, const float *S);
+
+/* Dequantise every item into S_out: device fp32 [batch, heads, dk, dv],
+ * S_ij = (r_i * c_j) * code_ij, or the stored binary16 value on pivot rows. */
+STEPQ_API stepq_status stepq_unpack(stepq_pool *pool, float *S_out);
+
+/*
+ * One decode step for every (request, head) item of the pool, in one fused
+ * kernel: reconstruct the state from the packed pool, apply the gated Delta
+ * update, read out, refit the scales, requantise and write the packed state
+ * back in place (ai.info summary, "Key Contributions" and "Methodology in
+ * Plain English"; ai-trend.me, "핵심 용어: Gated Delta Rule").
+ *   S'   = diag(alpha) S      (one alpha per item for GDN, per key row for KDA)
+ *   vold = S'^T k
+ *   S    = S' + beta k (v - vold)^T
+ *   out  = S^T q              (from the updated, unquantised state)
+ * Inputs (device fp32): q, k [batch, heads, dk]; v [batch, heads, dv];
+ * alpha [batch, heads] (GDN) or [batch, heads, dk] (KDA), each in (0, 1];
+ * beta [batch, heads].  Output: out [batch, heads, dv] (device fp32; must not
+ * alias an input).  Values are not range-checked on the device.
+ */
+STEPQ_API stepq_status stepq_decode_step(stepq_pool *pool, const float *q, const float *k, const float *v,
+                               const float *alpha, const float *beta, float *out);
+
+/*
+ * The same update and readout on an unquantised fp32 state, in place: the
+ * full-precision baseline the packed step is measured against.  S: device fp32
+ * [batch, heads, dk, dv]; other tensors as in stepq_decode_step.  Uses only
+ * desc->variant, batch, heads, dk, dv.  cuda_stream: cudaStream_t or NULL.
+ */
+STEPQ_API stepq_status stepq_fp32_step(const stepq_desc *desc, float *S, const float *q, const float *k,
+                             const float *v, const float *alpha, const float *beta, float *out,
+                             void *cuda_stream);
+
+/* Human-readable name of a status; never NULL. */
+STEPQ_API const char *stepq_status_string(stepq_status s);
+
+/* One-line description of the last failure on this thread ("" if none). */
+STEPQ_API const char *stepq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* STEPQ_H */

@@ -1,0 +1,94 @@
+"""The C-ABI library on the host: it loads, exports every declared symbol, and
+validates descriptors and handles without touching a GPU."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+from quantized_recurrent_state_sm_b200 import workload as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def S():
+    from quantized_recurrent_state_sm_b200 import build
+    build.build()
+    from quantized_recurrent_state_sm_b200 import stepq
+    return stepq
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"STEPQ_API\s+[\w\s\*]+?\b(stepq_\w+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(S):
+    names = declared_symbols()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(S.lib, n), n
+    assert set(S.EXPORTS) <= names
+
+
+def test_pool_bytes_matches_layout(S):
+    for ci in range(5):
+        cfg = W.CONFIGS[ci]
+        bits, rho = W.bit_table(cfg), W.rho(cfg)
+        _, total = W.item_offsets(bits, 128, cfg.batch)
+        d, keep = S.make_desc(cfg.variant, cfg.batch, cfg.heads, bits, rho)
+        assert S.lib.stepq_state_bytes(C.byref(d)) == total
+        assert S.lib.stepq_pool_bytes(C.byref(d)) >= total
+
+
+def test_descriptor_validation(S):
+    cfg = W.CONFIGS[1]
+    bits, rho = W.bit_table(cfg), W.rho(cfg)
+
+    def nbytes(**kw):
+        b = kw.pop("bits", bits); r = kw.pop("rho", rho)
+        d, keep = S.make_desc(cfg.variant, cfg.batch, cfg.heads, b, r)
+        for k, v in kw.items():
+            setattr(d, k, v)
+        n = S.lib.stepq_pool_bytes(C.byref(d))
+        return n, S.lib.stepq_last_error().decode()
+
+    assert nbytes()[0] > 0
+    assert nbytes(variant=7) == (0, nbytes(variant=7)[1]) and "variant" in nbytes(variant=7)[1]
+    assert nbytes(dk=64)[0] == 0 and "128" in nbytes(dk=64)[1]
+    assert nbytes(batch=-1)[0] == 0
+    assert nbytes(heads=0)[0] == 0
+    assert nbytes(ls_iters=9)[0] == 0
+    bad = bits.copy(); bad[0, 5] = 9
+    assert nbytes(bits=bad)[0] == 0
+    mixed = bits.copy(); mixed[0, 5] = 3 if mixed[0, 0] != 3 else 4
+    n, msg = nbytes(bits=mixed)
+    assert n == 0 and "one width per head" in msg
+    r2 = rho.copy(); r2[1, 1] = 0.0
+    assert nbytes(rho=r2)[0] == 0
+    r3 = rho.copy(); r3[1, 1] = np.nan
+    assert nbytes(rho=r3)[0] == 0
+    d, keep = S.make_desc(cfg.variant, cfg.batch, cfg.heads, bits, rho)
+    d.bits = None
+    assert S.lib.stepq_pool_bytes(C.byref(d)) == 0
+    assert S.lib.stepq_pool_bytes(None) == 0
+
+
+def test_null_and_dead_handles(S):
+    assert S.lib.stepq_pool_destroy(None) == S.ERR_INVALID_ARG
+    assert S.lib.stepq_decode_step(None, None, None, None, None, None, None) == S.ERR_INVALID_ARG
+    bogus = C.c_void_p(0x1000)
+    assert S.lib.stepq_pack(bogus, None) == S.ERR_STATE
+    out = C.c_void_p()
+    cfg = W.CONFIGS[0]
+    d, keep = S.make_desc(cfg.variant, cfg.batch, cfg.heads, W.bit_table(cfg), W.rho(cfg))
+    assert S.lib.stepq_pool_create(C.byref(d), None, 10 ** 9, None, C.byref(out)) == S.ERR_INVALID_ARG
+    assert S.lib.stepq_pool_create(C.byref(d), C.c_void_p(16), 16, None, C.byref(out)) == S.ERR_INVALID_ARG
+    assert S.lib.stepq_pool_create(C.byref(d), None, 0, None, None) == S.ERR_INVALID_ARG
+    assert S.lib.stepq_status_string(3) == b"STEPQ_ERR_CUDA"

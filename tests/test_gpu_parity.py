@@ -1,0 +1,286 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Every input is seeded and synthetic (quantized_recurrent_state_sm_b200.workload).
+The GPU always runs the whole batch; for the large configurations the oracle
+follows requests {0, 1, B/2, B-1} x all heads, whose packed bytes are copied
+into the GPU pool before each lockstep step (items are independent, so this is
+exact).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_recurrent_state_sm_b200 import workload as W
+from tests.parity import PoolComparison, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from quantized_recurrent_state_sm_b200 import stepq
+else:  # pragma: no cover
+    stepq = None
+
+
+def to_dev(x):
+    return {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in x.items()}
+
+
+class Setup:
+    """A GPU pool and the oracle's pool over the compared slots."""
+
+    def __init__(self, cfg, requests=None, bits=None, rho=None):
+        self.cfg = cfg
+        self.bits = W.bit_table(cfg) if bits is None else bits
+        self.rho = W.rho(cfg) if rho is None else rho
+        self.req = np.arange(cfg.batch) if requests is None else np.asarray(requests)
+        H = cfg.heads
+        self.slots = (self.req[:, None] * H + np.arange(H)[None, :]).reshape(-1)
+        self.kda = cfg.variant == W.KDA
+        self.gpu = stepq.PackedStatePool(cfg.variant, cfg.batch, H, self.bits, self.rho, cfg.ls_iters)
+        self.ref = oracle.SlotPool(self.slots % H, self.bits, self.rho, ls_iters=cfg.ls_iters, kda=self.kda)
+        offs, total = W.item_offsets(self.bits, 128, cfg.batch)
+        assert total == self.gpu.state_nbytes
+        self.gpu_off = offs.reshape(-1)[self.slots]
+
+    def slot_inputs(self, x):
+        n = len(self.slots)
+        sub = {k: v[self.req] for k, v in x.items()}
+        return (sub["q"].reshape(n, -1), sub["k"].reshape(n, -1), sub["v"].reshape(n, -1),
+                sub["alpha"].reshape(n, -1) if self.kda else sub["alpha"].reshape(-1),
+                sub["beta"].reshape(-1))
+
+    def push_oracle_bytes(self):
+        """Overwrite the compared GPU items with the oracle's bytes."""
+        st = self.gpu.state
+        for s in range(len(self.slots)):
+            o, n = int(self.gpu_off[s]), int(self.ref.sizes[s])
+            st[o:o + n].copy_(torch.from_numpy(self.ref.item(s).copy()))
+
+    def gpu_item(self, host_state, s):
+        o, n = int(self.gpu_off[s]), int(self.ref.sizes[s])
+        return host_state[o:o + n]
+
+    def head(self, s):
+        return self.bits[self.slots[s] % self.cfg.heads]
+
+
+def lockstep(setup, steps, t0=0, full_inputs=True):
+    cfg = setup.cfg
+    cmp = PoolComparison()
+    S0 = oracle.initial_state(cfg, setup.req)
+    setup.ref.pack(S0.reshape(-1, 128, 128))
+    worst = 0.0
+    for t in range(t0, t0 + steps):
+        setup.push_oracle_bytes()
+        x = W.step_inputs(cfg, t) if full_inputs else None
+        d = to_dev(x)
+        out = setup.gpu.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+        torch.cuda.synchronize()
+        o_ref, dg = setup.ref.step(*setup.slot_inputs(x), diag=True)
+        o = out.cpu().numpy()[setup.req].reshape(len(setup.slots), -1)
+        e = rel_l2(o, o_ref)
+        worst = max(worst, e)
+        assert e <= 1e-4, f"step {t}: readout rel L2 {e:.3e}"
+        host = setup.gpu.state.cpu().numpy()
+        for s in range(len(setup.slots)):
+            cmp.item(setup.head(s), setup.gpu_item(host, s), setup.ref.item(s), dg["tpre"][s],
+                     dg["lsgap"][s], dg["S_new"][s], where=f"step {t} slot {s}")
+    cmp.check_fraction()
+    return cmp, worst
+
+
+def test_unpack_is_exact():
+    cfg = W.with_overrides(W.CONFIGS[1], batch=3)
+    su = Setup(cfg)
+    S0 = oracle.initial_state(cfg)
+    su.ref.pack(S0.reshape(-1, 128, 128))
+    su.push_oracle_bytes()
+    got = su.gpu.unpack().cpu().numpy().reshape(-1, 128, 128)
+    np.testing.assert_array_equal(got, su.ref.unpack())
+
+
+@pytest.mark.parametrize("ci", [0, 1, 2, 4])
+def test_pack_matches_oracle(ci):
+    cfg = W.with_overrides(W.CONFIGS[ci], batch=min(W.CONFIGS[ci].batch, 4))
+    su = Setup(cfg)
+    S0 = oracle.initial_state(cfg)
+    su.gpu.pack(torch.from_numpy(S0).cuda())
+    torch.cuda.synchronize()
+    host = su.gpu.state.cpu().numpy()
+    cmp = PoolComparison()
+    for s, flat in enumerate(S0.reshape(-1, 128, 128)):
+        bh = su.head(s)
+        rh = su.rho[su.slots[s] % cfg.heads]
+        fit = oracle.fit_quantise(flat, bh, rh, cfg.ls_iters, diag=True)
+        want = oracle.pack_item(bh, fit["r"], fit["c"], fit["code"], fit["piv"])
+        cmp.item(bh, su.gpu_item(host, s), want, fit["tpre"], fit["lsgap"], flat, where=f"slot {s}")
+    cmp.check_fraction()
+
+
+def test_lockstep_config0_full():
+    cmp, worst = lockstep(Setup(W.CONFIGS[0]), steps=16)
+    print(f"config 0: {cmp.diff}/{cmp.codes} codes differ, worst readout {worst:.2e}")
+
+
+@pytest.mark.parametrize("ci,steps", [(1, 3), (2, 3), (4, 2)])
+def test_lockstep_subsampled_full_batch(ci, steps):
+    cfg = W.CONFIGS[ci]
+    cmp, worst = lockstep(Setup(cfg, W.parity_requests(cfg)), steps=steps, t0=100)
+    print(f"config {ci}: {cmp.diff}/{cmp.codes} codes differ, worst readout {worst:.2e}")
+
+
+def test_lockstep_config3_full_size_sampled():
+    """The serving-scale launch (512 x 48 items) on the oracle's sampled requests."""
+    cfg = W.CONFIGS[3]
+    cmp, worst = lockstep(Setup(cfg, W.parity_requests(cfg)), steps=2, t0=500)
+    print(f"config 3: {cmp.diff}/{cmp.codes} codes differ, worst readout {worst:.2e}")
+
+
+def test_every_width_and_pivot_rows_kda():
+    cfg = W.with_overrides(W.CONFIGS[2], batch=3, heads=2)
+    r = np.random.default_rng(0)
+    bits = r.choice([2, 3, 4, 5, 6, 7, 8, 16], size=(2, 128)).astype(np.uint8)
+    lockstep(Setup(cfg, bits=bits), steps=4)
+
+
+def perturbed_copy(ref, bits, heads, seed):
+    """The oracle pool with one code of every item moved by one step: a rollout
+    whose rounding noise is decorrelated from the original in every item."""
+    P = oracle.SlotPool(ref.slot_head, ref.bits, ref.rho, ls_iters=ref.ls_iters, kda=ref.kda)
+    P.pool[:] = ref.pool
+    r = np.random.default_rng(seed)
+    for s in range(P.n):
+        bh = bits[ref.slot_head[s]]
+        it = oracle.unpack_item(bh, P.item(s), 128, 128)
+        rows = np.flatnonzero(bh != 16)
+        if rows.size == 0:
+            continue
+        i, j = int(r.choice(rows)), int(r.integers(128))
+        Q = (1 << (int(bh[i]) - 1)) - 1
+        it["code"][i, j] += 1 if it["code"][i, j] < Q else -1
+        P.set_item(s, oracle.pack_item(bh, it["r"], it["c"], it["code"], it["piv"]))
+    return P
+
+
+def test_free_running_drift_config0():
+    """Free-running rollout, 64 steps.  Requantising every step is chaotic: one
+    rounding decision that differs (the fp32 sums run in a different order on
+    the GPU) decorrelates that item's quantisation noise within a step, so
+    per-step readout and code tolerances apply only in lockstep (above).  Here
+    the drift against each side's own unquantised fp32 recursion must agree
+    with the oracle's to within 1e-3 relative or, when larger, three times the
+    spread of the oracle's drift across rollouts whose items each start one
+    code step apart."""
+    cfg = W.CONFIGS[0]
+    su = Setup(cfg)
+    n = cfg.items
+    S0 = oracle.initial_state(cfg)
+    su.ref.pack(S0.reshape(n, 128, 128))
+    su.push_oracle_bytes()
+    others = [perturbed_copy(su.ref, su.bits, cfg.heads, seed) for seed in range(3)]
+    Sf_or = S0.reshape(n, 128, 128).copy()
+    Sf_gpu = torch.from_numpy(S0).cuda()
+    for t in range(cfg.steps):
+        x = W.step_inputs(cfg, t)
+        d = to_dev(x)
+        out = su.gpu.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+        stepq.fp32_step(cfg.variant, Sf_gpu, d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+        args = su.slot_inputs(x)
+        o_ref = su.ref.step(*args)
+        for P in others:
+            P.step(*args)
+        oracle.fp32_step(Sf_or, *args)
+        if t == 0:  # the first step starts from identical bytes
+            assert rel_l2(out.cpu().numpy().reshape(n, -1), o_ref) <= 1e-4
+        if (t + 1) % 16 == 0:
+            Sg = Sf_gpu.cpu().numpy().reshape(n, 128, 128)
+            assert rel_l2(Sg, Sf_or) < 1e-5  # the two fp32 references agree
+            D_gpu = rel_l2(su.gpu.unpack().cpu().numpy().reshape(n, 128, 128), Sg)
+            D_or = rel_l2(su.ref.unpack(), Sf_or)
+            spread = max(abs(rel_l2(P.unpack(), Sf_or) - D_or) for P in others)
+            tol = max(1e-3 * D_or, 3 * spread)
+            print(f"step {t}: drift gpu {D_gpu:.6f} oracle {D_or:.6f} spread {spread:.2e}")
+            assert abs(D_gpu - D_or) <= tol, f"step {t}: drift {D_gpu:.6e} vs oracle {D_or:.6e} (tol {tol:.2e})"
+
+
+@pytest.mark.parametrize("ci", [0, 2])
+def test_fp32_baseline_matches_oracle(ci):
+    cfg = W.with_overrides(W.CONFIGS[ci], batch=2)
+    n = cfg.items
+    S0 = oracle.initial_state(cfg)
+    S_gpu = torch.from_numpy(S0).cuda()
+    S_or = S0.reshape(n, 128, 128).copy()
+    kda = cfg.variant == W.KDA
+    for t in range(8):
+        x = W.step_inputs(cfg, t)
+        d = to_dev(x)
+        o = stepq.fp32_step(cfg.variant, S_gpu, d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+        o_ref = oracle.fp32_step(S_or, x["q"].reshape(n, -1), x["k"].reshape(n, -1), x["v"].reshape(n, -1),
+                                 x["alpha"].reshape(n, -1) if kda else x["alpha"].reshape(-1), x["beta"].reshape(-1), kda=kda)
+        assert rel_l2(o.cpu().numpy().reshape(n, -1), o_ref) < 1e-5
+    assert rel_l2(S_gpu.cpu().numpy().reshape(n, 128, 128), S_or) < 1e-5
+
+
+def test_zero_state_and_identity_update():
+    cfg = W.with_overrides(W.CONFIGS[1], batch=2, heads=8)
+    su = Setup(cfg)
+    n = cfg.items
+    su.gpu.pack(torch.zeros((cfg.batch, cfg.heads, 128, 128), device="cuda"))
+    su.ref.pack(np.zeros((n, 128, 128), np.float32))
+    torch.cuda.synchronize()
+    host = su.gpu.state.cpu().numpy()
+    for s in range(n):
+        assert bytes(su.gpu_item(host, s)) == bytes(su.ref.item(s))
+    # alpha = 1, beta = 0: the update is the identity and out = S^T q
+    x = W.step_inputs(cfg, 0)
+    x["alpha"][:] = 1.0
+    x["beta"][:] = 0.0
+    S0 = oracle.initial_state(cfg)
+    su.ref.pack(S0.reshape(n, 128, 128))
+    su.push_oracle_bytes()
+    Sd = su.ref.unpack()
+    d = to_dev(x)
+    out = su.gpu.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"]).cpu().numpy().reshape(n, -1)
+    want = np.einsum("nij,ni->nj", Sd.astype(np.float64), x["q"].reshape(n, -1).astype(np.float64))
+    assert rel_l2(out, want) < 1e-6
+
+
+def test_empty_batch_is_a_noop():
+    cfg = W.with_overrides(W.CONFIGS[0], batch=0)
+    pool = stepq.PackedStatePool(cfg.variant, 0, cfg.heads, W.bit_table(cfg), W.rho(cfg))
+    assert pool.state_nbytes == 0
+    e = torch.empty((0, cfg.heads, 128), device="cuda")
+    pool.decode_step(e, e, e, torch.empty((0, cfg.heads), device="cuda"), torch.empty((0, cfg.heads), device="cuda"))
+    pool.pack(torch.empty((0, cfg.heads, 128, 128), device="cuda"))
+    pool.close()
+
+
+def test_invalid_arguments_are_rejected_on_the_host():
+    cfg = W.with_overrides(W.CONFIGS[0], batch=2)
+    pool = stepq.PackedStatePool(cfg.variant, cfg.batch, cfg.heads, W.bit_table(cfg), W.rho(cfg))
+    d = to_dev(W.step_inputs(cfg, 0))
+    import ctypes as C
+    L = stepq.lib
+    h = pool._h
+    host = np.zeros(cfg.items * 128, np.float32)
+    P = lambda t: C.c_void_p(t.data_ptr())
+    # host memory where device memory is required
+    st = L.stepq_decode_step(h, host.ctypes.data_as(C.c_void_p), P(d["k"]), P(d["v"]), P(d["alpha"]), P(d["beta"]), P(d["v"]))
+    assert st == stepq.ERR_INVALID_ARG
+    # misaligned tensor
+    big = torch.zeros(cfg.items * 128 + 1, device="cuda")
+    st = L.stepq_decode_step(h, C.c_void_p(big.data_ptr() + 4), P(d["k"]), P(d["v"]), P(d["alpha"]), P(d["beta"]),
+                             P(torch.empty_like(d["v"])))
+    assert st == stepq.ERR_INVALID_ARG
+    # output aliasing an input
+    st = L.stepq_decode_step(h, P(d["q"]), P(d["k"]), P(d["v"]), P(d["alpha"]), P(d["beta"]), P(d["v"]))
+    assert st == stepq.ERR_INVALID_ARG
+    # shape checks in the binding
+    with pytest.raises(ValueError):
+        pool.decode_step(d["q"][:1], d["k"], d["v"], d["alpha"], d["beta"])
+    pool.close()
+    # a destroyed handle
+    st = L.stepq_decode_step(h, P(d["q"]), P(d["k"]), P(d["v"]), P(d["alpha"]), P(d["beta"]), P(torch.empty_like(d["v"])))
+    assert st == stepq.ERR_STATE
+    torch.cuda.synchronize()  # the context is still healthy
