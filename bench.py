@@ -48,6 +48,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--config", type=int, default=CONFIG_INDEX)
+    p.add_argument("--profile", action="store_true",
+                   help="short run for ncu: no fp32-baseline, end-to-end or CPU legs")
     return p.parse_args()
 
 
@@ -196,6 +198,46 @@ def run_reference(args, cfg):
     return 0
 
 
+def run_e2e(args, cfg, pool, host, out, stream, world):
+    """Same metric end to end through the public API with host buffers: every
+    step copies that step's inputs from pinned host memory, runs the decode
+    step and copies the readout back."""
+    import torch
+    import torch.distributed as dist
+    B, H = cfg.batch, cfg.heads
+    dev_in = {k: torch.empty_like(v, device="cuda") for k, v in host[0].items()}
+    out_host = torch.empty((B, H, cfg.dv), dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * 4 for v in host[0].values())
+    d2h = out_host.numel() * 4
+    def e2e_step(i):
+        hx = host[i % RING]
+        for k in dev_in:
+            dev_in[k].copy_(hx[k], non_blocking=True)
+        pool.decode_step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"], dev_in["beta"], out)
+        out_host.copy_(out, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for i in range(args.e2e_steps):
+        e2e_step(i)
+    g1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = g0.elapsed_time(g1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    value = world * cfg.items * args.e2e_steps / (e2e_ms * 1e-3)
+
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": args.e2e_steps}
+
+
 def main():
     args = parse()
     cfg = W.CONFIGS[args.config]
@@ -226,13 +268,31 @@ def main():
         x = W.step_inputs(cfg, t + 1000 * rank)
         ring.append({k: torch.from_numpy(v).cuda() for k, v in x.items()})
     out = torch.empty((B, H, cfg.dv), device="cuda")
-    # initial state: unquantised warm-up on the GPU (fp32 baseline kernel), then pack
+    stream = torch.cuda.current_stream()
+    # initial state: unquantised warm-up on the GPU (fp32 baseline kernel)
     S = torch.zeros((B, H, cfg.dk, cfg.dv), device="cuda")
     for t in range(-cfg.warmup, 0):
         d = ring[t % RING]
         stepq.fp32_step(cfg.variant, S, d["q"], d["k"], d["v"], d["alpha"], d["beta"], out)
+    torch.cuda.synchronize()
+    fp32_ms = None
+    if not args.profile:
+        # the fp32-state baseline kernel on the same inputs (packed/fp32 time ratio)
+        S_tmp = S.clone()
+        nf = max(10, args.steps // 20)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(nf):
+            d = ring[i % RING]
+            stepq.fp32_step(cfg.variant, S_tmp, d["q"], d["k"], d["v"], d["alpha"], d["beta"], out)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        fp32_ms = f0.elapsed_time(f1) / nf
+        del S_tmp
     pool.pack(S)
     torch.cuda.synchronize()
+    del S
+    torch.cuda.empty_cache()
 
     def step(i):
         d = ring[i % RING]
@@ -243,7 +303,6 @@ def main():
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         torch.cuda.synchronize()
@@ -262,58 +321,17 @@ def main():
     ms_per_step = ms / args.steps
     value = world * cfg.items * args.steps / (ms * 1e-3)
 
-    # fp32-state baseline kernel on the same inputs (the packed/fp32 time ratio)
-    for i in range(3):
-        d = ring[i % RING]
-        stepq.fp32_step(cfg.variant, S, d["q"], d["k"], d["v"], d["alpha"], d["beta"], out)
-    torch.cuda.synchronize()
-    nf = max(10, args.steps // 20)
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for i in range(nf):
-        d = ring[i % RING]
-        stepq.fp32_step(cfg.variant, S, d["q"], d["k"], d["v"], d["alpha"], d["beta"], out)
-    f1.record(stream)
-    torch.cuda.synchronize()
-    fp32_ms = f0.elapsed_time(f1) / nf
-    del S
-
     # end to end through the public API with host buffers: pinned H2D of the
     # step's inputs, the decode step, D2H of the readout, every step
+    e2e = None
     host = []
-    for t in range(RING):
+    for t in range(RING if not args.profile else 0):
         x = W.step_inputs(cfg, t + 1000 * rank)
         host.append({k: torch.from_numpy(v).pin_memory() for k, v in x.items()})
-    dev_in = {k: torch.empty_like(v, device="cuda") for k, v in host[0].items()}
-    out_host = torch.empty((B, H, cfg.dv), dtype=torch.float32).pin_memory()
-    h2d = sum(v.numel() * 4 for v in host[0].values())
-    d2h = out_host.numel() * 4
+    if not args.profile:
+        e2e = run_e2e(args, cfg, pool, host, out, stream, world)
 
-    def e2e_step(i):
-        hx = host[i % RING]
-        for k in dev_in:
-            dev_in[k].copy_(hx[k], non_blocking=True)
-        pool.decode_step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"], dev_in["beta"], out)
-        out_host.copy_(out, non_blocking=True)
-
-    for i in range(3):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g0.record(stream)
-    for i in range(args.e2e_steps):
-        e2e_step(i)
-    g1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = g0.elapsed_time(g1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * cfg.items * args.e2e_steps / (e2e_ms * 1e-3)
-
+    ring_bytes = sum(v.numel() * v.element_size() for v in ring[0].values())
     if rank == 0:
         peaks, src = measured_peaks()
         alg, state = algorithmic_bytes(cfg, bits)
@@ -326,19 +344,19 @@ def main():
             "config": {"workload": workload_name(cfg), "batch": B, "heads": H, "dk": cfg.dk, "dv": cfg.dv,
                        "packed_state_bytes": state, "per_gpu_items": cfg.items,
                        "l2": "inputs larger than L2 (packed pool %.0f MB + %d-step input ring %.0f MB, no flush)"
-                             % (state / 1e6, RING, RING * h2d / 1e6)},
+                             % (state / 1e6, RING, RING * ring_bytes / 1e6)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": recorded_traffic(cfg.name),
                          "algorithmic_bytes_per_launch": alg, "peak_source": src,
                          "kernel": "stepq fused decode step (k_item<0>)"},
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": args.e2e_steps},
+            "e2e": e2e,
             "gpu_launches": args.steps,
-            "fp32_state": {"ms_per_step": fp32_ms, "packed_speedup": fp32_ms / ms_per_step,
-                           "state_bytes": cfg.items * cfg.dk * cfg.dv * 4},
+            "fp32_state": None if fp32_ms is None else {
+                "ms_per_step": fp32_ms, "packed_speedup": fp32_ms / ms_per_step,
+                "state_bytes": cfg.items * cfg.dk * cfg.dv * 4},
             "clocks": clocks.summary(),
         }
-        if not args.no_cpu_baseline:
+        if not (args.no_cpu_baseline or args.profile):
             rate, meta = cpu_oracle_rate(cfg, args.cpu_seconds)
             line["cpu_baseline"] = dict(value=rate, unit=UNIT, **meta)
         print(json.dumps(line), flush=True)

@@ -165,6 +165,17 @@ STEPQ_API stepq_status stepq_fp32_step(const stepq_desc *desc, float *S, const f
                              const float *v, const float *alpha, const float *beta, float *out,
                              void *cuda_stream);
 
+/*
+ * Synchronise the pool's stream and read the pool's device status word.  The
+ * fused decode kernel stages items with asynchronous copies and waits for them
+ * with a bounded wait; if a wait ever gave up (the copy did not land within
+ * about two seconds), the kernel records it there and stops, leaving the
+ * remaining items of that step un-updated.  Returns STEPQ_OK if no kernel
+ * reported an error since the last check, else STEPQ_ERR_CUDA (and clears the
+ * word).
+ */
+STEPQ_API stepq_status stepq_pool_check(stepq_pool *pool);
+
 /* Human-readable name of a status; never NULL. */
 STEPQ_API const char *stepq_status_string(stepq_status s);
 

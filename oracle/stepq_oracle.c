@@ -70,47 +70,67 @@ double oracle_column_error_f64(int dk, int dv, int j, const double *S, const uin
     return e;
 }
 
-/* ---- the packed byte format ---------------------------------------------- */
+/* ---- the packed byte format ---------------------------------------------- *
+ * item = r[dk] fp32 | c[dv] fp32 | tile 0 | ... | tile dk/16 - 1.
+ * Tile T holds key rows 16T .. 16T+15.  For each column group g (value columns
+ * 4g .. 4g+3, g = 0 .. dv/4 - 1) the tile's codes are taken row by row, and
+ * within a row column by column, as fields of the row's width (the
+ * offset-binary code u = code + 2^(b-1), or the binary16 bits on a pivot row),
+ * concatenated into one little-endian bit stream that is zero-padded to whole
+ * 32-bit words.  Every stream of a tile has the same length W_T (the tile's
+ * rows fix it); word w of stream g is stored at word w * (dv/4) + g of the
+ * tile. */
 
-static size_t row_bytes(int dv, int b) { return (size_t)dv * (size_t)b / 8; }
+enum { TILE_ROWS = 16, GROUP_COLS = 4 };
+
+static int field_bits(int b) { return b; } /* a pivot row's field is its 16 binary16 bits */
+
+static size_t tile_words(const uint8_t *bits_tile)
+{
+    size_t nbits = 0;
+    for (int rr = 0; rr < TILE_ROWS; rr++) nbits += (size_t)GROUP_COLS * field_bits(bits_tile[rr]);
+    return (nbits + 31) / 32;
+}
 
 size_t oracle_item_bytes(int dk, int dv, const uint8_t *bits)
 {
     size_t n = 4 * (size_t)dk + 4 * (size_t)dv;
-    for (int i = 0; i < dk; i++) n += row_bytes(dv, bits[i]);
+    for (int T = 0; T < dk / TILE_ROWS; T++) n += 4 * tile_words(bits + T * TILE_ROWS) * (size_t)(dv / GROUP_COLS);
     return n;
 }
 
 static void put_f32(uint8_t *dst, float x) { memcpy(dst, &x, 4); } /* host is little-endian */
 static float get_f32(const uint8_t *src) { float x; memcpy(&x, src, 4); return x; }
 
+/* bit t of word index wi (little-endian 32-bit words) */
+static void set_bit(uint8_t *words, size_t wi, int t) { words[4 * wi + t / 8] |= (uint8_t)(1u << (t % 8)); }
+static int get_bit(const uint8_t *words, size_t wi, int t) { return (words[4 * wi + t / 8] >> (t % 8)) & 1; }
+
 void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
                       const int32_t *code, const float *piv, uint8_t *item)
 {
     uint8_t *p = item;
+    const int G = dv / GROUP_COLS;
     for (int i = 0; i < dk; i++, p += 4) put_f32(p, r[i]);
     for (int j = 0; j < dv; j++, p += 4) put_f32(p, c[j]);
-    for (int i = 0; i < dk; i++) {
-        int b = bits[i];
-        size_t nb = row_bytes(dv, b);
-        memset(p, 0, nb);
-        if (b == ORACLE_PIVOT_BITS) {
-            for (int j = 0; j < dv; j++) {
-                uint16_t h = oracle_to_fp16((double)piv[i * dv + j]);
-                p[2 * j] = (uint8_t)(h & 0xFF);
-                p[2 * j + 1] = (uint8_t)(h >> 8);
-            }
-        } else {
-            /* offset-binary code, bit t of column j at stream bit j*b + t */
-            for (int j = 0; j < dv; j++) {
-                uint32_t u = (uint32_t)(code[i * dv + j] + (1 << (b - 1)));
-                for (int t = 0; t < b; t++) {
-                    size_t bit = (size_t)j * b + t;
-                    p[bit / 8] |= (uint8_t)(((u >> t) & 1u) << (bit % 8));
+    for (int T = 0; T < dk / TILE_ROWS; T++) {
+        const size_t W = tile_words(bits + T * TILE_ROWS);
+        memset(p, 0, 4 * W * G);
+        for (int g = 0; g < G; g++) {
+            size_t pos = 0; /* bit position in stream g */
+            for (int rr = 0; rr < TILE_ROWS; rr++) {
+                const int i = T * TILE_ROWS + rr, b = bits[i];
+                for (int kk = 0; kk < GROUP_COLS; kk++) {
+                    const int j = g * GROUP_COLS + kk;
+                    const uint32_t u = (b == ORACLE_PIVOT_BITS)
+                                           ? oracle_to_fp16((double)piv[i * dv + j])
+                                           : (uint32_t)(code[i * dv + j] + (1 << (b - 1)));
+                    for (int t = 0; t < field_bits(b); t++, pos++)
+                        if ((u >> t) & 1u) set_bit(p, (pos / 32) * G + g, (int)(pos % 32));
                 }
             }
         }
-        p += nb;
+        p += 4 * W * G;
     }
 }
 
@@ -118,28 +138,31 @@ void oracle_unpack_item(int dk, int dv, const uint8_t *bits, const uint8_t *item
                         float *r, float *c, int32_t *code, float *piv)
 {
     const uint8_t *p = item;
+    const int G = dv / GROUP_COLS;
     for (int i = 0; i < dk; i++, p += 4) r[i] = get_f32(p);
     for (int j = 0; j < dv; j++, p += 4) c[j] = get_f32(p);
-    for (int i = 0; i < dk; i++) {
-        int b = bits[i];
-        if (b == ORACLE_PIVOT_BITS) {
-            for (int j = 0; j < dv; j++) {
-                uint16_t h = (uint16_t)(p[2 * j] | (p[2 * j + 1] << 8));
-                piv[i * dv + j] = (float)oracle_from_fp16(h);
-                code[i * dv + j] = 0;
-            }
-        } else {
-            for (int j = 0; j < dv; j++) {
-                uint32_t u = 0;
-                for (int t = 0; t < b; t++) {
-                    size_t bit = (size_t)j * b + t;
-                    u |= (uint32_t)((p[bit / 8] >> (bit % 8)) & 1u) << t;
+    for (int T = 0; T < dk / TILE_ROWS; T++) {
+        const size_t W = tile_words(bits + T * TILE_ROWS);
+        for (int g = 0; g < G; g++) {
+            size_t pos = 0;
+            for (int rr = 0; rr < TILE_ROWS; rr++) {
+                const int i = T * TILE_ROWS + rr, b = bits[i];
+                for (int kk = 0; kk < GROUP_COLS; kk++) {
+                    const int j = g * GROUP_COLS + kk;
+                    uint32_t u = 0;
+                    for (int t = 0; t < field_bits(b); t++, pos++)
+                        u |= (uint32_t)get_bit(p, (pos / 32) * G + g, (int)(pos % 32)) << t;
+                    if (b == ORACLE_PIVOT_BITS) {
+                        piv[i * dv + j] = (float)oracle_from_fp16((uint16_t)u);
+                        code[i * dv + j] = 0;
+                    } else {
+                        code[i * dv + j] = (int32_t)u - (1 << (b - 1));
+                        piv[i * dv + j] = 0;
+                    }
                 }
-                code[i * dv + j] = (int32_t)u - (1 << (b - 1));
-                piv[i * dv + j] = 0;
             }
         }
-        p += row_bytes(dv, b);
+        p += 4 * W * G;
     }
 }
 

@@ -103,11 +103,12 @@ uint16_t oracle_to_fp16(double x);
 double oracle_from_fp16(uint16_t h);
 
 /* ---- packed byte format (the pool) ---------------------------------------- *
- * item = r[dk] fp32 | c[dv] fp32 | row 0 | ... | row dk-1
- * quantised row i: dv * b_i / 8 bytes, a little-endian bit stream with the
- *   offset-binary code of column j in bits [j b_i, (j+1) b_i);
- * pivot row: dv binary16 values, little-endian.
- * Requires dv * b_i % 8 == 0 for every row. */
+ * item = r[dk] fp32 | c[dv] fp32 | tile 0 | ... | tile dk/16 - 1; tile T holds
+ * key rows 16T..16T+15.  Column group g (columns 4g..4g+3) of a tile is one
+ * little-endian bit stream: row by row, column by column, the row's b-bit
+ * offset-binary code (or 16 binary16 bits on a pivot row), zero-padded to whole
+ * 32-bit words; word w of stream g sits at word w * (dv/4) + g of the tile.
+ * Requires dk % 16 == 0 and dv % 4 == 0. */
 size_t oracle_item_bytes(int dk, int dv, const uint8_t *bits);
 void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
                       const int32_t *code, const float *piv, uint8_t *item);

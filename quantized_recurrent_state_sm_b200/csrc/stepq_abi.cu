@@ -27,6 +27,9 @@ struct stepq_pool {
     long long req_bytes = 0;
     cudaStream_t stream = nullptr;
     stepq::Tables t{};
+    int n_pivot_items = 0;
+    int nslots = 0, slot_bytes = 0;
+    int off_q = 0, off_k = 0, off_v = 0, off_alpha = 0, off_ab = 0, off_rec = 0;
 };
 
 namespace {
@@ -53,10 +56,11 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
     size_t state = 0;
-    size_t off_row_off = 0, off_row_bits = 0, off_row_s = 0, off_row_rho = 0;
-    size_t off_head_off = 0, off_head_nq = 0, off_order = 0, total = 0;
+    size_t off_rec = 0, off_head_off = 0, off_head_bytes = 0, off_order = 0, off_stage = 0, off_status = 0,
+           total = 0;
     long long req_bytes = 0;
     std::vector<long long> item_bytes;  // per head
+    std::vector<int> tile_words;        // per head and tile
 };
 
 // Checks a descriptor; fills the layout when valid.
@@ -90,25 +94,32 @@ stepq_status check_desc(const stepq_desc *d, bool need_tables, Layout *L)
         }
     }
     if (L) {
+        // packed item: header, then 8 tiles of 16 rows; a tile stores 32 column-group
+        // streams of W words each, W = ceil(4 * sum of the tile's widths / 32)
         L->item_bytes.assign(H, 0);
+        L->tile_words.assign((size_t)H * stepq::kTiles, 0);
         long long req = 0;
         for (int h = 0; h < H; h++) {
             long long n = stepq::kHeaderBytes;
-            for (int i = 0; i < kDK; i++) n += (long long)kDV * d->bits[h * kDK + i] / 8;
+            for (int T = 0; T < stepq::kTiles; T++) {
+                int bitsum = 0;
+                for (int rr = 0; rr < stepq::kRowsPerWarp; rr++) bitsum += d->bits[h * kDK + T * stepq::kRowsPerWarp + rr];
+                const int W = (4 * bitsum + 31) / 32;
+                L->tile_words[(size_t)h * stepq::kTiles + T] = W;
+                n += 4LL * W * stepq::kGroups;
+            }
             L->item_bytes[h] = n;
             req += n;
         }
         L->req_bytes = req;
         L->state = (size_t)req * (size_t)d->batch;
         size_t o = align_up(L->state, 256);
-        const size_t HD = (size_t)H * kDK;
-        L->off_row_off = o;  o = align_up(o + 4 * HD, 16);
-        L->off_row_bits = o; o = align_up(o + HD, 16);
-        L->off_row_s = o;    o = align_up(o + 4 * HD, 16);
-        L->off_row_rho = o;  o = align_up(o + 4 * HD, 16);
-        L->off_head_off = o; o = align_up(o + 8 * (size_t)H, 16);
-        L->off_head_nq = o;  o = align_up(o + 4 * (size_t)H, 16);
-        L->off_order = o;    o = align_up(o + 4 * (size_t)H * d->batch, 16);
+        L->off_rec = o;        o = align_up(o + sizeof(stepq::HeadRec) * (size_t)H, 256);
+        L->off_head_off = o;   o = align_up(o + 8 * (size_t)H, 16);
+        L->off_head_bytes = o; o = align_up(o + 4 * (size_t)H, 16);
+        L->off_status = o;     o = align_up(o + 16, 16);
+        L->off_order = o;      o = align_up(o + 4 * (size_t)H * d->batch, 16);
+        L->off_stage = o;      o = align_up(o + 16 * (size_t)H * d->batch, 16);
         L->total = o;
     }
     return STEPQ_OK;
@@ -160,6 +171,11 @@ stepq::StepArgs base_args(const stepq_pool *p)
     a.n_items = p->desc.batch * p->desc.heads;
     a.ls_iters = p->desc.ls_iters;
     a.kda = p->desc.variant == STEPQ_KDA;
+    a.nslots = p->nslots;
+    a.slot_bytes = p->slot_bytes;
+    a.off_q = p->off_q; a.off_k = p->off_k; a.off_v = p->off_v;
+    a.off_alpha = p->off_alpha; a.off_ab = p->off_ab; a.off_rec = p->off_rec;
+    a.n_pivot_items = p->n_pivot_items;
     return a;
 }
 
@@ -192,49 +208,95 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
 
     const int H = desc->heads, B = desc->batch;
     const size_t HD = (size_t)H * kDK;
-    std::vector<uint8_t> host(L.total - L.off_row_off, 0);
-    auto at = [&](size_t off) { return host.data() + (off - L.off_row_off); };
-    uint32_t *row_off = reinterpret_cast<uint32_t *>(at(L.off_row_off));
-    uint8_t *row_bits = at(L.off_row_bits);
-    float *row_s = reinterpret_cast<float *>(at(L.off_row_s));
-    float *row_rho = reinterpret_cast<float *>(at(L.off_row_rho));
+    std::vector<uint8_t> host(L.total - L.off_rec, 0);
+    auto at = [&](size_t off) { return host.data() + (off - L.off_rec); };
+    stepq::HeadRec *rec = reinterpret_cast<stepq::HeadRec *>(at(L.off_rec));
     long long *head_off = reinterpret_cast<long long *>(at(L.off_head_off));
-    int *head_nq = reinterpret_cast<int *>(at(L.off_head_nq));
+    int *head_bytes = reinterpret_cast<int *>(at(L.off_head_bytes));
     int *order = reinterpret_cast<int *>(at(L.off_order));
     long long pre = 0;
+    long long max_staged = 0;
+    std::vector<int> kind(H, stepq::kHeadQuant);
     for (int h = 0; h < H; h++) {
+        stepq::HeadRec &R = rec[h];
         head_off[h] = pre;
+        head_bytes[h] = (int)L.item_bytes[h];
+        R.head_off = pre;
+        R.head_bytes = (int)L.item_bytes[h];
         pre += L.item_bytes[h];
-        uint32_t o = stepq::kHeaderBytes;
-        int nq = 0;
+        int npiv = 0, b0 = desc->bits[h * kDK], same = 1;
         for (int i = 0; i < kDK; i++) {
             const int b = desc->bits[h * kDK + i];
-            row_off[h * kDK + i] = o;
-            o += (uint32_t)(kDV * b / 8);
-            row_bits[h * kDK + i] = (uint8_t)b;
-            const float r = desc->rho[h * kDK + i];
-            if (b != STEPQ_PIVOT_BITS) {
-                nq++;
-                row_s[h * kDK + i] = (float)(1.0 / std::sqrt((double)r));
-                row_rho[h * kDK + i] = r;
+            R.bits[i] = (uint8_t)b;
+            same &= (b == b0);
+            if (b == STEPQ_PIVOT_BITS) {
+                npiv++;
+                R.s[i] = 0.f;
+                R.rho[i] = 0.f;
             } else {
-                row_s[h * kDK + i] = 0.f;
-                row_rho[h * kDK + i] = 0.f;
+                R.s[i] = (float)(1.0 / std::sqrt((double)desc->rho[h * kDK + i]));
+                R.rho[i] = desc->rho[h * kDK + i];
             }
         }
-        head_nq[h] = nq;
+        kind[h] = npiv == 0 ? stepq::kHeadQuant : (npiv == kDK ? stepq::kHeadAllPivot : stepq::kHeadMixed);
+        R.head_kind = kind[h];
+        R.head_b = (same && b0 != STEPQ_PIVOT_BITS) ? b0 : 0;
+        uint32_t toff = stepq::kHeaderBytes;
+        for (int T = 0; T < stepq::kTiles; T++) {
+            const int W = L.tile_words[(size_t)h * stepq::kTiles + T];
+            R.tile_off[T] = toff;
+            R.tile_words[T] = (uint8_t)W;
+            toff += 4u * W * stepq::kGroups;
+        }
+        if (kind[h] != stepq::kHeadAllPivot) max_staged = std::max(max_staged, L.item_bytes[h]);
     }
-    // heaviest items (most packed bytes) are scheduled first
+    // order: items of all-pivot heads first (processed from global memory), then
+    // the staged items, heaviest first
     std::vector<int> idx((size_t)B * H);
     std::iota(idx.begin(), idx.end(), 0);
     std::stable_sort(idx.begin(), idx.end(), [&](int x, int y) {
-        return L.item_bytes[x % H] > L.item_bytes[y % H];
+        const int hx = x % H, hy = y % H;
+        const int px = kind[hx] == stepq::kHeadAllPivot, py = kind[hy] == stepq::kHeadAllPivot;
+        if (px != py) return px > py;
+        return L.item_bytes[hx] > L.item_bytes[hy];
     });
     std::memcpy(order, idx.data(), idx.size() * sizeof(int));
+    int *stage = reinterpret_cast<int *>(at(L.off_stage));
+    for (size_t n = 0; n < idx.size(); n++) {
+        const int item = idx[n], h = item % H;
+        const unsigned long long off = (unsigned long long)(item / H) * (unsigned long long)L.req_bytes +
+                                       (unsigned long long)head_off[h];
+        stage[4 * n + 0] = item;
+        stage[4 * n + 1] = (int)L.item_bytes[h];
+        stage[4 * n + 2] = (int)(uint32_t)(off & 0xFFFFFFFFull);
+        stage[4 * n + 3] = (int)(uint32_t)(off >> 32);
+    }
+    int n_pivot_items = 0;
+    for (int h = 0; h < H; h++) n_pivot_items += (kind[h] == stepq::kHeadAllPivot) ? B : 0;
+
+    // staging slot geometry of the fused decode kernel
+    const int kda = desc->variant == STEPQ_KDA;
+    int off = (int)align_up((size_t)max_staged, 16);
+    const int off_q = off; off += 4 * kDK;
+    const int off_k = off; off += 4 * kDK;
+    const int off_v = off; off += 4 * kDV;
+    const int off_alpha = off; off += kda ? 4 * kDK : 0;
+    const int off_ab = off; off += 16;
+    const int off_rec = off; off += (int)sizeof(stepq::HeadRec);
+    const int slot_bytes = (int)align_up((size_t)off, 128);
+    int nslots = 0;
+    for (int ns = stepq::kMaxSlots; ns >= 2; ns--) {
+        if (stepq::decode_ctas_per_sm(ns, slot_bytes) >= 2) { nslots = ns; break; }
+    }
+    if (nslots == 0) {
+        for (int ns = stepq::kMaxSlots; ns >= 2; ns--)
+            if (stepq::decode_ctas_per_sm(ns, slot_bytes) >= 1) { nslots = ns; break; }
+    }
+    if (nslots == 0 && max_staged > 0) return fail(STEPQ_ERR_CUDA, "no staging ring fits in shared memory");
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(cuda_stream);
     uint8_t *dev = static_cast<uint8_t *>(dev_buf);
-    cudaError_t e = cudaMemcpyAsync(dev + L.off_row_off, host.data(), host.size(), cudaMemcpyHostToDevice, s);
+    cudaError_t e = cudaMemcpyAsync(dev + L.off_rec, host.data(), host.size(), cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return cuda_fail(e, "table upload");
     e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "table upload sync");
@@ -250,13 +312,17 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
     p->state_bytes = L.state;
     p->req_bytes = L.req_bytes;
     p->stream = s;
-    p->t.row_off = reinterpret_cast<const uint32_t *>(dev + L.off_row_off);
-    p->t.row_bits = dev + L.off_row_bits;
-    p->t.row_s = reinterpret_cast<const float *>(dev + L.off_row_s);
-    p->t.row_rho = reinterpret_cast<const float *>(dev + L.off_row_rho);
+    p->t.rowrec = reinterpret_cast<const stepq::HeadRec *>(dev + L.off_rec);
     p->t.head_off = reinterpret_cast<const long long *>(dev + L.off_head_off);
-    p->t.head_nq = reinterpret_cast<const int *>(dev + L.off_head_nq);
+    p->t.head_bytes = reinterpret_cast<const int *>(dev + L.off_head_bytes);
     p->t.order = reinterpret_cast<const int *>(dev + L.off_order);
+    p->t.stage = reinterpret_cast<const int4 *>(dev + L.off_stage);
+    p->t.status = reinterpret_cast<int *>(dev + L.off_status);
+    p->n_pivot_items = n_pivot_items;
+    p->nslots = nslots;
+    p->slot_bytes = slot_bytes;
+    p->off_q = off_q; p->off_k = off_k; p->off_v = off_v;
+    p->off_alpha = off_alpha; p->off_ab = off_ab; p->off_rec = off_rec;
     {
         std::lock_guard<std::mutex> g(g_live_mu);
         g_live.insert(p);
@@ -368,6 +434,24 @@ stepq_status stepq_fp32_step(const stepq_desc *desc, float *S, const float *q, c
                                             desc->variant == STEPQ_KDA,
                                             reinterpret_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "stepq_fp32_step launch");
+}
+
+stepq_status stepq_pool_check(stepq_pool *pool)
+{
+    stepq_status st = check_pool(pool);
+    if (st != STEPQ_OK) return st;
+    cudaError_t e = cudaStreamSynchronize(pool->stream);
+    if (e != cudaSuccess) return cuda_fail(e, "stepq_pool_check sync");
+    int code = 0;
+    e = cudaMemcpy(&code, pool->t.status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "stepq_pool_check read");
+    if (code != 0) {
+        const int zero = 0;
+        cudaMemcpy(pool->t.status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        return fail(STEPQ_ERR_CUDA, "a kernel gave up waiting for a staged copy (device status %d); "
+                                    "the affected items were not updated", code);
+    }
+    return STEPQ_OK;
 }
 
 const char *stepq_status_string(stepq_status s)

@@ -1,0 +1,181 @@
+// Device helpers of the packed-state decode step: bulk-copy / mbarrier PTX,
+// the packed stream codec, and the float tricks the kernels use.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+
+#include "stepq_internal.cuh"
+
+namespace stepq {
+namespace dev {
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk asynchronous copy (the TMA engine, non-tensor form, from this
+// GPU's own global memory into this CTA's shared memory; no multicast).
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// One bulk copy global -> shared, completing on the barrier.  dst, src and
+// bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for a phase of the barrier: gives up after `limit` SM clock
+// cycles and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, long long limit)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > limit) return false;
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// float helpers
+// ---------------------------------------------------------------------------
+
+// 2^23: adding it to a float in [0, 2^22] leaves the integer part in the low
+// mantissa bits; a float whose bits are 0x4B000000 | u has the value 2^23 + u.
+constexpr float kMagic = 8388608.0f;
+constexpr uint32_t kMagicBits = 0x4B000000u;
+
+// The code u (< 2^22) of a float built as 0x4B000000 | u, minus the offset z:
+// exact in fp32.
+__device__ __forceinline__ float code_to_float(uint32_t u, float magic_plus_z)
+{
+    return __fsub_rn(__uint_as_float(kMagicBits | u), magic_plus_z);
+}
+
+// ---------------------------------------------------------------------------
+// packed stream codec: a column-group stream is a little-endian sequence of
+// fields; the fixed-width form keeps the stream words in registers.
+// ---------------------------------------------------------------------------
+
+// Field number c (width B) of a stream held in words w[].
+template <int B>
+__device__ __forceinline__ uint32_t field_at(const uint32_t *w, int c)
+{
+    const int pos = c * B, lo = pos >> 5, sh = pos & 31;
+    constexpr uint32_t mask = (1u << B) - 1u;
+    if (sh + B <= 32) return (w[lo] >> sh) & mask;
+    return __funnelshift_r(w[lo], w[lo + 1], sh) & mask;
+}
+
+// OR field value u (< 2^B) into position c of words w[].
+template <int B>
+__device__ __forceinline__ void field_put(uint32_t *w, int c, uint32_t u)
+{
+    const int pos = c * B, lo = pos >> 5, sh = pos & 31;
+    w[lo] |= u << sh;
+    if (sh + B > 32) w[lo + 1] |= u >> (32 - sh);
+}
+
+// Variable-width reader over stream words fetched on demand from shared memory
+// (word m of the stream at base[m * stride]).
+struct BitReader {
+    const uint32_t *base;
+    int stride;
+    int next;        // next word index
+    uint64_t buf;    // unread bits, LSB first
+    int nbits;       // number of unread bits in buf (0..63)
+    __device__ __forceinline__ void init(const uint32_t *b, int s)
+    {
+        base = b; stride = s; next = 0; buf = 0; nbits = 0;
+    }
+    // The next n (<= 32) bits.
+    __device__ __forceinline__ uint32_t take(int n)
+    {
+        if (nbits < n) {
+            buf |= (uint64_t)base[next * stride] << nbits;
+            nbits += 32;
+            next++;
+        }
+        const uint32_t v = (uint32_t)buf & (n == 32 ? 0xFFFFFFFFu : ((1u << n) - 1u));
+        buf >>= n;
+        nbits -= n;
+        return v;
+    }
+};
+
+// Variable-width writer emitting whole words to global memory (word m of the
+// stream at base[m * stride]); flush() writes the zero-padded last word.
+struct BitWriter {
+    uint32_t *base;
+    int stride;
+    int next;
+    uint64_t buf;
+    int nbits;
+    __device__ __forceinline__ void init(uint32_t *b, int s)
+    {
+        base = b; stride = s; next = 0; buf = 0; nbits = 0;
+    }
+    __device__ __forceinline__ void put(uint32_t v, int n)
+    {
+        buf |= (uint64_t)v << nbits;
+        nbits += n;
+        if (nbits >= 32) {
+            base[next * stride] = (uint32_t)buf;
+            next++;
+            buf >>= 32;
+            nbits -= 32;
+        }
+    }
+    __device__ __forceinline__ void flush()
+    {
+        if (nbits > 0) {
+            base[next * stride] = (uint32_t)buf;
+            next++;
+            buf = 0;
+            nbits = 0;
+        }
+    }
+};
+
+__device__ __forceinline__ int qmax_of(int b) { return (1 << (b - 1)) - 1; }
+
+}  // namespace dev
+}  // namespace stepq

@@ -10,20 +10,43 @@ namespace stepq {
 constexpr int kDK = 128;          // key dimension (rows of a state)
 constexpr int kDV = 128;          // value dimension (columns of a state)
 constexpr int kThreads = 256;     // threads per item: 8 warps x 16 rows, lane = 4 columns
-constexpr int kRowsPerWarp = 16;
+constexpr int kRowsPerWarp = 16;  // = rows of a packed tile
+constexpr int kTiles = kDK / kRowsPerWarp;
+constexpr int kGroups = kDV / 4;  // column groups (lanes) per tile
 constexpr int kPivotBits = 16;
 constexpr int kHeaderBytes = 4 * kDK + 4 * kDV;  // r[dk] | c[dv]
+constexpr int kMaxSlots = 8;
+
+// Head kinds.
+constexpr int kHeadQuant = 0;     // every row quantised
+constexpr int kHeadAllPivot = 1;  // every row a binary16 pivot
+constexpr int kHeadMixed = 2;     // some rows pivots
+
+// Per-head record (host-built, staged with every item): the fit constants and
+// the tile layout of the head's items.
+struct HeadRec {
+    float s[kDK];                // fp32(rho_i^-1/2), rounded once from fp64
+    float rho[kDK];              // row-impact weights
+    uint8_t bits[kDK];           // row widths (16 = pivot)
+    uint32_t tile_off[kTiles];   // byte offset of tile T inside the item
+    uint8_t tile_words[kTiles];  // 32-bit words per column-group stream of tile T
+    long long head_off;          // byte offset of the head's item inside a request
+    int head_b;                  // common row width, 0 if the rows differ
+    int head_kind;               // kHeadQuant / kHeadAllPivot / kHeadMixed
+    int head_bytes;              // bytes of one item
+    int pad;
+};
+static_assert(sizeof(HeadRec) % 16 == 0, "head record must be a multiple of 16 bytes");
 
 // Per-head tables derived on the host at pool creation, resident in the tail
 // of the caller's pool buffer.
 struct Tables {
-    const uint32_t *row_off;   // [H*dk] byte offset of row i inside its item
-    const uint8_t *row_bits;   // [H*dk] width of row i (16 = pivot)
-    const float *row_s;        // [H*dk] fp32(rho^-1/2), rounded once from fp64
-    const float *row_rho;      // [H*dk] impact weight
-    const long long *head_off; // [H] byte offset of head h's item inside a request
-    const int *head_nq;        // [H] number of quantised (non-pivot) rows
-    const int *order;          // [B*H] item processing order (heaviest first)
+    const HeadRec *rowrec;      // [H] head records
+    const long long *head_off;  // [H] byte offset of head h's item inside a request
+    const int *head_bytes;      // [H] bytes of an item of head h
+    const int *order;           // [B*H] item processing order: all-pivot heads' items first
+    const int4 *stage;          // [B*H] per position: {item, item bytes, pool offset lo, hi}
+    int *status;                // device status word: 0 ok, else an error code
 };
 
 struct StepArgs {
@@ -34,11 +57,19 @@ struct StepArgs {
     int n_items;
     int ls_iters;
     int kda;
+    // staging ring of the fused decode kernel
+    int nslots;
+    int slot_bytes;
+    int off_q, off_k, off_v, off_alpha, off_ab, off_rec;  // offsets inside a slot
+    int n_pivot_items;  // items of all-pivot heads, placed first in the order
     const float *q, *k, *v, *alpha, *beta;
     float *out;
     const float *S_in;  // pack
     float *S_out;       // unpack
 };
+
+// Device status codes.
+constexpr int kStatusWaitTimeout = 1;
 
 cudaError_t launch_decode_step(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_pack(const StepArgs &a, cudaStream_t s);
@@ -46,5 +77,8 @@ cudaError_t launch_unpack(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_fp32_step(float *S, const float *q, const float *k, const float *v,
                              const float *alpha, const float *beta, float *out, int n_items,
                              int kda, cudaStream_t s);
+// CTAs the fused decode kernel runs per SM and the dynamic shared memory it
+// gets for nslots staging slots of slot_bytes each; 0 if it cannot run.
+int decode_ctas_per_sm(int nslots, int slot_bytes);
 
 }  // namespace stepq

@@ -37,7 +37,7 @@ class Desc(C.Structure):
 
 EXPORTS = ("stepq_pool_bytes", "stepq_state_bytes", "stepq_pool_create", "stepq_pool_destroy",
            "stepq_pool_set_stream", "stepq_pack", "stepq_unpack", "stepq_decode_step",
-           "stepq_fp32_step", "stepq_status_string", "stepq_last_error")
+           "stepq_fp32_step", "stepq_pool_check", "stepq_status_string", "stepq_last_error")
 
 
 def _load():
@@ -51,11 +51,12 @@ def _load():
     L.stepq_pool_create.argtypes = [D, P, C.c_size_t, P, C.POINTER(P)]
     L.stepq_pool_destroy.argtypes = [P]
     L.stepq_pool_set_stream.argtypes = [P, P]
+    L.stepq_pool_check.argtypes = [P]
     L.stepq_pack.argtypes = [P, P]
     L.stepq_unpack.argtypes = [P, P]
     L.stepq_decode_step.argtypes = [P, P, P, P, P, P, P]
     L.stepq_fp32_step.argtypes = [D, P, P, P, P, P, P, P, P]
-    for fn in ("stepq_pool_create", "stepq_pool_destroy", "stepq_pool_set_stream", "stepq_pack",
+    for fn in ("stepq_pool_create", "stepq_pool_destroy", "stepq_pool_set_stream", "stepq_pool_check", "stepq_pack",
                "stepq_unpack", "stepq_decode_step", "stepq_fp32_step"):
         getattr(L, fn).restype = C.c_int
     L.stepq_status_string.argtypes = [C.c_int]; L.stepq_status_string.restype = C.c_char_p
@@ -162,6 +163,11 @@ class PackedStatePool:
                                      _dev(v, "v", (B, H, DV)), _dev(alpha, "alpha", ash),
                                      _dev(beta, "beta", (B, H)), _dev(out, "out", (B, H, DV))))
         return out
+
+    def check(self):
+        """Synchronise the pool's stream and raise if a kernel reported an error."""
+        self._sync_stream()
+        _check(lib.stepq_pool_check(self._h))
 
     def close(self):
         if getattr(self, "_h", None):

@@ -301,14 +301,21 @@ def parity_requests(cfg: Config):
 # packed pool layout (format arithmetic only)
 # ----------------------------------------------------------------------------
 
-def row_bytes(bits_row: np.ndarray, dv: int) -> np.ndarray:
-    return (dv * bits_row.astype(np.int64)) // 8
+TILE_ROWS, GROUP_COLS = 16, 4
+
+
+def tile_words(bits: np.ndarray) -> np.ndarray:
+    """32-bit words per column-group stream of each 16-row tile: [H, dk/16]."""
+    H, dk = bits.shape
+    per_tile = bits.astype(np.int64).reshape(H, dk // TILE_ROWS, TILE_ROWS).sum(axis=2)
+    return (GROUP_COLS * per_tile + 31) // 32
 
 
 def head_item_bytes(bits: np.ndarray, dv: int) -> np.ndarray:
-    """Bytes of one packed (request, head) item: r[dk] f32 | c[dv] f32 | rows."""
+    """Bytes of one packed (request, head) item: r[dk] f32 | c[dv] f32 | tiles,
+    a tile holding dv/4 interleaved streams of tile_words words each."""
     dk = bits.shape[1]
-    return 4 * dk + 4 * dv + row_bytes(bits, dv).sum(axis=1)
+    return 4 * dk + 4 * dv + 4 * (dv // GROUP_COLS) * tile_words(bits).sum(axis=1)
 
 
 def item_offsets(bits: np.ndarray, dv: int, batch: int) -> np.ndarray:

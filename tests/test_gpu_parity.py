@@ -87,6 +87,7 @@ def lockstep(setup, steps, t0=0, full_inputs=True):
             cmp.item(setup.head(s), setup.gpu_item(host, s), setup.ref.item(s), dg["tpre"][s],
                      dg["lsgap"][s], dg["S_new"][s], where=f"step {t} slot {s}")
     cmp.check_fraction()
+    setup.gpu.check()  # no kernel reported an error
     return cmp, worst
 
 

@@ -304,10 +304,20 @@ def test_zero_state_and_degenerate_columns():
 # packed byte format: an independent big-integer formulation of the bit stream
 # --------------------------------------------------------------------------
 
-def test_pack_format_bitstream():
+def stream_words(fields, nwords):
+    """Independent formulation of one column-group stream: a big integer with
+    field m (value, width) at bit sum of the previous widths, cut into words."""
+    acc, pos = 0, 0
+    for val, width in fields:
+        acc |= int(val) << pos
+        pos += width
+    return [(acc >> (32 * w)) & 0xFFFFFFFF for w in range(nwords)]
+
+
+def test_pack_format_tiled_streams():
     r = rng(11)
-    dk, dv = 12, 128
-    bits = np.array([2, 3, 4, 5, 6, 7, 8, 16, 3, 6, 16, 8], np.uint8)
+    dk, dv = 128, 128
+    bits = r.choice([2, 3, 4, 5, 6, 7, 8, 16], size=dk).astype(np.uint8)
     code = np.zeros((dk, dv), np.int32); piv = np.zeros((dk, dv), np.float32)
     for i, b in enumerate(bits):
         if b == 16:
@@ -317,47 +327,65 @@ def test_pack_format_bitstream():
             code[i] = r.integers(-Q, Q + 1, dv)
     rr = r.standard_normal(dk).astype(np.float32); cc = r.standard_normal(dv).astype(np.float32)
     item = oracle.pack_item(bits, rr, cc, code, piv)
-    assert item.size == 4 * dk + 4 * dv + int(sum(dv * int(b) // 8 for b in bits))
+    words_per_tile = [(4 * int(bits[16 * T:16 * T + 16].astype(int).sum()) + 31) // 32 for T in range(8)]
+    assert item.size == 4 * dk + 4 * dv + 128 * sum(words_per_tile)
     assert bytes(item[:4 * dk]) == rr.astype("<f4").tobytes()
     assert bytes(item[4 * dk: 4 * dk + 4 * dv]) == cc.astype("<f4").tobytes()
-    off = 4 * dk + 4 * dv
-    for i, b in enumerate(bits):
-        nb = dv * int(b) // 8
-        if b == 16:
-            want = piv[i].astype("<f2").tobytes()
-        else:
-            u = code[i] + (1 << (int(b) - 1))
-            assert np.all(u >= 1)
-            acc = 0
-            for j in range(dv):
-                acc |= int(u[j]) << (j * int(b))
-            want = acc.to_bytes(nb, "little")
-        assert bytes(item[off: off + nb]) == want, i
-        off += nb
+    words = item[4 * dk + 4 * dv:].view("<u4")
+    base = 0
+    for T in range(8):
+        W_T = words_per_tile[T]
+        tile = words[base: base + 32 * W_T].reshape(W_T, 32)  # word w of stream g at w*32 + g
+        for g in range(32):
+            fields = []
+            for rho_ in range(16):
+                i = 16 * T + rho_
+                b = int(bits[i])
+                for k in range(4):
+                    j = 4 * g + k
+                    if b == 16:
+                        fields.append((int(np.array([piv[i, j]], "<f2").view("<u2")[0]), 16))
+                    else:
+                        u = code[i, j] + (1 << (b - 1))
+                        assert 1 <= u <= (1 << b) - 1
+                        fields.append((u, b))
+            assert list(tile[:, g]) == stream_words(fields, W_T), (T, g)
+        base += 32 * W_T
     back = oracle.unpack_item(bits, item, dk, dv)
     np.testing.assert_array_equal(back["code"], code)
     np.testing.assert_array_equal(back["piv"], piv)
     np.testing.assert_array_equal(back["r"], rr)
 
 
-def test_golden_pack_rows():
-    """Hand-derived rows of the little-endian offset-binary bit stream."""
+def test_golden_pack_streams():
+    """Hand-derived column-group streams (tests/golden/pack_streams.txt)."""
     import os
-    path = os.path.join(os.path.dirname(__file__), "golden", "pack_rows.txt")
+    path = os.path.join(os.path.dirname(__file__), "golden", "pack_streams.txt")
     n = 0
     for line in open(path):
         line = line.split("#")[0].strip()
         if not line:
             continue
-        b_s, codes_s, hex_s = [x.strip() for x in line.split("|")]
+        b_s, pat, hex_s = [x.strip() for x in line.split("|")]
         b = int(b_s)
-        codes = np.array([int(x) for x in codes_s.split()], np.int32)
-        dv = codes.size
-        bits = np.array([b], np.uint8)
-        item = oracle.pack_item(bits, np.zeros(1), np.zeros(dv), codes[None, :], np.zeros((1, dv)))
-        assert bytes(item[4 + 4 * dv:]).hex() == hex_s.lower(), line
+        bits = np.full(128, b, np.uint8)
+        code = np.zeros((128, 128), np.int32)
+        if pat.startswith("all"):
+            code[:] = int(pat.split()[1])
+        else:
+            assert pat == "rowramp"
+            code[:] = (np.arange(128) % 16 % 15 - 7)[:, None]
+        item = oracle.pack_item(bits, np.zeros(128), np.zeros(128), code, np.zeros((128, 128)))
+        want = [int(x, 16) for x in hex_s.split()]
+        words = item[1024:].view("<u4")
+        W_T = len(want)
+        assert words.size == 8 * 32 * W_T
+        for T in range(8):
+            tile = words[T * 32 * W_T:(T + 1) * 32 * W_T].reshape(W_T, 32)
+            for g in (0, 7, 31):
+                assert list(tile[:, g]) == want, (line, T, g)
         n += 1
-    assert n >= 3
+    assert n >= 5
 
 
 # --------------------------------------------------------------------------
