@@ -70,6 +70,7 @@ struct StepArgs {
 
 // Device status codes.
 constexpr int kStatusWaitTimeout = 1;
+constexpr int kStatusBadHead = 2;
 
 cudaError_t launch_decode_step(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_pack(const StepArgs &a, cudaStream_t s);

@@ -4,7 +4,11 @@
 // head) item at a time; warp w owns key rows 16w .. 16w+15 (= packed tile w),
 // lane l owns value columns 4l .. 4l+3 (= column group l), so a thread holds
 // 64 state elements in registers and reads / writes exactly one column-group
-// stream of one tile: the pool layout is built around this mapping.
+// stream of one tile: the pool layout is built around this mapping.  The
+// elements are kept as float2 pairs (columns 4l, 4l+1 and 4l+2, 4l+3) so that
+// every floating-point operation on the state is one packed f32x2 instruction;
+// per-row factors are stored duplicated, (x, x), so that broadcasting them
+// costs nothing.
 //
 // Method (ai.info summary of STEPQuant, "Key Contributions" and "Methodology in
 // Plain English"; ai-papers.net, "STEPQuantの仕組み"; ai-trend.me, "핵심 용어"):
@@ -33,30 +37,61 @@ constexpr long long kWaitLimit = 4000000000LL;  // SM clock cycles before a wait
 constexpr float kRoundMagic = 12582912.0f;      // 1.5 * 2^23: x + it rounds x to an integer
 
 struct alignas(16) ItemSmem {
-    float rk[kDK], rl[kDK], rg[kDK], ra[kDK];  // update factors per row
-    float rs[kDK], rrho[kDK];                  // s_i, rho_i
-    float rh[kDK], rw[kDK], rqi[kDK];          // fit factors per row
-    int rb[kDK];                               // row widths
+    float2 rk2[kDK], rl2[kDK], rg2[kDK], ra2[kDK];  // update factors per row, duplicated
+    float2 rh2[kDK], rw2[kDK], rq2[kDK];            // fit factors per row, duplicated
+    float ra[kDK], rs[kDK], rrho[kDK];              // a_i, s_i, rho_i
+    int rb[kDK];                                    // row widths
     float cc[kDV], cv[kDV], cd[kDV], cdt[kDV], cu[kDV];
-    float cc0[kDV], ci0[kDV], cnew[kDV], ci[kDV], crat[kDV];
+    float cc0[kDV], cnew[kDV], ci[kDV], crat[kDV];
     float red[2][8][kDV];
-    float rowt[8][16][36];                     // per-warp transposition for row sums
+    float rowt[8][16][36];  // per-warp transposition for row sums
     float kq[4];
-    float alpha_item, beta_item;
+    float beta_item;
     uint32_t tile_off[kTiles];
     int head_b, head_kind;
     long long head_off;
     uint64_t bar[kMaxSlots];
 };
 
+using X2 = float2[kRowsPerWarp][2];  // the thread's 16 x 4 block as float2 pairs
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float2 ld2(const float2 *p) { return *p; }
+
+// Call-free reciprocal, quotient and square root (within 2 ulp of the correctly
+// rounded results) for the per-row and per-column factors computed while the
+// thread's state is live in registers: the correctly rounded forms branch to a
+// slow-path subroutine whose call would force the state out to local memory.
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float div_approx(float a, float b) { return a * rcp_approx(b); }
+__device__ __forceinline__ float sqrt_approx(float x)
+{
+    float r;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// 3-input maximum of a, |b| and |c|.
+__device__ __forceinline__ float max_abs3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+    return r;
+}
 
 // ---------------------------------------------------------------------------
-// Column sums over the 8 warps of per-thread partials (two vectors at once).
+// Column sums over the 8 warps of per-thread partials.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void stash_partials(ItemSmem &sm, int vec, const float (&x)[4])
+__device__ __forceinline__ void stash(ItemSmem &sm, int vec, float2 a, float2 b)
 {
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    *reinterpret_cast<float4 *>(&sm.red[vec][w][4 * l]) = make_float4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<float4 *>(&sm.red[vec][w][4 * l]) = make_float4(a.x, a.y, b.x, b.y);
 }
 
 __device__ __forceinline__ float sum_partials(const ItemSmem &sm, int vec, int j)
@@ -75,27 +110,29 @@ __device__ __forceinline__ float max_partials(const ItemSmem &sm, int vec, int j
     return acc;
 }
 
-__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
-
 // ---------------------------------------------------------------------------
 // Decode the thread's column-group stream of its tile into X (code values as
-// floats; pivot rows: binary16 values times mult_piv).  Fixed width B > 0 keeps
-// the stream in registers; B == 0 reads widths per row from sm.rb.
+// floats; pivot rows: their binary16 values).  Fixed width B > 0 keeps the
+// stream in registers; B == 0 reads widths per row from sm.rb.
 // ---------------------------------------------------------------------------
 template <int B>
-__device__ __forceinline__ void decode_stream(const ItemSmem &sm, const uint32_t *words, int stride,
-                                              float (&X)[kRowsPerWarp][4])
+__device__ __forceinline__ void decode_stream(const ItemSmem &sm, const uint32_t *words, int stride, X2 &X)
 {
     const int w = threadIdx.x >> 5;
     if constexpr (B > 0) {
         uint32_t wd[2 * B];
 #pragma unroll
         for (int m = 0; m < 2 * B; m++) wd[m] = words[m * stride];
-        const float mz = kMagic + (float)(1 << (B - 1));
+        const float mz = -(kMagic + (float)(1 << (B - 1)));
+        const float2 mz2 = f2(mz, mz);
 #pragma unroll
         for (int rr = 0; rr < kRowsPerWarp; rr++)
 #pragma unroll
-            for (int kk = 0; kk < 4; kk++) X[rr][kk] = code_to_float(field_at<B>(wd, 4 * rr + kk), mz);
+            for (int hh = 0; hh < 2; hh++) {
+                const uint32_t u0 = field_at<B>(wd, 4 * rr + 2 * hh) | kMagicBits;
+                const uint32_t u1 = field_at<B>(wd, 4 * rr + 2 * hh + 1) | kMagicBits;
+                X[rr][hh] = __fadd2_rn(f2(__uint_as_float(u0), __uint_as_float(u1)), mz2);
+            }
     } else {
         BitReader br;
         br.init(words, stride);
@@ -104,18 +141,21 @@ __device__ __forceinline__ void decode_stream(const ItemSmem &sm, const uint32_t
             const int b = sm.rb[kRowsPerWarp * w + rr];
             if (b == kPivotBits) {
 #pragma unroll
-                for (int half = 0; half < 2; half++) {
+                for (int hh = 0; hh < 2; hh++) {
                     const uint32_t hv = br.take(32);
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hv));
-                    X[rr][2 * half] = f.x;
-                    X[rr][2 * half + 1] = f.y;
+                    X[rr][hh] = __half22float2(*reinterpret_cast<const __half2 *>(&hv));
                 }
             } else {
                 const uint32_t f = br.take(4 * b);
                 const uint32_t mask = (1u << b) - 1u;
-                const float mz = kMagic + (float)(1 << (b - 1));
+                const float mz = -(kMagic + (float)(1 << (b - 1)));
+                const float2 mz2 = f2(mz, mz);
 #pragma unroll
-                for (int kk = 0; kk < 4; kk++) X[rr][kk] = code_to_float((f >> (kk * b)) & mask, mz);
+                for (int hh = 0; hh < 2; hh++) {
+                    const uint32_t u0 = ((f >> (2 * hh * b)) & mask) | kMagicBits;
+                    const uint32_t u1 = ((f >> ((2 * hh + 1) * b)) & mask) | kMagicBits;
+                    X[rr][hh] = __fadd2_rn(f2(__uint_as_float(u0), __uint_as_float(u1)), mz2);
+                }
             }
         }
     }
@@ -124,24 +164,23 @@ __device__ __forceinline__ void decode_stream(const ItemSmem &sm, const uint32_t
 // ---------------------------------------------------------------------------
 // The fit (row scales, column scales, least squares), requantisation and the
 // packed store.  On entry X holds P_ij = S_ij / a_i on quantised rows and S_ij
-// on pivot rows; sm.ra, rs, rrho, rb, rqi and sm.head_b are set.  Writes r', c
-// and the streams of the item at item_g.  Contains __syncthreads.
+// on pivot rows; sm.ra, rs, rrho, rb, rq2 and sm.head_b / head_kind are set.
+// Writes r', c and the item's streams at item_g.  Contains __syncthreads.
+// ROWWISE: rows may differ in width and may be pivots.
 // ---------------------------------------------------------------------------
 template <int B, bool ROWWISE>
-__device__ __forceinline__ void fit_and_store(ItemSmem &sm, float (&X)[kRowsPerWarp][4], uint8_t *item_g,
-                                              int ls_iters)
+__device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item_g, int ls_iters)
 {
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    const int r0 = kRowsPerWarp * w;
     // ---- row magnitudes: sum over the 128 columns of P^2 -------------------
     {
         float *t = &sm.rowt[w][0][0];
 #pragma unroll
         for (int rr = 0; rr < kRowsPerWarp; rr++) {
-            float ss = X[rr][0] * X[rr][0];
-            ss = fmaf(X[rr][1], X[rr][1], ss);
-            ss = fmaf(X[rr][2], X[rr][2], ss);
-            ss = fmaf(X[rr][3], X[rr][3], ss);
-            t[rr * 36 + l] = ss;
+            float2 s2 = __fmul2_rn(X[rr][0], X[rr][0]);
+            s2 = __ffma2_rn(X[rr][1], X[rr][1], s2);
+            t[rr * 36 + l] = s2.x + s2.y;
         }
         __syncwarp();
         const int rr = l >> 1, hf = l & 1;
@@ -153,95 +192,96 @@ __device__ __forceinline__ void fit_and_store(ItemSmem &sm, float (&X)[kRowsPerW
         }
         ss += __shfl_xor_sync(0xffffffffu, ss, 1);
         if (hf == 0) {
-            const int i = kRowsPerWarp * w + rr;
+            const int i = r0 + rr;
             const int b = sm.rb[i];
-            float rnew = 0.f, h = 0.f, wt = 0.f;
+            float rnew = 0.f, h = 1.f, wt = 0.f;  // pivot rows: p = S, not part of any fit
             if (b != kPivotBits) {
                 const float a = sm.ra[i];
-                float m = a * sqrtf(ss * (1.0f / kDV));
+                float m = a * sqrt_approx(ss * (1.0f / kDV));
                 if (m == 0.f) m = 1.f;
-                rnew = __fdiv_rn(m * sm.rs[i], (float)qmax_of(b));
-                h = __fdiv_rn(a, rnew);
+                rnew = (m * sm.rs[i]) * sm.rq2[i].x;
+                h = div_approx(a, rnew);
                 wt = (sm.rrho[i] * rnew) * rnew;
             }
-            sm.rh[i] = h;
-            sm.rw[i] = wt;
+            sm.rh2[i] = f2(h, h);
+            sm.rw2[i] = f2(wt, wt);
             reinterpret_cast<float *>(item_g)[i] = rnew;
         }
         __syncwarp();
     }
-    // ---- p = P h; column maxima ------------------------------------------
+    // ---- p = P h; column maxima (of |p| / Q_i for row-wise widths) ----------
     {
         float mx[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int r4 = 0; r4 < kRowsPerWarp; r4 += 4) {
-            const float4 h4 = ld4(&sm.rh[kRowsPerWarp * w + r4]);
-            const float4 q4 = ld4(&sm.rqi[kRowsPerWarp * w + r4]);
-            const float hv[4] = {h4.x, h4.y, h4.z, h4.w};
-            const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+        for (int rr = 0; rr < kRowsPerWarp; rr += 2) {
+            float2 p[2][2];
 #pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const int rr = r4 + u;
-                if (ROWWISE && sm.rb[kRowsPerWarp * w + rr] == kPivotBits) continue;
-#pragma unroll
-                for (int kk = 0; kk < 4; kk++) {
-                    const float p = X[rr][kk] * hv[u];
-                    X[rr][kk] = p;
-                    mx[kk] = fmaxf(mx[kk], ROWWISE ? fabsf(p) * qv[u] : fabsf(p));
+            for (int u = 0; u < 2; u++) {
+                const int i = r0 + rr + u;
+                const float2 hh = ld2(&sm.rh2[i]);
+                p[u][0] = __fmul2_rn(X[rr + u][0], hh);
+                p[u][1] = __fmul2_rn(X[rr + u][1], hh);
+                X[rr + u][0] = p[u][0];
+                X[rr + u][1] = p[u][1];
+                if (ROWWISE) {  // pivot rows have rq2 = 0 and do not count
+                    const float2 qq = ld2(&sm.rq2[i]);
+                    p[u][0] = __fmul2_rn(p[u][0], qq);
+                    p[u][1] = __fmul2_rn(p[u][1], qq);
                 }
             }
+            mx[0] = max_abs3(mx[0], p[0][0].x, p[1][0].x);
+            mx[1] = max_abs3(mx[1], p[0][0].y, p[1][0].y);
+            mx[2] = max_abs3(mx[2], p[0][1].x, p[1][1].x);
+            mx[3] = max_abs3(mx[3], p[0][1].y, p[1][1].y);
         }
-        stash_partials(sm, 0, mx);
+        stash(sm, 0, f2(mx[0], mx[1]), f2(mx[2], mx[3]));
     }
     __syncthreads();
     if (tid < kDV) {
         const int j = tid;
         float m = max_partials(sm, 0, j);
-        if (!ROWWISE) m = __fdiv_rn(m, (float)qmax_of(sm.head_b));
+        if (!ROWWISE) m = m * sm.rq2[0].x;  // every row has the head's width
         const float c0 = (m > 0.f) ? m : 1.f;
-        const float ic0 = __frcp_rn(c0);
         sm.cc0[j] = c0;
-        sm.ci0[j] = ic0;
         sm.cnew[j] = c0;
-        sm.ci[j] = ic0;
+        sm.ci[j] = rcp_approx(c0);
         sm.crat[j] = 1.f;
     }
     __syncthreads();
     // ---- impact-weighted least squares for the column scales ---------------
+    const float2 rm2 = f2(kRoundMagic, kRoundMagic), nrm2 = f2(-kRoundMagic, -kRoundMagic);
     for (int it = 0; it < ls_iters; it++) {
-        float ic[4];
-        {
-            const float4 v = ld4(&sm.ci[4 * l]);
-            ic[0] = v.x; ic[1] = v.y; ic[2] = v.z; ic[3] = v.w;
-        }
-        float N[4] = {0.f, 0.f, 0.f, 0.f}, D[4] = {0.f, 0.f, 0.f, 0.f};
+        const float4 i4 = ld4(&sm.ci[4 * l]);
+        const float2 ic0 = f2(i4.x, i4.y), ic1 = f2(i4.z, i4.w);
+        float2 N0 = f2(0.f, 0.f), N1 = N0, D0 = N0, D1 = N0;
 #pragma unroll
-        for (int r4 = 0; r4 < kRowsPerWarp; r4 += 4) {
-            const float4 w4 = ld4(&sm.rw[kRowsPerWarp * w + r4]);
-            const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const int rr = r4 + u;
-                if (ROWWISE && sm.rb[kRowsPerWarp * w + rr] == kPivotBits) continue;
-                const float Q = (float)qmax_of(ROWWISE ? sm.rb[kRowsPerWarp * w + rr] : B);
-#pragma unroll
-                for (int kk = 0; kk < 4; kk++) {
-                    float n = __fmaf_rn(X[rr][kk], ic[kk], kRoundMagic) - kRoundMagic;
-                    if (it > 0 || ROWWISE) n = fminf(fmaxf(n, -Q), Q);  // later rounds may clip
-                    const float wn = wv[u] * n;
-                    N[kk] = fmaf(wn, X[rr][kk], N[kk]);
-                    D[kk] = fmaf(wn, n, D[kk]);
-                }
+        for (int rr = 0; rr < kRowsPerWarp; rr++) {
+            const int i = r0 + rr;
+            if (ROWWISE && sm.rb[i] == kPivotBits) continue;
+            const float2 ww = ld2(&sm.rw2[i]);
+            // round p / c to the nearest integer: |p / c0| <= Q, so no clipping in
+            // the first round; later rounds clip to the row's range
+            float2 n0 = __fadd2_rn(__ffma2_rn(X[rr][0], ic0, rm2), nrm2);
+            float2 n1 = __fadd2_rn(__ffma2_rn(X[rr][1], ic1, rm2), nrm2);
+            if (it > 0) {
+                const float Q = (float)qmax_of(ROWWISE ? sm.rb[i] : B);
+                n0 = f2(fminf(fmaxf(n0.x, -Q), Q), fminf(fmaxf(n0.y, -Q), Q));
+                n1 = f2(fminf(fmaxf(n1.x, -Q), Q), fminf(fmaxf(n1.y, -Q), Q));
             }
+            const float2 wn0 = __fmul2_rn(ww, n0), wn1 = __fmul2_rn(ww, n1);
+            N0 = __ffma2_rn(wn0, X[rr][0], N0);
+            N1 = __ffma2_rn(wn1, X[rr][1], N1);
+            D0 = __ffma2_rn(wn0, n0, D0);
+            D1 = __ffma2_rn(wn1, n1, D1);
         }
-        stash_partials(sm, 0, N);
-        stash_partials(sm, 1, D);
+        stash(sm, 0, N0, N1);
+        stash(sm, 1, D0, D1);
         __syncthreads();
         if (tid < kDV) {
             const int j = tid;
             const float nn = sum_partials(sm, 0, j), dd = sum_partials(sm, 1, j);
-            const float c = (dd > 0.f) ? __fdiv_rn(nn, dd) : sm.cnew[j];
-            const float icn = __frcp_rn(c);
+            const float c = (dd > 0.f) ? div_approx(nn, dd) : sm.cnew[j];
+            const float icn = rcp_approx(c);
             sm.cnew[j] = c;
             sm.ci[j] = icn;
             sm.crat[j] = sm.cc0[j] * icn;
@@ -249,73 +289,86 @@ __device__ __forceinline__ void fit_and_store(ItemSmem &sm, float (&X)[kRowsPerW
         __syncthreads();
     }
     // ---- requantise, pack, store -------------------------------------------
-    float ic[4], rat = 0.f;
+    const float4 i4 = ld4(&sm.ci[4 * l]);
+    const float2 ic0 = f2(i4.x, i4.y), ic1 = f2(i4.z, i4.w);
+    float rat;
     {
-        const float4 v = ld4(&sm.ci[4 * l]);
-        ic[0] = v.x; ic[1] = v.y; ic[2] = v.z; ic[3] = v.w;
         const float4 r = ld4(&sm.crat[4 * l]);
         rat = fmaxf(fmaxf(r.x, r.y), fmaxf(r.z, r.w));
     }
-    // the largest |p / c| of a column is Q c0 / c: clip only where it can pass Q + 1/2
+    // the largest |p / c| of a column is at most Q c0 / c: clip only where that
+    // can reach Q + 1/2
     rat = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(rat)));
     uint32_t *words = reinterpret_cast<uint32_t *>(item_g + sm.tile_off[w]) + l;
     if constexpr (B > 0) {
         constexpr int Qb = (1 << (B - 1)) - 1;
+        constexpr uint32_t mask = (1u << B) - 1u;
         const bool clip = (float)Qb * (rat - 1.f) >= 0.49f;
         const float mz = kMagic + (float)(1 << (B - 1));
-        constexpr uint32_t mask = (1u << B) - 1u;
-        uint32_t ow[2 * B];
+        const float2 mz2 = f2(mz, mz);
+        uint32_t ow[2 * B + 1];
 #pragma unroll
-        for (int m = 0; m < 2 * B; m++) ow[m] = 0u;
+        for (int m = 0; m <= 2 * B; m++) ow[m] = 0u;
 #pragma unroll
         for (int rr = 0; rr < kRowsPerWarp; rr++)
 #pragma unroll
-            for (int kk = 0; kk < 4; kk++) {
-                float mm;
+            for (int hh = 0; hh < 2; hh++) {
+                float2 mm;
                 if (!clip) {
-                    mm = __fmaf_rn(X[rr][kk], ic[kk], mz);
+                    mm = __ffma2_rn(X[rr][hh], hh ? ic1 : ic0, mz2);
                 } else {
-                    const float t = fminf(fmaxf(X[rr][kk] * ic[kk], -(float)Qb), (float)Qb);
-                    mm = t + mz;
+                    float2 t = __fmul2_rn(X[rr][hh], hh ? ic1 : ic0);
+                    t = f2(fminf(fmaxf(t.x, -(float)Qb), (float)Qb), fminf(fmaxf(t.y, -(float)Qb), (float)Qb));
+                    mm = __fadd2_rn(t, mz2);
                 }
-                field_put<B>(ow, 4 * rr + kk, __float_as_uint(mm) & mask);
-            }
 #pragma unroll
-        for (int m = 0; m < 2 * B; m++) words[m * kGroups] = ow[m];
+                for (int e = 0; e < 2; e++) {
+                    const int c = 4 * rr + 2 * hh + e;
+                    field_put<B>(ow, c, __float_as_uint(e ? mm.y : mm.x) & mask);
+                    // store every word the code completed (known at compile time)
+#pragma unroll
+                    for (int m = (c * B) / 32; m < ((c + 1) * B) / 32; m++) words[m * kGroups] = ow[m];
+                }
+            }
     } else {
         BitWriter bw;
         bw.init(words, kGroups);
 #pragma unroll
         for (int rr = 0; rr < kRowsPerWarp; rr++) {
-            const int b = sm.rb[kRowsPerWarp * w + rr];
+            const int b = sm.rb[r0 + rr];
             if (b == kPivotBits) {
-                const __half2 h0 = __floats2half2_rn(X[rr][0], X[rr][1]);
-                const __half2 h1 = __floats2half2_rn(X[rr][2], X[rr][3]);
-                bw.put(*reinterpret_cast<const uint32_t *>(&h0), 32);
-                bw.put(*reinterpret_cast<const uint32_t *>(&h1), 32);
+#pragma unroll
+                for (int hh = 0; hh < 2; hh++) {
+                    const __half2 hv = __floats2half2_rn(X[rr][hh].x, X[rr][hh].y);
+                    bw.put(*reinterpret_cast<const uint32_t *>(&hv), 32);
+                }
             } else {
                 const int Qb = qmax_of(b);
                 const bool clip = (float)Qb * (rat - 1.f) >= 0.49f;
                 const float mz = kMagic + (float)(1 << (b - 1));
+                const float2 mz2 = f2(mz, mz);
                 const uint32_t mask = (1u << b) - 1u;
                 uint32_t f = 0;
 #pragma unroll
-                for (int kk = 0; kk < 4; kk++) {
-                    float mm;
+                for (int hh = 0; hh < 2; hh++) {
+                    float2 mm;
                     if (!clip) {
-                        mm = __fmaf_rn(X[rr][kk], ic[kk], mz);
+                        mm = __ffma2_rn(X[rr][hh], hh ? ic1 : ic0, mz2);
                     } else {
-                        const float t = fminf(fmaxf(X[rr][kk] * ic[kk], -(float)Qb), (float)Qb);
-                        mm = t + mz;
+                        float2 t = __fmul2_rn(X[rr][hh], hh ? ic1 : ic0);
+                        t = f2(fminf(fmaxf(t.x, -(float)Qb), (float)Qb), fminf(fmaxf(t.y, -(float)Qb), (float)Qb));
+                        mm = __fadd2_rn(t, mz2);
                     }
-                    f |= (__float_as_uint(mm) & mask) << (kk * b);
+                    f |= (__float_as_uint(mm.x) & mask) << (2 * hh * b);
+                    f |= (__float_as_uint(mm.y) & mask) << ((2 * hh + 1) * b);
                 }
                 bw.put(f, 4 * b);
             }
         }
         bw.flush();
     }
-    if (tid < kDV) reinterpret_cast<float *>(item_g)[kDK + tid] = (sm.head_kind == kHeadAllPivot) ? 0.f : sm.cnew[tid];
+    if (tid < kDV)
+        reinterpret_cast<float *>(item_g)[kDK + tid] = (sm.head_kind == kHeadAllPivot) ? 0.f : sm.cnew[tid];
 }
 
 // ---------------------------------------------------------------------------
@@ -339,10 +392,10 @@ __device__ void pivot_item(ItemSmem &sm, const StepArgs &a, int item)
         const int i = tid;
         const float al = a.kda ? a.alpha[vec + i] : a.alpha[item];
         const float k = a.k[vec + i], q = a.q[vec + i];
-        sm.rk[i] = al * k;
-        sm.rl[i] = al * q;
-        sm.rg[i] = beta * k;
-        sm.ra[i] = al;
+        sm.rk2[i] = f2(al * k, al * k);
+        sm.rl2[i] = f2(al * q, al * q);
+        sm.rg2[i] = f2(beta * k, beta * k);
+        sm.ra2[i] = f2(al, al);
         float kq = k * q;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, o);
@@ -352,28 +405,27 @@ __device__ void pivot_item(ItemSmem &sm, const StepArgs &a, int item)
     }
     __syncthreads();
     uint32_t *words = reinterpret_cast<uint32_t *>(item_g + rec->tile_off[w]) + l;
-    float X[kRowsPerWarp][4];
-    float V[4] = {0.f, 0.f, 0.f, 0.f}, U[4] = {0.f, 0.f, 0.f, 0.f};
+    X2 X;
+    float2 V0 = f2(0.f, 0.f), V1 = V0, U0 = V0, U1 = V0;
 #pragma unroll
     for (int rr = 0; rr < kRowsPerWarp; rr++) {
         const int i = kRowsPerWarp * w + rr;
         const uint32_t w0 = words[(2 * rr) * kGroups], w1 = words[(2 * rr + 1) * kGroups];
-        const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&w0));
-        const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&w1));
-        const float hv[4] = {f0.x, f0.y, f1.x, f1.y};
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++) {
-            X[rr][kk] = sm.ra[i] * hv[kk];
-            V[kk] = fmaf(sm.rk[i], hv[kk], V[kk]);
-            U[kk] = fmaf(sm.rl[i], hv[kk], U[kk]);
-        }
+        const float2 h0 = __half22float2(*reinterpret_cast<const __half2 *>(&w0));
+        const float2 h1 = __half22float2(*reinterpret_cast<const __half2 *>(&w1));
+        const float2 kk = ld2(&sm.rk2[i]), ll = ld2(&sm.rl2[i]), aa = ld2(&sm.ra2[i]);
+        X[rr][0] = __fmul2_rn(aa, h0);
+        X[rr][1] = __fmul2_rn(aa, h1);
+        V0 = __ffma2_rn(kk, h0, V0);
+        V1 = __ffma2_rn(kk, h1, V1);
+        U0 = __ffma2_rn(ll, h0, U0);
+        U1 = __ffma2_rn(ll, h1, U1);
     }
-    stash_partials(sm, 0, V);
-    stash_partials(sm, 1, U);
+    stash(sm, 0, V0, V1);
+    stash(sm, 1, U0, U1);
     __syncthreads();
     if (tid < kDV) {
-        const float d = sm.cv[tid] - sum_partials(sm, 0, tid);
-        sm.cd[tid] = d;
+        sm.cd[tid] = sm.cv[tid] - sum_partials(sm, 0, tid);
     } else {
         sm.cu[tid - kDK] = sum_partials(sm, 1, tid - kDK);
     }
@@ -383,13 +435,14 @@ __device__ void pivot_item(ItemSmem &sm, const StepArgs &a, int item)
         a.out[(long long)item * kDV + tid] = fmaf(beta * kq, sm.cd[tid], sm.cu[tid]);
     }
     const float4 d4 = ld4(&sm.cd[4 * l]);
-    const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+    const float2 d0 = f2(d4.x, d4.y), d1 = f2(d4.z, d4.w);
 #pragma unroll
     for (int rr = 0; rr < kRowsPerWarp; rr++) {
         const int i = kRowsPerWarp * w + rr;
-        const float g = sm.rg[i];
-        const __half2 h0 = __floats2half2_rn(fmaf(g, dd[0], X[rr][0]), fmaf(g, dd[1], X[rr][1]));
-        const __half2 h1 = __floats2half2_rn(fmaf(g, dd[2], X[rr][2]), fmaf(g, dd[3], X[rr][3]));
+        const float2 gg = ld2(&sm.rg2[i]);
+        const float2 s0 = __ffma2_rn(gg, d0, X[rr][0]), s1 = __ffma2_rn(gg, d1, X[rr][1]);
+        const __half2 h0 = __floats2half2_rn(s0.x, s0.y);
+        const __half2 h1 = __floats2half2_rn(s1.x, s1.y);
         words[(2 * rr) * kGroups] = *reinterpret_cast<const uint32_t *>(&h0);
         words[(2 * rr + 1) * kGroups] = *reinterpret_cast<const uint32_t *>(&h1);
     }
@@ -423,8 +476,8 @@ __device__ __forceinline__ void stage_item(const StepArgs &a, int4 st, uint8_t *
 // Producer state, held by thread 0: the next position to stage and its record,
 // loaded one issue ahead so that no global load sits on the critical path.
 struct Producer {
-    int n;          // next position to stage
-    int4 rec;       // its staging record
+    int n;  // next position to stage
+    int4 rec;
     uint32_t issued;
     __device__ __forceinline__ void load(const StepArgs &a)
     {
@@ -432,6 +485,7 @@ struct Producer {
     }
 };
 
+// Phase 0 of a staged item: per-row and per-column factors from the slot.
 template <bool KDA>
 __device__ __forceinline__ void phase0(ItemSmem &sm, const StepArgs &a, const uint8_t *sb)
 {
@@ -447,24 +501,25 @@ __device__ __forceinline__ void phase0(ItemSmem &sm, const StepArgs &a, const ui
                              : *reinterpret_cast<const float *>(sb + a.off_ab);
         const float k = reinterpret_cast<const float *>(sb + a.off_k)[i];
         const float q = reinterpret_cast<const float *>(sb + a.off_q)[i];
+        float A, g, qi = 0.f, s = 0.f, rh = 0.f;
         if (b == kPivotBits) {
-            sm.rk[i] = al * k;
-            sm.rl[i] = al * q;
-            sm.rg[i] = beta * k;
-            sm.ra[i] = al;
-            sm.rs[i] = 0.f;
-            sm.rrho[i] = 0.f;
-            sm.rqi[i] = 0.f;
+            A = al;
+            g = beta * k;
         } else {
-            const float A = al * s_r[i];
-            sm.rk[i] = A * k;
-            sm.rl[i] = A * q;
-            sm.rg[i] = __fdiv_rn(beta * k, A);
-            sm.ra[i] = A;
-            sm.rs[i] = rec->s[i];
-            sm.rrho[i] = rec->rho[i];
-            sm.rqi[i] = __frcp_rn((float)qmax_of(b));
+            A = al * s_r[i];
+            g = __fdiv_rn(beta * k, A);
+            qi = __frcp_rn((float)qmax_of(b));
+            s = rec->s[i];
+            rh = rec->rho[i];
         }
+        sm.rk2[i] = f2(A * k, A * k);
+        sm.rl2[i] = f2(A * q, A * q);
+        sm.rg2[i] = f2(g, g);
+        sm.ra2[i] = f2(al, al);
+        sm.rq2[i] = f2(qi, qi);
+        sm.ra[i] = A;
+        sm.rs[i] = s;
+        sm.rrho[i] = rh;
         sm.rb[i] = b;
         float kq = k * q;
 #pragma unroll
@@ -491,48 +546,43 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
                                          Producer &prod, uint8_t *ring)
 {
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    const int r0 = kRowsPerWarp * w;
     constexpr bool ROWWISE = (B == 0);
-    float X[kRowsPerWarp][4];
+    X2 X;
     // ---- phase A: codes -> floats, key and query projections ---------------
     decode_stream<B>(sm, reinterpret_cast<const uint32_t *>(sb + sm.tile_off[w]) + l, kGroups, X);
-    float cj[4], icj[4];
+    const float4 c4 = ld4(&sm.cc[4 * l]);
+    const float2 c0 = f2(c4.x, c4.y), c1 = f2(c4.z, c4.w);
     {
-        const float4 c4 = ld4(&sm.cc[4 * l]);
-        cj[0] = c4.x; cj[1] = c4.y; cj[2] = c4.z; cj[3] = c4.w;
+        float2 V0 = f2(0.f, 0.f), V1 = V0, U0 = V0, U1 = V0;
+        float2 ic0 = V0, ic1 = V0;
+        if (ROWWISE) {
+            ic0 = f2(rcp_approx(c4.x), rcp_approx(c4.y));
+            ic1 = f2(rcp_approx(c4.z), rcp_approx(c4.w));
+        }
 #pragma unroll
-        for (int kk = 0; kk < 4; kk++) icj[kk] = ROWWISE ? __frcp_rn(cj[kk]) : 0.f;
-    }
-    {
-        float V[4] = {0.f, 0.f, 0.f, 0.f}, U[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int r4 = 0; r4 < kRowsPerWarp; r4 += 4) {
-            const float4 k4 = ld4(&sm.rk[kRowsPerWarp * w + r4]);
-            const float4 l4 = ld4(&sm.rl[kRowsPerWarp * w + r4]);
-            const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const int rr = r4 + u, i = kRowsPerWarp * w + rr;
-                if (ROWWISE && sm.rb[i] == kPivotBits) {
-                    const float al = sm.ra[i];
-#pragma unroll
-                    for (int kk = 0; kk < 4; kk++) {
-                        const float hs = X[rr][kk] * icj[kk];  // pivot value in units of c_j
-                        V[kk] = fmaf(kv[u], hs, V[kk]);
-                        U[kk] = fmaf(lv[u], hs, U[kk]);
-                        X[rr][kk] = al * X[rr][kk];           // S' = alpha h
-                    }
-                } else {
-#pragma unroll
-                    for (int kk = 0; kk < 4; kk++) {
-                        V[kk] = fmaf(kv[u], X[rr][kk], V[kk]);
-                        U[kk] = fmaf(lv[u], X[rr][kk], U[kk]);
-                    }
-                }
+        for (int rr = 0; rr < kRowsPerWarp; rr++) {
+            const int i = r0 + rr;
+            const float2 kk = ld2(&sm.rk2[i]), ll = ld2(&sm.rl2[i]);
+            if (ROWWISE && sm.rb[i] == kPivotBits) {
+                // a pivot value enters the projections in units of c_j; S' = alpha h
+                const float2 hs0 = __fmul2_rn(X[rr][0], ic0), hs1 = __fmul2_rn(X[rr][1], ic1);
+                V0 = __ffma2_rn(kk, hs0, V0);
+                V1 = __ffma2_rn(kk, hs1, V1);
+                U0 = __ffma2_rn(ll, hs0, U0);
+                U1 = __ffma2_rn(ll, hs1, U1);
+                const float2 aa = ld2(&sm.ra2[i]);
+                X[rr][0] = __fmul2_rn(aa, X[rr][0]);
+                X[rr][1] = __fmul2_rn(aa, X[rr][1]);
+            } else {
+                V0 = __ffma2_rn(kk, X[rr][0], V0);
+                V1 = __ffma2_rn(kk, X[rr][1], V1);
+                U0 = __ffma2_rn(ll, X[rr][0], U0);
+                U1 = __ffma2_rn(ll, X[rr][1], U1);
             }
         }
-        stash_partials(sm, 0, V);
-        stash_partials(sm, 1, U);
+        stash(sm, 0, V0, V1);
+        stash(sm, 1, U0, U1);
     }
     __syncthreads();
     // the slot has been read by every thread: stage the next item into it
@@ -547,7 +597,7 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
         const float c = sm.cc[j];
         const float d = sm.cv[j] - c * sum_partials(sm, 0, j);
         sm.cd[j] = d;
-        sm.cdt[j] = __fdiv_rn(d, c);
+        sm.cdt[j] = div_approx(d, c);
     } else {
         const int j = tid - kDK;
         sm.cu[j] = sm.cc[j] * sum_partials(sm, 1, j);
@@ -560,23 +610,23 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
     // ---- phase B: Delta update in old-scale units; P = S / a ----------------
     {
         const float4 t4 = ld4(&sm.cdt[4 * l]);
-        const float4 d4 = ld4(&sm.cd[4 * l]);
-        const float dt[4] = {t4.x, t4.y, t4.z, t4.w};
-        const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+        const float2 dt0 = f2(t4.x, t4.y), dt1 = f2(t4.z, t4.w);
+        float2 dd0 = dt0, dd1 = dt1;
+        if (ROWWISE) {
+            const float4 d4 = ld4(&sm.cd[4 * l]);
+            dd0 = f2(d4.x, d4.y);
+            dd1 = f2(d4.z, d4.w);
+        }
 #pragma unroll
-        for (int r4 = 0; r4 < kRowsPerWarp; r4 += 4) {
-            const float4 g4 = ld4(&sm.rg[kRowsPerWarp * w + r4]);
-            const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-#pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const int rr = r4 + u, i = kRowsPerWarp * w + rr;
-                if (ROWWISE && sm.rb[i] == kPivotBits) {
-#pragma unroll
-                    for (int kk = 0; kk < 4; kk++) X[rr][kk] = fmaf(gv[u], dd[kk], X[rr][kk]);
-                } else {
-#pragma unroll
-                    for (int kk = 0; kk < 4; kk++) X[rr][kk] = cj[kk] * fmaf(gv[u], dt[kk], X[rr][kk]);
-                }
+        for (int rr = 0; rr < kRowsPerWarp; rr++) {
+            const int i = r0 + rr;
+            const float2 gg = ld2(&sm.rg2[i]);
+            if (ROWWISE && sm.rb[i] == kPivotBits) {
+                X[rr][0] = __ffma2_rn(gg, dd0, X[rr][0]);
+                X[rr][1] = __ffma2_rn(gg, dd1, X[rr][1]);
+            } else {
+                X[rr][0] = __fmul2_rn(c0, __ffma2_rn(gg, dt0, X[rr][0]));
+                X[rr][1] = __fmul2_rn(c1, __ffma2_rn(gg, dt1, X[rr][1]));
             }
         }
     }
@@ -641,27 +691,23 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
             __syncthreads();
             return;
         }
-        const int hb = sm.head_b;
-        // dispatch on the head's row width
-#define STEPQ_ITEM_CASE(BB)                                                        \
-    case BB:                                                                       \
-        run_item<BB, KDA>(sm, a, item, sb, slot, prod, ring);         \
-        break;
         if (KDA) {
             run_item<0, KDA>(sm, a, item, sb, slot, prod, ring);
         } else {
-            switch (hb) {
-                STEPQ_ITEM_CASE(2)
-                STEPQ_ITEM_CASE(3)
-                STEPQ_ITEM_CASE(4)
-                STEPQ_ITEM_CASE(5)
-                STEPQ_ITEM_CASE(6)
-                STEPQ_ITEM_CASE(7)
-                STEPQ_ITEM_CASE(8)
-                default: run_item<0, KDA>(sm, a, item, sb, slot, prod, ring); break;
+            switch (sm.head_b) {
+                case 2: run_item<2, KDA>(sm, a, item, sb, slot, prod, ring); break;
+                case 3: run_item<3, KDA>(sm, a, item, sb, slot, prod, ring); break;
+                case 4: run_item<4, KDA>(sm, a, item, sb, slot, prod, ring); break;
+                case 5: run_item<5, KDA>(sm, a, item, sb, slot, prod, ring); break;
+                case 6: run_item<6, KDA>(sm, a, item, sb, slot, prod, ring); break;
+                case 7: run_item<7, KDA>(sm, a, item, sb, slot, prod, ring); break;
+                case 8: run_item<8, KDA>(sm, a, item, sb, slot, prod, ring); break;
+                default:  // unreachable: Gated-DeltaNet heads have one width, validated on the host
+                    if (tid == 0) atomicExch(a.t.status, kStatusBadHead);
+                    __syncthreads();
+                    break;
             }
         }
-#undef STEPQ_ITEM_CASE
     }
 }
 
@@ -675,11 +721,12 @@ __device__ __forceinline__ void load_head(ItemSmem &sm, const StepArgs &a, int h
     const HeadRec *rec = a.t.rowrec + h;
     if (tid < kDK) {
         const int i = tid, b = rec->bits[i];
+        const float qi = (b == kPivotBits) ? 0.f : __frcp_rn((float)qmax_of(b));
         sm.rb[i] = b;
         sm.ra[i] = 1.f;
         sm.rs[i] = rec->s[i];
         sm.rrho[i] = rec->rho[i];
-        sm.rqi[i] = (b == kPivotBits) ? 0.f : __frcp_rn((float)qmax_of(b));
+        sm.rq2[i] = f2(qi, qi);
     } else {
         const int j = tid - kDK;
         if (j < kTiles) sm.tile_off[j] = rec->tile_off[j];
@@ -695,12 +742,13 @@ template <int B, bool ROWWISE>
 __device__ __forceinline__ void pack_body(ItemSmem &sm, const StepArgs &a, int item, uint8_t *item_g)
 {
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    float X[kRowsPerWarp][4];
+    X2 X;
     const float *src = a.S_in + (long long)item * kDK * kDV;
 #pragma unroll
     for (int rr = 0; rr < kRowsPerWarp; rr++) {
         const float4 x = ld4(src + (kRowsPerWarp * w + rr) * kDV + 4 * l);
-        X[rr][0] = x.x; X[rr][1] = x.y; X[rr][2] = x.z; X[rr][3] = x.w;
+        X[rr][0] = f2(x.x, x.y);
+        X[rr][1] = f2(x.z, x.w);
     }
     fit_and_store<B, ROWWISE>(sm, X, item_g, a.ls_iters);
 }
@@ -729,25 +777,23 @@ template <int B>
 __device__ __forceinline__ void unpack_body(ItemSmem &sm, const StepArgs &a, int item, const uint8_t *item_g)
 {
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    float X[kRowsPerWarp][4];
+    X2 X;
     decode_stream<B>(sm, reinterpret_cast<const uint32_t *>(item_g + sm.tile_off[w]) + l, kGroups, X);
     const float *r = reinterpret_cast<const float *>(item_g);
     const float4 c4 = ld4(r + kDK + 4 * l);
-    const float cj[4] = {c4.x, c4.y, c4.z, c4.w};
     float *dst = a.S_out + (long long)item * kDK * kDV;
 #pragma unroll
     for (int rr = 0; rr < kRowsPerWarp; rr++) {
         const int i = kRowsPerWarp * w + rr;
-        float y[4];
+        float4 y;
         if (B == 0 && sm.rb[i] == kPivotBits) {
-#pragma unroll
-            for (int kk = 0; kk < 4; kk++) y[kk] = X[rr][kk];
+            y = make_float4(X[rr][0].x, X[rr][0].y, X[rr][1].x, X[rr][1].y);
         } else {
             const float ri = r[i];
-#pragma unroll
-            for (int kk = 0; kk < 4; kk++) y[kk] = __fmul_rn(__fmul_rn(ri, cj[kk]), X[rr][kk]);
+            y = make_float4(__fmul_rn(__fmul_rn(ri, c4.x), X[rr][0].x), __fmul_rn(__fmul_rn(ri, c4.y), X[rr][0].y),
+                            __fmul_rn(__fmul_rn(ri, c4.z), X[rr][1].x), __fmul_rn(__fmul_rn(ri, c4.w), X[rr][1].y));
         }
-        *reinterpret_cast<float4 *>(dst + i * kDV + 4 * l) = make_float4(y[0], y[1], y[2], y[3]);
+        *reinterpret_cast<float4 *>(dst + i * kDV + 4 * l) = y;
     }
 }
 
@@ -878,7 +924,8 @@ int decode_ctas_per_sm(int nslots, int slot_bytes)
     const int dyn = nslots * slot_bytes;
     int per_sm = 0;
     if (cudaFuncSetAttribute(k_decode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<false>, kThreads, dyn) != cudaSuccess) {
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<false>, kThreads, dyn) != cudaSuccess ||
+        cudaFuncSetAttribute(k_decode<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess) {
         cudaGetLastError();
         return 0;
     }
