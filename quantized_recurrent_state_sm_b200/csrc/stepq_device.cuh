@@ -114,6 +114,17 @@ __device__ __forceinline__ void field_put(uint32_t *w, int c, uint32_t u)
     if (sh + B > 32) w[lo + 1] |= u >> (32 - sh);
 }
 
+// OR the low B bits of `bits` into position c of words w[] (the masking and
+// the merge are one logic operation per word touched).
+template <int B>
+__device__ __forceinline__ void field_put_bits(uint32_t *w, int c, uint32_t bits)
+{
+    const int pos = c * B, lo = pos >> 5, sh = pos & 31;
+    constexpr uint32_t mask = (1u << B) - 1u;
+    w[lo] |= (bits << sh) & (mask << sh);
+    if (sh + B > 32) w[lo + 1] |= (bits & mask) >> (32 - sh);
+}
+
 // Variable-width reader over stream words fetched on demand from shared memory
 // (word m of the stream at base[m * stride]).
 struct BitReader {

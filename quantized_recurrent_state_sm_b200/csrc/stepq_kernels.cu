@@ -51,6 +51,9 @@ struct alignas(16) ItemSmem {
     int head_b, head_kind;
     long long head_off;
     uint64_t bar[kMaxSlots];
+    int4 prod_rec;          // producer (thread 0): staging record of position prod_n
+    int prod_n;             // producer: next position to stage
+    uint32_t prod_issued;   // producer: items staged so far
 };
 
 using X2 = float2[kRowsPerWarp][2];  // the thread's 16 x 4 block as float2 pairs
@@ -110,6 +113,29 @@ __device__ __forceinline__ float max_partials(const ItemSmem &sm, int vec, int j
     return acc;
 }
 
+// Half of a column reduction: the partials of warps 4 half .. 4 half + 3.
+__device__ __forceinline__ float sum_partials4(const ItemSmem &sm, int vec, int j, int half)
+{
+    const float a = sm.red[vec][4 * half][j], b = sm.red[vec][4 * half + 1][j];
+    const float c = sm.red[vec][4 * half + 2][j], d = sm.red[vec][4 * half + 3][j];
+    return (a + b) + (c + d);
+}
+
+__device__ __forceinline__ float max_partials4(const ItemSmem &sm, int vec, int j, int half)
+{
+    const float a = sm.red[vec][4 * half][j], b = sm.red[vec][4 * half + 1][j];
+    const float c = sm.red[vec][4 * half + 2][j], d = sm.red[vec][4 * half + 3][j];
+    return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+// The duplicated factors of two consecutive rows (p 16-byte aligned) in one load.
+__device__ __forceinline__ void ld_pairs(const float2 *p, float2 (&out)[2])
+{
+    const float4 v = *reinterpret_cast<const float4 *>(p);
+    out[0] = make_float2(v.x, v.y);
+    out[1] = make_float2(v.z, v.w);
+}
+
 // ---------------------------------------------------------------------------
 // Decode the thread's column-group stream of its tile into X (code values as
 // floats; pivot rows: their binary16 values).  Fixed width B > 0 keeps the
@@ -161,6 +187,100 @@ __device__ __forceinline__ void decode_stream(const ItemSmem &sm, const uint32_t
     }
 }
 
+// One least-squares round's partial sums over the thread's rows, stashed for
+// the column reduction: with n = rne(p / c) (clipped to the row's range when
+// CLIP), N_j = sum w_i n_ij p_ij and D_j = sum w_i n_ij^2.
+template <int B, bool ROWWISE, bool CLIP>
+__device__ __forceinline__ void ls_partials(ItemSmem &sm, const X2 &X)
+{
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    const int r0 = kRowsPerWarp * w;
+    const float2 rm2 = f2(kRoundMagic, kRoundMagic), nrm2 = f2(-kRoundMagic, -kRoundMagic);
+    const float4 i4 = ld4(&sm.ci[4 * l]);
+    const float2 ic0 = f2(i4.x, i4.y), ic1 = f2(i4.z, i4.w);
+    float2 N0 = f2(0.f, 0.f), N1 = N0, D0 = N0, D1 = N0;
+#pragma unroll
+    for (int rr = 0; rr < kRowsPerWarp; rr += 2) {
+        float2 wp[2];
+        ld_pairs(&sm.rw2[r0 + rr], wp);
+#pragma unroll
+        for (int u = 0; u < 2; u++) {
+            const int i = r0 + rr + u;
+            if (ROWWISE && sm.rb[i] == kPivotBits) continue;
+            // round to the nearest integer, ties to even: x + 1.5 * 2^23 - 1.5 * 2^23;
+            // clipping acts on the biased value (for a fixed width the bounds are
+            // immediates)
+            float2 m0 = __ffma2_rn(X[rr + u][0], ic0, rm2);
+            float2 m1 = __ffma2_rn(X[rr + u][1], ic1, rm2);
+            if (CLIP) {
+                const float Q = (float)qmax_of(ROWWISE ? sm.rb[i] : B);
+                const float lo = kRoundMagic - Q, hi = kRoundMagic + Q;
+                m0 = f2(fminf(fmaxf(m0.x, lo), hi), fminf(fmaxf(m0.y, lo), hi));
+                m1 = f2(fminf(fmaxf(m1.x, lo), hi), fminf(fmaxf(m1.y, lo), hi));
+            }
+            const float2 n0 = __fadd2_rn(m0, nrm2), n1 = __fadd2_rn(m1, nrm2);
+            const float2 wn0 = __fmul2_rn(wp[u], n0), wn1 = __fmul2_rn(wp[u], n1);
+            N0 = __ffma2_rn(wn0, X[rr + u][0], N0);
+            N1 = __ffma2_rn(wn1, X[rr + u][1], N1);
+            D0 = __ffma2_rn(wn0, n0, D0);
+            D1 = __ffma2_rn(wn1, n1, D1);
+        }
+    }
+    stash(sm, 0, N0, N1);
+    stash(sm, 1, D0, D1);
+}
+
+// The least-squares column scales from the stashed partials, two threads per
+// column: c_j = N_j / D_j (kept when D_j = 0), its reciprocal, and c0_j / c_j.
+__device__ __forceinline__ void ls_update_columns(ItemSmem &sm)
+{
+    const int j = threadIdx.x >> 1, half = threadIdx.x & 1;
+    float nn = sum_partials4(sm, 0, j, half), dd = sum_partials4(sm, 1, j, half);
+    nn += __shfl_xor_sync(0xffffffffu, nn, 1);
+    dd += __shfl_xor_sync(0xffffffffu, dd, 1);
+    if (half == 0) {
+        const float c = (dd > 0.f) ? div_approx(nn, dd) : sm.cnew[j];
+        const float icn = rcp_approx(c);
+        sm.cnew[j] = c;
+        sm.ci[j] = icn;
+        sm.crat[j] = sm.cc0[j] * icn;
+    }
+}
+
+// Final codes of a fixed-width tile stream and their store: u = z + clip(rne(p / c))
+// taken from the low mantissa bits of p / c + 2^23 + z; each 32-bit word is
+// stored as soon as its last code is placed.
+template <int B, bool CLIP>
+__device__ __forceinline__ void pack_fixed(const X2 &X, float2 ic0, float2 ic1, uint32_t *words)
+{
+    constexpr int Qb = (1 << (B - 1)) - 1;
+    const float mz = kMagic + (float)(1 << (B - 1));
+    const float2 mz2 = f2(mz, mz);
+    uint32_t ow[2 * B + 1];
+#pragma unroll
+    for (int m = 0; m <= 2 * B; m++) ow[m] = 0u;
+#pragma unroll
+    for (int rr = 0; rr < kRowsPerWarp; rr++)
+#pragma unroll
+        for (int hh = 0; hh < 2; hh++) {
+            float2 mm;
+            if (!CLIP) {
+                mm = __ffma2_rn(X[rr][hh], hh ? ic1 : ic0, mz2);
+            } else {
+                float2 t = __fmul2_rn(X[rr][hh], hh ? ic1 : ic0);
+                t = f2(fminf(fmaxf(t.x, -(float)Qb), (float)Qb), fminf(fmaxf(t.y, -(float)Qb), (float)Qb));
+                mm = __fadd2_rn(t, mz2);
+            }
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+                const int c = 4 * rr + 2 * hh + e;
+                field_put_bits<B>(ow, c, __float_as_uint(e ? mm.y : mm.x));
+#pragma unroll
+                for (int m = (c * B) / 32; m < ((c + 1) * B) / 32; m++) words[m * kGroups] = ow[m];
+            }
+        }
+}
+
 // ---------------------------------------------------------------------------
 // The fit (row scales, column scales, least squares), requantisation and the
 // packed store.  On entry X holds P_ij = S_ij / a_i on quantised rows and S_ij
@@ -168,11 +288,15 @@ __device__ __forceinline__ void decode_stream(const ItemSmem &sm, const uint32_t
 // Writes r', c and the item's streams at item_g.  Contains __syncthreads.
 // ROWWISE: rows may differ in width and may be pivots.
 // ---------------------------------------------------------------------------
-template <int B, bool ROWWISE>
-__device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item_g, int ls_iters)
+template <int B, bool ROWWISE, bool MULTI>
+__device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item_g, int ls_iters,
+                                              bool store_c = true)
 {
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int r0 = kRowsPerWarp * w;
+    // read now: the next item's phase 0 may rewrite them while this item's last
+    // phase still runs
+    const uint32_t tile_off = sm.tile_off[w];
     // ---- row magnitudes: sum over the 128 columns of P^2 -------------------
     {
         float *t = &sm.rowt[w][0][0];
@@ -214,19 +338,18 @@ __device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item
         float mx[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int rr = 0; rr < kRowsPerWarp; rr += 2) {
-            float2 p[2][2];
+            float2 p[2][2], hh[2], qq[2];
+            ld_pairs(&sm.rh2[r0 + rr], hh);
+            if (ROWWISE) ld_pairs(&sm.rq2[r0 + rr], qq);
 #pragma unroll
             for (int u = 0; u < 2; u++) {
-                const int i = r0 + rr + u;
-                const float2 hh = ld2(&sm.rh2[i]);
-                p[u][0] = __fmul2_rn(X[rr + u][0], hh);
-                p[u][1] = __fmul2_rn(X[rr + u][1], hh);
+                p[u][0] = __fmul2_rn(X[rr + u][0], hh[u]);
+                p[u][1] = __fmul2_rn(X[rr + u][1], hh[u]);
                 X[rr + u][0] = p[u][0];
                 X[rr + u][1] = p[u][1];
                 if (ROWWISE) {  // pivot rows have rq2 = 0 and do not count
-                    const float2 qq = ld2(&sm.rq2[i]);
-                    p[u][0] = __fmul2_rn(p[u][0], qq);
-                    p[u][1] = __fmul2_rn(p[u][1], qq);
+                    p[u][0] = __fmul2_rn(p[u][0], qq[u]);
+                    p[u][1] = __fmul2_rn(p[u][1], qq[u]);
                 }
             }
             mx[0] = max_abs3(mx[0], p[0][0].x, p[1][0].x);
@@ -237,56 +360,42 @@ __device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item
         stash(sm, 0, f2(mx[0], mx[1]), f2(mx[2], mx[3]));
     }
     __syncthreads();
-    if (tid < kDV) {
-        const int j = tid;
-        float m = max_partials(sm, 0, j);
-        if (!ROWWISE) m = m * sm.rq2[0].x;  // every row has the head's width
-        const float c0 = (m > 0.f) ? m : 1.f;
-        sm.cc0[j] = c0;
-        sm.cnew[j] = c0;
-        sm.ci[j] = rcp_approx(c0);
-        sm.crat[j] = 1.f;
+    {
+        // two threads per column, each over four warps' partials
+        const int j = tid >> 1, half = tid & 1;
+        float m = max_partials4(sm, 0, j, half);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        if (half == 0) {
+            if (!ROWWISE) m = m * sm.rq2[0].x;  // every row has the head's width
+            const float c0 = (m > 0.f) ? m : 1.f;
+            sm.cc0[j] = c0;
+            sm.cnew[j] = c0;
+            sm.ci[j] = rcp_approx(c0);
+            sm.crat[j] = 1.f;
+        }
     }
     __syncthreads();
     // ---- impact-weighted least squares for the column scales ---------------
-    const float2 rm2 = f2(kRoundMagic, kRoundMagic), nrm2 = f2(-kRoundMagic, -kRoundMagic);
-    for (int it = 0; it < ls_iters; it++) {
-        const float4 i4 = ld4(&sm.ci[4 * l]);
-        const float2 ic0 = f2(i4.x, i4.y), ic1 = f2(i4.z, i4.w);
-        float2 N0 = f2(0.f, 0.f), N1 = N0, D0 = N0, D1 = N0;
-#pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; rr++) {
-            const int i = r0 + rr;
-            if (ROWWISE && sm.rb[i] == kPivotBits) continue;
-            const float2 ww = ld2(&sm.rw2[i]);
-            // round p / c to the nearest integer: |p / c0| <= Q, so no clipping in
-            // the first round; later rounds clip to the row's range
-            float2 n0 = __fadd2_rn(__ffma2_rn(X[rr][0], ic0, rm2), nrm2);
-            float2 n1 = __fadd2_rn(__ffma2_rn(X[rr][1], ic1, rm2), nrm2);
-            if (it > 0) {
-                const float Q = (float)qmax_of(ROWWISE ? sm.rb[i] : B);
-                n0 = f2(fminf(fmaxf(n0.x, -Q), Q), fminf(fmaxf(n0.y, -Q), Q));
-                n1 = f2(fminf(fmaxf(n1.x, -Q), Q), fminf(fmaxf(n1.y, -Q), Q));
-            }
-            const float2 wn0 = __fmul2_rn(ww, n0), wn1 = __fmul2_rn(ww, n1);
-            N0 = __ffma2_rn(wn0, X[rr][0], N0);
-            N1 = __ffma2_rn(wn1, X[rr][1], N1);
-            D0 = __ffma2_rn(wn0, n0, D0);
-            D1 = __ffma2_rn(wn1, n1, D1);
+    // |p / c0| <= Q, so the first round needs no clipping; later rounds clip to
+    // the row's range.  More than one round is a separate instantiation (MULTI)
+    // so that the one-round code holds a single round body.
+    if (!MULTI) {
+        if (ls_iters > 0) {
+            ls_partials<B, ROWWISE, false>(sm, X);
+            __syncthreads();
+            ls_update_columns(sm);
+            __syncthreads();
         }
-        stash(sm, 0, N0, N1);
-        stash(sm, 1, D0, D1);
-        __syncthreads();
-        if (tid < kDV) {
-            const int j = tid;
-            const float nn = sum_partials(sm, 0, j), dd = sum_partials(sm, 1, j);
-            const float c = (dd > 0.f) ? div_approx(nn, dd) : sm.cnew[j];
-            const float icn = rcp_approx(c);
-            sm.cnew[j] = c;
-            sm.ci[j] = icn;
-            sm.crat[j] = sm.cc0[j] * icn;
+    } else {
+        for (int it = 0; it < ls_iters; it++) {
+            if (it == 0)
+                ls_partials<B, ROWWISE, false>(sm, X);
+            else
+                ls_partials<B, ROWWISE, true>(sm, X);
+            __syncthreads();
+            ls_update_columns(sm);
+            __syncthreads();
         }
-        __syncthreads();
     }
     // ---- requantise, pack, store -------------------------------------------
     const float4 i4 = ld4(&sm.ci[4 * l]);
@@ -299,37 +408,13 @@ __device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item
     // the largest |p / c| of a column is at most Q c0 / c: clip only where that
     // can reach Q + 1/2
     rat = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(rat)));
-    uint32_t *words = reinterpret_cast<uint32_t *>(item_g + sm.tile_off[w]) + l;
+    uint32_t *words = reinterpret_cast<uint32_t *>(item_g + tile_off) + l;
     if constexpr (B > 0) {
         constexpr int Qb = (1 << (B - 1)) - 1;
-        constexpr uint32_t mask = (1u << B) - 1u;
-        const bool clip = (float)Qb * (rat - 1.f) >= 0.49f;
-        const float mz = kMagic + (float)(1 << (B - 1));
-        const float2 mz2 = f2(mz, mz);
-        uint32_t ow[2 * B + 1];
-#pragma unroll
-        for (int m = 0; m <= 2 * B; m++) ow[m] = 0u;
-#pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; rr++)
-#pragma unroll
-            for (int hh = 0; hh < 2; hh++) {
-                float2 mm;
-                if (!clip) {
-                    mm = __ffma2_rn(X[rr][hh], hh ? ic1 : ic0, mz2);
-                } else {
-                    float2 t = __fmul2_rn(X[rr][hh], hh ? ic1 : ic0);
-                    t = f2(fminf(fmaxf(t.x, -(float)Qb), (float)Qb), fminf(fmaxf(t.y, -(float)Qb), (float)Qb));
-                    mm = __fadd2_rn(t, mz2);
-                }
-#pragma unroll
-                for (int e = 0; e < 2; e++) {
-                    const int c = 4 * rr + 2 * hh + e;
-                    field_put<B>(ow, c, __float_as_uint(e ? mm.y : mm.x) & mask);
-                    // store every word the code completed (known at compile time)
-#pragma unroll
-                    for (int m = (c * B) / 32; m < ((c + 1) * B) / 32; m++) words[m * kGroups] = ow[m];
-                }
-            }
+        if ((float)Qb * (rat - 1.f) >= 0.49f)
+            pack_fixed<B, true>(X, ic0, ic1, words);
+        else
+            pack_fixed<B, false>(X, ic0, ic1, words);
     } else {
         BitWriter bw;
         bw.init(words, kGroups);
@@ -367,8 +452,7 @@ __device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item
         }
         bw.flush();
     }
-    if (tid < kDV)
-        reinterpret_cast<float *>(item_g)[kDK + tid] = (sm.head_kind == kHeadAllPivot) ? 0.f : sm.cnew[tid];
+    if (tid < kDV) reinterpret_cast<float *>(item_g)[kDK + tid] = store_c ? sm.cnew[tid] : 0.f;
 }
 
 // ---------------------------------------------------------------------------
@@ -473,17 +557,29 @@ __device__ __forceinline__ void stage_item(const StepArgs &a, int4 st, uint8_t *
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// Producer state, held by thread 0: the next position to stage and its record,
-// loaded one issue ahead so that no global load sits on the critical path.
-struct Producer {
-    int n;  // next position to stage
-    int4 rec;
-    uint32_t issued;
-    __device__ __forceinline__ void load(const StepArgs &a)
-    {
-        if (n < a.n_items) rec = a.t.stage[n];
-    }
-};
+// Producer state, used by thread 0 only and kept in shared memory so that it
+// costs no registers in the other threads: the next position to stage, the
+// number staged so far, and that position's staging record, fetched one issue
+// ahead with an asynchronous copy so that no global load stalls the thread.
+__device__ __forceinline__ void prefetch_stage_rec(ItemSmem &sm, const StepArgs &a)
+{
+    if (sm.prod_n < a.n_items)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_addr(&sm.prod_rec)),
+                     "l"(a.t.stage + sm.prod_n)
+                     : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Stage the next position into slot buffer sb (thread 0).
+template <bool KDA>
+__device__ __forceinline__ void produce(ItemSmem &sm, const StepArgs &a, uint8_t *sb, uint64_t *bar)
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    stage_item<KDA>(a, sm.prod_rec, sb, bar);
+    sm.prod_n += gridDim.x;
+    sm.prod_issued++;
+    prefetch_stage_rec(sm, a);
+}
 
 // Phase 0 of a staged item: per-row and per-column factors from the slot.
 template <bool KDA>
@@ -541,9 +637,9 @@ __device__ __forceinline__ void phase0(ItemSmem &sm, const StepArgs &a, const ui
 
 // Phases after phase 0 of a staged item: reconstruct + project, release the
 // slot (stage the next item into it), Delta update, readout, fit, store.
-template <int B, bool KDA>
+template <int B, bool KDA, bool MULTI>
 __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int item, const uint8_t *sb, int slot,
-                                         Producer &prod, uint8_t *ring)
+                                         uint8_t *ring)
 {
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int r0 = kRowsPerWarp * w;
@@ -551,9 +647,8 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
     X2 X;
     // ---- phase A: codes -> floats, key and query projections ---------------
     decode_stream<B>(sm, reinterpret_cast<const uint32_t *>(sb + sm.tile_off[w]) + l, kGroups, X);
-    const float4 c4 = ld4(&sm.cc[4 * l]);
-    const float2 c0 = f2(c4.x, c4.y), c1 = f2(c4.z, c4.w);
     {
+        const float4 c4 = ld4(&sm.cc[4 * l]);
         float2 V0 = f2(0.f, 0.f), V1 = V0, U0 = V0, U1 = V0;
         float2 ic0 = V0, ic1 = V0;
         if (ROWWISE) {
@@ -561,24 +656,29 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
             ic1 = f2(rcp_approx(c4.z), rcp_approx(c4.w));
         }
 #pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; rr++) {
-            const int i = r0 + rr;
-            const float2 kk = ld2(&sm.rk2[i]), ll = ld2(&sm.rl2[i]);
-            if (ROWWISE && sm.rb[i] == kPivotBits) {
-                // a pivot value enters the projections in units of c_j; S' = alpha h
-                const float2 hs0 = __fmul2_rn(X[rr][0], ic0), hs1 = __fmul2_rn(X[rr][1], ic1);
-                V0 = __ffma2_rn(kk, hs0, V0);
-                V1 = __ffma2_rn(kk, hs1, V1);
-                U0 = __ffma2_rn(ll, hs0, U0);
-                U1 = __ffma2_rn(ll, hs1, U1);
-                const float2 aa = ld2(&sm.ra2[i]);
-                X[rr][0] = __fmul2_rn(aa, X[rr][0]);
-                X[rr][1] = __fmul2_rn(aa, X[rr][1]);
-            } else {
-                V0 = __ffma2_rn(kk, X[rr][0], V0);
-                V1 = __ffma2_rn(kk, X[rr][1], V1);
-                U0 = __ffma2_rn(ll, X[rr][0], U0);
-                U1 = __ffma2_rn(ll, X[rr][1], U1);
+        for (int r2 = 0; r2 < kRowsPerWarp; r2 += 2) {
+            float2 kp[2], lp[2];
+            ld_pairs(&sm.rk2[r0 + r2], kp);
+            ld_pairs(&sm.rl2[r0 + r2], lp);
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                const int rr = r2 + u, i = r0 + rr;
+                if (ROWWISE && sm.rb[i] == kPivotBits) {
+                    // a pivot value enters the projections in units of c_j; S' = alpha h
+                    const float2 hs0 = __fmul2_rn(X[rr][0], ic0), hs1 = __fmul2_rn(X[rr][1], ic1);
+                    V0 = __ffma2_rn(kp[u], hs0, V0);
+                    V1 = __ffma2_rn(kp[u], hs1, V1);
+                    U0 = __ffma2_rn(lp[u], hs0, U0);
+                    U1 = __ffma2_rn(lp[u], hs1, U1);
+                    const float2 aa = ld2(&sm.ra2[i]);
+                    X[rr][0] = __fmul2_rn(aa, X[rr][0]);
+                    X[rr][1] = __fmul2_rn(aa, X[rr][1]);
+                } else {
+                    V0 = __ffma2_rn(kp[u], X[rr][0], V0);
+                    V1 = __ffma2_rn(kp[u], X[rr][1], V1);
+                    U0 = __ffma2_rn(lp[u], X[rr][0], U0);
+                    U1 = __ffma2_rn(lp[u], X[rr][1], U1);
+                }
             }
         }
         stash(sm, 0, V0, V1);
@@ -586,21 +686,21 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
     }
     __syncthreads();
     // the slot has been read by every thread: stage the next item into it
-    if (tid == 0 && prod.n < a.n_items) {
-        stage_item<KDA>(a, prod.rec, ring + slot * a.slot_bytes, &sm.bar[slot]);
-        prod.n += gridDim.x;
-        prod.issued++;
-        prod.load(a);
-    }
-    if (tid < kDV) {
-        const int j = tid;
+    if (tid == 0 && sm.prod_n < a.n_items) produce<KDA>(sm, a, ring + slot * a.slot_bytes, &sm.bar[slot]);
+    {
+        // two threads per column, each over four warps' partials
+        const int j = tid >> 1, half = tid & 1;
+        float vs = sum_partials4(sm, 0, j, half), us = sum_partials4(sm, 1, j, half);
+        vs += __shfl_xor_sync(0xffffffffu, vs, 1);
+        us += __shfl_xor_sync(0xffffffffu, us, 1);
         const float c = sm.cc[j];
-        const float d = sm.cv[j] - c * sum_partials(sm, 0, j);
-        sm.cd[j] = d;
-        sm.cdt[j] = div_approx(d, c);
-    } else {
-        const int j = tid - kDK;
-        sm.cu[j] = sm.cc[j] * sum_partials(sm, 1, j);
+        if (half == 0) {
+            const float d = sm.cv[j] - c * vs;
+            sm.cd[j] = d;
+            sm.cdt[j] = div_approx(d, c);
+        } else {
+            sm.cu[j] = c * us;
+        }
     }
     __syncthreads();
     if (tid < kDV) {
@@ -609,6 +709,8 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
     }
     // ---- phase B: Delta update in old-scale units; P = S / a ----------------
     {
+        const float4 c4 = ld4(&sm.cc[4 * l]);
+        const float2 c0 = f2(c4.x, c4.y), c1 = f2(c4.z, c4.w);
         const float4 t4 = ld4(&sm.cdt[4 * l]);
         const float2 dt0 = f2(t4.x, t4.y), dt1 = f2(t4.z, t4.w);
         float2 dd0 = dt0, dd1 = dt1;
@@ -618,25 +720,31 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
             dd1 = f2(d4.z, d4.w);
         }
 #pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; rr++) {
-            const int i = r0 + rr;
-            const float2 gg = ld2(&sm.rg2[i]);
-            if (ROWWISE && sm.rb[i] == kPivotBits) {
-                X[rr][0] = __ffma2_rn(gg, dd0, X[rr][0]);
-                X[rr][1] = __ffma2_rn(gg, dd1, X[rr][1]);
-            } else {
-                X[rr][0] = __fmul2_rn(c0, __ffma2_rn(gg, dt0, X[rr][0]));
-                X[rr][1] = __fmul2_rn(c1, __ffma2_rn(gg, dt1, X[rr][1]));
+        for (int r2 = 0; r2 < kRowsPerWarp; r2 += 2) {
+            float2 gp[2];
+            ld_pairs(&sm.rg2[r0 + r2], gp);
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                const int rr = r2 + u, i = r0 + rr;
+                if (ROWWISE && sm.rb[i] == kPivotBits) {
+                    X[rr][0] = __ffma2_rn(gp[u], dd0, X[rr][0]);
+                    X[rr][1] = __ffma2_rn(gp[u], dd1, X[rr][1]);
+                } else {
+                    X[rr][0] = __fmul2_rn(c0, __ffma2_rn(gp[u], dt0, X[rr][0]));
+                    X[rr][1] = __fmul2_rn(c1, __ffma2_rn(gp[u], dt1, X[rr][1]));
+                }
             }
         }
     }
     const int rq = item / a.heads;
     uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + sm.head_off;
-    fit_and_store<B, ROWWISE>(sm, X, item_g, a.ls_iters);
-    __syncthreads();
+    fit_and_store<B, ROWWISE, MULTI>(sm, X, item_g, a.ls_iters);
+    // the row-wise store reads the row widths, which the next item's phase 0
+    // rewrites; the fixed-width store reads no shared state phase 0 writes
+    if (ROWWISE) __syncthreads();
 }
 
-template <bool KDA>
+template <bool KDA, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
 {
     extern __shared__ __align__(128) uint8_t ring[];
@@ -653,18 +761,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
     // first staged position of this CTA: the smallest n >= npiv with n = blockIdx.x (mod G)
     int n_first = blockIdx.x;
     if (n_first < npiv) n_first += ((npiv - n_first + G - 1) / G) * G;
-    Producer prod;  // used by thread 0 only
-    prod.n = n_first;
-    prod.issued = 0;
-    prod.rec = make_int4(0, 0, 0, 0);
     if (tid == 0) {
-        prod.load(a);
-        for (int s = 0; s < a.nslots && prod.n < a.n_items; s++) {
-            stage_item<KDA>(a, prod.rec, ring + s * a.slot_bytes, &sm.bar[s]);
-            prod.n += G;
-            prod.issued++;
-            prod.load(a);
-        }
+        sm.prod_n = n_first;
+        sm.prod_issued = 0;
+        prefetch_stage_rec(sm, a);
+        for (int s = 0; s < a.nslots && sm.prod_n < a.n_items; s++)
+            produce<KDA>(sm, a, ring + s * a.slot_bytes, &sm.bar[s]);
     }
     uint32_t n_cons = 0;
     int next_item = (blockIdx.x < a.n_items) ? a.t.order[blockIdx.x] : 0;
@@ -685,23 +787,23 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
             // a staged copy never completed: record it, drain what is in flight, stop
             if (tid == 0) {
                 atomicExch(a.t.status, kStatusWaitTimeout);
-                for (uint32_t m = n_cons - 1; m < prod.issued; m++)
+                for (uint32_t m = n_cons - 1; m < sm.prod_issued; m++)
                     mbar_wait_bounded(&sm.bar[m % (uint32_t)a.nslots], (m / (uint32_t)a.nslots) & 1u, kWaitLimit);
             }
             __syncthreads();
             return;
         }
         if (KDA) {
-            run_item<0, KDA>(sm, a, item, sb, slot, prod, ring);
+            run_item<0, KDA, MULTI>(sm, a, item, sb, slot, ring);
         } else {
             switch (sm.head_b) {
-                case 2: run_item<2, KDA>(sm, a, item, sb, slot, prod, ring); break;
-                case 3: run_item<3, KDA>(sm, a, item, sb, slot, prod, ring); break;
-                case 4: run_item<4, KDA>(sm, a, item, sb, slot, prod, ring); break;
-                case 5: run_item<5, KDA>(sm, a, item, sb, slot, prod, ring); break;
-                case 6: run_item<6, KDA>(sm, a, item, sb, slot, prod, ring); break;
-                case 7: run_item<7, KDA>(sm, a, item, sb, slot, prod, ring); break;
-                case 8: run_item<8, KDA>(sm, a, item, sb, slot, prod, ring); break;
+                case 2: run_item<2, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
+                case 3: run_item<3, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
+                case 4: run_item<4, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
+                case 5: run_item<5, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
+                case 6: run_item<6, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
+                case 7: run_item<7, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
+                case 8: run_item<8, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
                 default:  // unreachable: Gated-DeltaNet heads have one width, validated on the host
                     if (tid == 0) atomicExch(a.t.status, kStatusBadHead);
                     __syncthreads();
@@ -750,7 +852,7 @@ __device__ __forceinline__ void pack_body(ItemSmem &sm, const StepArgs &a, int i
         X[rr][0] = f2(x.x, x.y);
         X[rr][1] = f2(x.z, x.w);
     }
-    fit_and_store<B, ROWWISE>(sm, X, item_g, a.ls_iters);
+    fit_and_store<B, ROWWISE, true>(sm, X, item_g, a.ls_iters, sm.head_kind != kHeadAllPivot);
 }
 
 __global__ void __launch_bounds__(kThreads) k_pack(StepArgs a)
@@ -895,19 +997,19 @@ int sm_count()
     return g_sms;
 }
 
-template <bool KDA>
+template <bool KDA, bool MULTI>
 cudaError_t launch_decode_t(const StepArgs &a, cudaStream_t s)
 {
     const int dyn = a.nslots * a.slot_bytes;
-    cudaError_t e = cudaFuncSetAttribute(k_decode<KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    cudaError_t e = cudaFuncSetAttribute(k_decode<KDA, MULTI>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<KDA>, kThreads, dyn);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<KDA, MULTI>, kThreads, dyn);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const long long want = (long long)per_sm * sm_count();
     const int grid = (int)(a.n_items < want ? a.n_items : want);
-    k_decode<KDA><<<grid, kThreads, dyn, s>>>(a);
+    k_decode<KDA, MULTI><<<grid, kThreads, dyn, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -916,16 +1018,16 @@ cudaError_t launch_decode_t(const StepArgs &a, cudaStream_t s)
 cudaError_t launch_decode_step(const StepArgs &a, cudaStream_t s)
 {
     if (a.n_items == 0) return cudaSuccess;
-    return a.kda ? launch_decode_t<true>(a, s) : launch_decode_t<false>(a, s);
+    if (a.ls_iters <= 1) return a.kda ? launch_decode_t<true, false>(a, s) : launch_decode_t<false, false>(a, s);
+    return a.kda ? launch_decode_t<true, true>(a, s) : launch_decode_t<false, true>(a, s);
 }
 
 int decode_ctas_per_sm(int nslots, int slot_bytes)
 {
     const int dyn = nslots * slot_bytes;
     int per_sm = 0;
-    if (cudaFuncSetAttribute(k_decode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<false>, kThreads, dyn) != cudaSuccess ||
-        cudaFuncSetAttribute(k_decode<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess) {
+    if (cudaFuncSetAttribute(k_decode<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<false, false>, kThreads, dyn) != cudaSuccess) {
         cudaGetLastError();
         return 0;
     }

@@ -288,3 +288,11 @@ def test_invalid_arguments_are_rejected_on_the_host():
     st = L.stepq_decode_step(h, P(d["q"]), P(d["k"]), P(d["v"]), P(d["alpha"]), P(d["beta"]), P(torch.empty_like(d["v"])))
     assert st == stepq.ERR_STATE
     torch.cuda.synchronize()  # the context is still healthy
+
+
+@pytest.mark.parametrize("ci,ls", [(1, 2), (2, 0), (2, 3)])
+def test_least_squares_round_counts(ci, ls):
+    """0 rounds (maximum-based column scales), and several rounds (later
+    rounds clip to the row's range)."""
+    cfg = W.with_overrides(W.CONFIGS[ci], batch=2, ls_iters=ls)
+    lockstep(Setup(cfg), steps=2, t0=7)
