@@ -348,7 +348,7 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": recorded_traffic(cfg.name),
                          "algorithmic_bytes_per_launch": alg, "peak_source": src,
-                         "kernel": "stepq fused decode step (k_item<0>)"},
+                         "kernel": "fused decode step k_decode"},
             "e2e": e2e,
             "gpu_launches": args.steps,
             "fp32_state": None if fp32_ms is None else {

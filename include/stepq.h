@@ -15,7 +15,9 @@
  * Conventions for every entry point:
  *   - Pointers marked "device" are CUDA device pointers on the current device;
  *     "host" pointers are read during the call only.  All device tensors are
- *     contiguous fp32, 16-byte aligned, row-major in the shapes given.
+ *     contiguous fp32, row-major in the shapes given, and 16-byte aligned,
+ *     except the [batch, heads] tensors (beta, and alpha of Gated-DeltaNet),
+ *     which need 4-byte alignment only.
  *   - The caller owns every buffer passed in.  The library allocates no device
  *     memory and never frees a caller buffer.
  *   - Kernels are enqueued on the pool's stream (or the stream argument) and
@@ -90,12 +92,19 @@ typedef struct stepq_pool stepq_pool; /* opaque handle */
  * Packed state layout (offsets in bytes from the start of the buffer):
  *   item (b, h) starts at b * R + P_h, R = sum over heads of the item sizes,
  *   P_h = sum of the item sizes of heads 0..h-1;
- *   item = r[dk] fp32 | c[dv] fp32 | row 0 | ... | row dk-1, where a row of
- *   width b_i holds dv * b_i / 8 bytes: a little-endian bit stream with the
- *   offset-binary code (code + 2^(b_i - 1), in 1 .. 2^b_i - 1) of value column
- *   j in bits [j * b_i, (j + 1) * b_i); a pivot row holds dv binary16 values.
- *   The stored element is r_i * c_j * code_ij (ai-papers.net,
- *   "STEPQuantの仕組み"); pivot rows keep r_i = 0.
+ *   item = r[dk] fp32 | c[dv] fp32 | tile 0 | ... | tile dk/16 - 1.
+ *   Tile T covers key rows 16T .. 16T+15 and holds dv/4 = 32 interleaved
+ *   column-group streams: stream g carries the fields of value columns
+ *   4g .. 4g+3 of the tile's rows, row-major (row 16T, columns 4g..4g+3 first),
+ *   each field b_i bits wide, packed little-endian into 32-bit words and
+ *   zero-padded to W_T = ceil(4 * sum of the tile's widths / 32) words.  Word w
+ *   of stream g sits at tile byte offset 4 * (w * 32 + g), so the tile takes
+ *   128 * W_T bytes.  A field of a quantised row holds the offset-binary code
+ *   (code + 2^(b_i - 1), in 1 .. 2^b_i - 1); a field of a pivot row holds the
+ *   binary16 bits of the element.  The stored element is r_i * c_j * code_ij
+ *   (ai-papers.net, "STEPQuantの仕組み"); pivot rows keep r_i = 0, and a
+ *   Gated-DeltaNet pivot head keeps c_j = 0 as well.  The interleave lets the
+ *   32 lanes of a warp read and write one tile with whole 128-byte lines.
  */
 STEPQ_API size_t stepq_pool_bytes(const stepq_desc *desc);
 
