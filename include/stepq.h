@@ -92,19 +92,22 @@ typedef struct stepq_pool stepq_pool; /* opaque handle */
  * Packed state layout (offsets in bytes from the start of the buffer):
  *   item (b, h) starts at b * R + P_h, R = sum over heads of the item sizes,
  *   P_h = sum of the item sizes of heads 0..h-1;
- *   item = r[dk] fp32 | c[dv] fp32 | tile 0 | ... | tile dk/16 - 1.
- *   Tile T covers key rows 16T .. 16T+15 and holds dv/4 = 32 interleaved
- *   column-group streams: stream g carries the fields of value columns
- *   4g .. 4g+3 of the tile's rows, row-major (row 16T, columns 4g..4g+3 first),
- *   each field b_i bits wide, packed little-endian into 32-bit words and
- *   zero-padded to W_T = ceil(4 * sum of the tile's widths / 32) words.  Word w
- *   of stream g sits at tile byte offset 4 * (w * 32 + g), so the tile takes
- *   128 * W_T bytes.  A field of a quantised row holds the offset-binary code
- *   (code + 2^(b_i - 1), in 1 .. 2^b_i - 1); a field of a pivot row holds the
- *   binary16 bits of the element.  The stored element is r_i * c_j * code_ij
- *   (ai-papers.net, "STEPQuantの仕組み"); pivot rows keep r_i = 0, and a
- *   Gated-DeltaNet pivot head keeps c_j = 0 as well.  The interleave lets the
- *   32 lanes of a warp read and write one tile with whole 128-byte lines.
+ *   item = r[dk] fp32 | c[dv] fp32 | slab 0 | ... | slab dv/16 - 1.
+ *   Slab s covers value columns 16s .. 16s+15 of all dk key rows and holds
+ *   32 interleaved streams: stream l (rg = l % 8, cg = l / 8) carries the
+ *   fields of key rows 16rg .. 16rg+15 and value columns 16s + 4cg .. +3,
+ *   row-major (row 16rg, its 4 columns first), each field b_i bits wide,
+ *   packed little-endian into 32-bit words and zero-padded to W words, where
+ *   W (one value per head) is the largest over the 8 row groups of
+ *   ceil(4 * sum of the group's widths / 32); for a head of one width b,
+ *   W = 2b.  Word m of stream l sits at slab byte offset 4 * (32 m + l), so
+ *   a slab takes 128 W bytes and an item 4 dk + 4 dv + 1024 W bytes.  A field
+ *   of a quantised row holds the offset-binary code (code + 2^(b_i - 1), in
+ *   1 .. 2^b_i - 1); a field of a pivot row holds the binary16 bits of the
+ *   element.  The stored element is r_i * c_j * code_ij (ai-papers.net,
+ *   "STEPQuantの仕組み"); pivot rows keep r_i = 0, and a Gated-DeltaNet
+ *   pivot head keeps c_j = 0 as well.  The interleave lets the 32 lanes of a
+ *   warp that own one slab read and write it in whole 128-byte lines.
  */
 STEPQ_API size_t stepq_pool_bytes(const stepq_desc *desc);
 

@@ -71,32 +71,37 @@ double oracle_column_error_f64(int dk, int dv, int j, const double *S, const uin
 }
 
 /* ---- the packed byte format ---------------------------------------------- *
- * item = r[dk] fp32 | c[dv] fp32 | tile 0 | ... | tile dk/16 - 1.
- * Tile T holds key rows 16T .. 16T+15.  For each column group g (value columns
- * 4g .. 4g+3, g = 0 .. dv/4 - 1) the tile's codes are taken row by row, and
- * within a row column by column, as fields of the row's width (the
- * offset-binary code u = code + 2^(b-1), or the binary16 bits on a pivot row),
- * concatenated into one little-endian bit stream that is zero-padded to whole
- * 32-bit words.  Every stream of a tile has the same length W_T (the tile's
- * rows fix it); word w of stream g is stored at word w * (dv/4) + g of the
- * tile. */
+ * item = r[dk] fp32 | c[dv] fp32 | slab 0 | ... | slab dv/16 - 1.
+ * Slab s holds value columns 16s .. 16s+15 of every key row as NS = 4 dk/16
+ * streams.  Stream l covers the key rows of row group l % (dk/16) (rows
+ * 16 (l % (dk/16)) .. +15) and the value columns 16s + 4 (l / (dk/16)) .. +3:
+ * its codes are taken row by row, and within a row column by column, as fields
+ * of the row's width (the offset-binary code u = code + 2^(b-1), or the
+ * binary16 bits on a pivot row), concatenated into one little-endian bit
+ * stream that is zero-padded to W 32-bit words.  W is one number per head: the
+ * largest over the row groups of the words the group's fields need.  Word m of
+ * stream l is stored at word m * NS + l of the slab. */
 
-enum { TILE_ROWS = 16, GROUP_COLS = 4 };
+enum { GROUP_ROWS = 16, GROUP_COLS = 4, SLAB_COLS = 16 };
 
 static int field_bits(int b) { return b; } /* a pivot row's field is its 16 binary16 bits */
 
-static size_t tile_words(const uint8_t *bits_tile)
+static size_t stream_words(int dk, const uint8_t *bits)
 {
-    size_t nbits = 0;
-    for (int rr = 0; rr < TILE_ROWS; rr++) nbits += (size_t)GROUP_COLS * field_bits(bits_tile[rr]);
-    return (nbits + 31) / 32;
+    size_t W = 0;
+    for (int g = 0; g < dk / GROUP_ROWS; g++) {
+        size_t nbits = 0;
+        for (int rr = 0; rr < GROUP_ROWS; rr++) nbits += (size_t)GROUP_COLS * field_bits(bits[g * GROUP_ROWS + rr]);
+        const size_t w = (nbits + 31) / 32;
+        if (w > W) W = w;
+    }
+    return W;
 }
 
 size_t oracle_item_bytes(int dk, int dv, const uint8_t *bits)
 {
-    size_t n = 4 * (size_t)dk + 4 * (size_t)dv;
-    for (int T = 0; T < dk / TILE_ROWS; T++) n += 4 * tile_words(bits + T * TILE_ROWS) * (size_t)(dv / GROUP_COLS);
-    return n;
+    const size_t NS = (size_t)GROUP_COLS * (dk / GROUP_ROWS);
+    return 4 * (size_t)dk + 4 * (size_t)dv + 4 * stream_words(dk, bits) * NS * (size_t)(dv / SLAB_COLS);
 }
 
 static void put_f32(uint8_t *dst, float x) { memcpy(dst, &x, 4); } /* host is little-endian */
@@ -110,27 +115,28 @@ void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const
                       const int32_t *code, const float *piv, uint8_t *item)
 {
     uint8_t *p = item;
-    const int G = dv / GROUP_COLS;
+    const int RG = dk / GROUP_ROWS, NS = GROUP_COLS * RG;
+    const size_t W = stream_words(dk, bits);
     for (int i = 0; i < dk; i++, p += 4) put_f32(p, r[i]);
     for (int j = 0; j < dv; j++, p += 4) put_f32(p, c[j]);
-    for (int T = 0; T < dk / TILE_ROWS; T++) {
-        const size_t W = tile_words(bits + T * TILE_ROWS);
-        memset(p, 0, 4 * W * G);
-        for (int g = 0; g < G; g++) {
-            size_t pos = 0; /* bit position in stream g */
-            for (int rr = 0; rr < TILE_ROWS; rr++) {
-                const int i = T * TILE_ROWS + rr, b = bits[i];
+    for (int sl = 0; sl < dv / SLAB_COLS; sl++) {
+        memset(p, 0, 4 * W * NS);
+        for (int l = 0; l < NS; l++) {
+            const int g = l % RG, cg = l / RG;
+            size_t pos = 0; /* bit position in stream l */
+            for (int rr = 0; rr < GROUP_ROWS; rr++) {
+                const int i = g * GROUP_ROWS + rr, b = bits[i];
                 for (int kk = 0; kk < GROUP_COLS; kk++) {
-                    const int j = g * GROUP_COLS + kk;
+                    const int j = sl * SLAB_COLS + cg * GROUP_COLS + kk;
                     const uint32_t u = (b == ORACLE_PIVOT_BITS)
                                            ? oracle_to_fp16((double)piv[i * dv + j])
                                            : (uint32_t)(code[i * dv + j] + (1 << (b - 1)));
                     for (int t = 0; t < field_bits(b); t++, pos++)
-                        if ((u >> t) & 1u) set_bit(p, (pos / 32) * G + g, (int)(pos % 32));
+                        if ((u >> t) & 1u) set_bit(p, (pos / 32) * NS + l, (int)(pos % 32));
                 }
             }
         }
-        p += 4 * W * G;
+        p += 4 * W * NS;
     }
 }
 
@@ -138,20 +144,21 @@ void oracle_unpack_item(int dk, int dv, const uint8_t *bits, const uint8_t *item
                         float *r, float *c, int32_t *code, float *piv)
 {
     const uint8_t *p = item;
-    const int G = dv / GROUP_COLS;
+    const int RG = dk / GROUP_ROWS, NS = GROUP_COLS * RG;
+    const size_t W = stream_words(dk, bits);
     for (int i = 0; i < dk; i++, p += 4) r[i] = get_f32(p);
     for (int j = 0; j < dv; j++, p += 4) c[j] = get_f32(p);
-    for (int T = 0; T < dk / TILE_ROWS; T++) {
-        const size_t W = tile_words(bits + T * TILE_ROWS);
-        for (int g = 0; g < G; g++) {
+    for (int sl = 0; sl < dv / SLAB_COLS; sl++) {
+        for (int l = 0; l < NS; l++) {
+            const int g = l % RG, cg = l / RG;
             size_t pos = 0;
-            for (int rr = 0; rr < TILE_ROWS; rr++) {
-                const int i = T * TILE_ROWS + rr, b = bits[i];
+            for (int rr = 0; rr < GROUP_ROWS; rr++) {
+                const int i = g * GROUP_ROWS + rr, b = bits[i];
                 for (int kk = 0; kk < GROUP_COLS; kk++) {
-                    const int j = g * GROUP_COLS + kk;
+                    const int j = sl * SLAB_COLS + cg * GROUP_COLS + kk;
                     uint32_t u = 0;
                     for (int t = 0; t < field_bits(b); t++, pos++)
-                        u |= (uint32_t)get_bit(p, (pos / 32) * G + g, (int)(pos % 32)) << t;
+                        u |= (uint32_t)get_bit(p, (pos / 32) * NS + l, (int)(pos % 32)) << t;
                     if (b == ORACLE_PIVOT_BITS) {
                         piv[i * dv + j] = (float)oracle_from_fp16((uint16_t)u);
                         code[i * dv + j] = 0;
@@ -162,7 +169,7 @@ void oracle_unpack_item(int dk, int dv, const uint8_t *bits, const uint8_t *item
                 }
             }
         }
-        p += 4 * W * G;
+        p += 4 * W * NS;
     }
 }
 

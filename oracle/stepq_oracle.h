@@ -103,12 +103,13 @@ uint16_t oracle_to_fp16(double x);
 double oracle_from_fp16(uint16_t h);
 
 /* ---- packed byte format (the pool) ---------------------------------------- *
- * item = r[dk] fp32 | c[dv] fp32 | tile 0 | ... | tile dk/16 - 1; tile T holds
- * key rows 16T..16T+15.  Column group g (columns 4g..4g+3) of a tile is one
- * little-endian bit stream: row by row, column by column, the row's b-bit
- * offset-binary code (or 16 binary16 bits on a pivot row), zero-padded to whole
- * 32-bit words; word w of stream g sits at word w * (dv/4) + g of the tile.
- * Requires dk % 16 == 0 and dv % 4 == 0. */
+ * item = r[dk] fp32 | c[dv] fp32 | slab 0 | ... | slab dv/16 - 1; slab s holds
+ * value columns 16s..16s+15 as NS = 4 dk/16 streams.  Stream l covers key rows
+ * 16 (l % (dk/16)) .. +15 and columns 16s + 4 (l / (dk/16)) .. +3: row by row,
+ * column by column, the row's b-bit offset-binary code (or 16 binary16 bits on
+ * a pivot row), little-endian, zero-padded to W words, W per head = the most
+ * any row group needs; word m of stream l sits at word m * NS + l of the slab.
+ * Requires dk % 16 == 0 and dv % 16 == 0. */
 size_t oracle_item_bytes(int dk, int dv, const uint8_t *bits);
 void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
                       const int32_t *code, const float *piv, uint8_t *item);

@@ -60,7 +60,7 @@ struct Layout {
            total = 0;
     long long req_bytes = 0;
     std::vector<long long> item_bytes;  // per head
-    std::vector<int> tile_words;        // per head and tile
+    std::vector<int> slab_words;        // per head: 32-bit words per stream
 };
 
 // Checks a descriptor; fills the layout when valid.
@@ -94,20 +94,22 @@ stepq_status check_desc(const stepq_desc *d, bool need_tables, Layout *L)
         }
     }
     if (L) {
-        // packed item: header, then 8 tiles of 16 rows; a tile stores 32 column-group
-        // streams of W words each, W = ceil(4 * sum of the tile's widths / 32)
+        // packed item: header, then 8 slabs of 16 value columns; a slab holds 32
+        // streams (8 row groups x 4 column groups) of W words each, W = the
+        // largest over the row groups of ceil(4 * sum of the group's widths / 32)
         L->item_bytes.assign(H, 0);
-        L->tile_words.assign((size_t)H * stepq::kTiles, 0);
+        L->slab_words.assign(H, 0);
         long long req = 0;
         for (int h = 0; h < H; h++) {
-            long long n = stepq::kHeaderBytes;
-            for (int T = 0; T < stepq::kTiles; T++) {
+            int W = 0;
+            for (int g = 0; g < stepq::kRowGroups; g++) {
                 int bitsum = 0;
-                for (int rr = 0; rr < stepq::kRowsPerWarp; rr++) bitsum += d->bits[h * kDK + T * stepq::kRowsPerWarp + rr];
-                const int W = (4 * bitsum + 31) / 32;
-                L->tile_words[(size_t)h * stepq::kTiles + T] = W;
-                n += 4LL * W * stepq::kGroups;
+                for (int rr = 0; rr < stepq::kRowsPerGroup; rr++)
+                    bitsum += d->bits[h * kDK + g * stepq::kRowsPerGroup + rr];
+                W = std::max(W, (4 * bitsum + 31) / 32);
             }
+            L->slab_words[h] = W;
+            const long long n = stepq::kHeaderBytes + 4LL * W * stepq::kStreams * stepq::kSlabs;
             L->item_bytes[h] = n;
             req += n;
         }
@@ -233,21 +235,17 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
                 npiv++;
                 R.s[i] = 0.f;
                 R.rho[i] = 0.f;
+                R.rq[i] = 0.f;
             } else {
                 R.s[i] = (float)(1.0 / std::sqrt((double)desc->rho[h * kDK + i]));
                 R.rho[i] = desc->rho[h * kDK + i];
+                R.rq[i] = (float)(1.0 / (double)((1 << (b - 1)) - 1));
             }
         }
         kind[h] = npiv == 0 ? stepq::kHeadQuant : (npiv == kDK ? stepq::kHeadAllPivot : stepq::kHeadMixed);
         R.head_kind = kind[h];
         R.head_b = (same && b0 != STEPQ_PIVOT_BITS) ? b0 : 0;
-        uint32_t toff = stepq::kHeaderBytes;
-        for (int T = 0; T < stepq::kTiles; T++) {
-            const int W = L.tile_words[(size_t)h * stepq::kTiles + T];
-            R.tile_off[T] = toff;
-            R.tile_words[T] = (uint8_t)W;
-            toff += 4u * W * stepq::kGroups;
-        }
+        R.slab_words = L.slab_words[h];
         if (kind[h] != stepq::kHeadAllPivot) max_staged = std::max(max_staged, L.item_bytes[h]);
     }
     // order: items of all-pivot heads first (processed from global memory), then
@@ -274,7 +272,8 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
     int n_pivot_items = 0;
     for (int h = 0; h < H; h++) n_pivot_items += (kind[h] == stepq::kHeadAllPivot) ? B : 0;
 
-    // staging slot geometry of the fused decode kernel
+    // staging slot geometry of the fused decode kernel: the item as stored, then
+    // the step inputs and the head record
     const int kda = desc->variant == STEPQ_KDA;
     int off = (int)align_up((size_t)max_staged, 16);
     const int off_q = off; off += 4 * kDK;

@@ -9,10 +9,12 @@ namespace stepq {
 
 constexpr int kDK = 128;          // key dimension (rows of a state)
 constexpr int kDV = 128;          // value dimension (columns of a state)
-constexpr int kThreads = 256;     // threads per item: 8 warps x 16 rows, lane = 4 columns
-constexpr int kRowsPerWarp = 16;  // = rows of a packed tile
-constexpr int kTiles = kDK / kRowsPerWarp;
-constexpr int kGroups = kDV / 4;  // column groups (lanes) per tile
+constexpr int kThreads = 256;     // threads per item (8 warps)
+constexpr int kRowsPerGroup = 16; // key rows of a stream's row group = rows a thread holds
+constexpr int kRowGroups = kDK / kRowsPerGroup;
+constexpr int kSlabCols = 16;     // value columns of a slab = columns a warp owns
+constexpr int kSlabs = kDV / kSlabCols;
+constexpr int kStreams = 32;      // streams per slab: 8 row groups x 4 column groups of 4
 constexpr int kPivotBits = 16;
 constexpr int kHeaderBytes = 4 * kDK + 4 * kDV;  // r[dk] | c[dv]
 constexpr int kMaxSlots = 8;
@@ -25,16 +27,16 @@ constexpr int kHeadMixed = 2;     // some rows pivots
 // Per-head record (host-built, staged with every item): the fit constants and
 // the tile layout of the head's items.
 struct HeadRec {
-    float s[kDK];                // fp32(rho_i^-1/2), rounded once from fp64
-    float rho[kDK];              // row-impact weights
+    float s[kDK];                // fp32(rho_i^-1/2), rounded once from fp64 (0 on pivot rows)
+    float rho[kDK];              // row-impact weights (0 on pivot rows)
+    float rq[kDK];               // fp32(1 / Q_i), Q_i = 2^(b_i - 1) - 1 (0 on pivot rows)
     uint8_t bits[kDK];           // row widths (16 = pivot)
-    uint32_t tile_off[kTiles];   // byte offset of tile T inside the item
-    uint8_t tile_words[kTiles];  // 32-bit words per column-group stream of tile T
     long long head_off;          // byte offset of the head's item inside a request
     int head_b;                  // common row width, 0 if the rows differ
     int head_kind;               // kHeadQuant / kHeadAllPivot / kHeadMixed
     int head_bytes;              // bytes of one item
-    int pad;
+    int slab_words;              // 32-bit words per stream (W)
+    int pad[2];
 };
 static_assert(sizeof(HeadRec) % 16 == 0, "head record must be a multiple of 16 bytes");
 

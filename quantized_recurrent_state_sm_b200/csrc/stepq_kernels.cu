@@ -1,14 +1,19 @@
 // Kernels of the packed-state gated Delta-rule decode step (sm_100a).
 //
-// Thread mapping (every kernel): a CTA of 256 threads owns one (request,
-// head) item at a time; warp w owns key rows 16w .. 16w+15 (= packed tile w),
-// lane l owns value columns 4l .. 4l+3 (= column group l), so a thread holds
-// 64 state elements in registers and reads / writes exactly one column-group
-// stream of one tile: the pool layout is built around this mapping.  The
-// elements are kept as float2 pairs (columns 4l, 4l+1 and 4l+2, 4l+3) so that
-// every floating-point operation on the state is one packed f32x2 instruction;
-// per-row factors are stored duplicated, (x, x), so that broadcasting them
-// costs nothing.
+// Thread mapping (every kernel): a CTA of 256 threads owns one (request, head)
+// item at a time.  Warp w owns value columns 16w .. 16w+15 over all 128 key
+// rows (= packed slab w); lane l = rg + 8 cg owns key rows 16rg .. 16rg+15 and
+// value columns 16w + 4cg .. +3 (= stream l of slab w).  A thread therefore
+// holds 64 state values in registers and reads / writes exactly one stream of
+// the pool, and the 32 lanes of a warp touch whole 128-byte lines.  The values are
+// kept as float2 pairs (columns 4g, 4g+1 and 4g+2, 4g+3) so that every
+// floating-point operation on the state is one packed f32x2 instruction;
+// per-row factors are stored duplicated, (x, x), so broadcasting them is free.
+//
+// Every column sum of the step (key projection, readout, column maxima,
+// least-squares sums) runs over the 8 lanes of one warp that share cg, by
+// shuffles; only the row magnitudes cross warps, through shared memory, so an
+// item costs two CTA barriers.
 //
 // Method (ai.info summary of STEPQuant, "Key Contributions" and "Methodology in
 // Plain English"; ai-papers.net, "STEPQuantの仕組み"; ai-trend.me, "핵심 용어"):
@@ -35,35 +40,34 @@ using namespace dev;
 
 constexpr long long kWaitLimit = 4000000000LL;  // SM clock cycles before a wait gives up
 constexpr float kRoundMagic = 12582912.0f;      // 1.5 * 2^23: x + it rounds x to an integer
-
-struct alignas(16) ItemSmem {
-    float2 rk2[kDK], rl2[kDK], rg2[kDK], ra2[kDK];  // update factors per row, duplicated
-    float2 rh2[kDK], rw2[kDK], rq2[kDK];            // fit factors per row, duplicated
-    float ra[kDK], rs[kDK], rrho[kDK];              // a_i, s_i, rho_i
-    int rb[kDK];                                    // row widths
-    float cc[kDV], cv[kDV], cd[kDV], cdt[kDV], cu[kDV];
-    float cc0[kDV], cnew[kDV], ci[kDV], crat[kDV];
-    float red[2][8][kDV];
-    float rowt[8][16][36];  // per-warp transposition for row sums
-    float kq[4];
-    float beta_item;
-    uint32_t tile_off[kTiles];
-    int head_b, head_kind;
-    long long head_off;
-    uint64_t bar[kMaxSlots];
-    int4 prod_rec;          // producer (thread 0): staging record of position prod_n
-    int prod_n;             // producer: next position to stage
-    uint32_t prod_issued;   // producer: items staged so far
-};
-
-using X2 = float2[kRowsPerWarp][2];  // the thread's 16 x 4 block as float2 pairs
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kProducerWarp = 7;                // the warp that issues the staging copies
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
-__device__ __forceinline__ float2 ld2(const float2 *p) { return *p; }
+
+// Row i's place in the arrays of duplicated row factors: float4 number
+// pslot(i) holds rows i & ~1 and i | 1 as (f, f, f', f'), ordered so that the
+// 8 row groups of a warp read 8 consecutive float4.
+__device__ __forceinline__ int pslot(int i) { return ((i & 15) >> 1) * 8 + (i >> 4); }
+// Row i's place in per-row scalar arrays read by row group.
+__device__ __forceinline__ int sslot(int i) { return (i & 15) * 8 + (i >> 4); }
+
+__device__ __forceinline__ void put_pair(float4 *arr, int i, float v)
+{
+    reinterpret_cast<float2 *>(arr + pslot(i))[i & 1] = make_float2(v, v);
+}
+
+// The duplicated factors of rows 16 rg + 2p and 16 rg + 2p + 1.
+__device__ __forceinline__ void ld_pairs(const float4 *arr, int p, int rg, float2 (&out)[2])
+{
+    const float4 v = arr[p * 8 + rg];
+    out[0] = make_float2(v.x, v.y);
+    out[1] = make_float2(v.z, v.w);
+}
 
 // Call-free reciprocal, quotient and square root (within 2 ulp of the correctly
-// rounded results) for the per-row and per-column factors computed while the
+// rounded results) for the per-row and per-column factors computed while a
 // thread's state is live in registers: the correctly rounded forms branch to a
 // slow-path subroutine whose call would force the state out to local memory.
 __device__ __forceinline__ float rcp_approx(float x)
@@ -88,71 +92,61 @@ __device__ __forceinline__ float max_abs3(float a, float b, float c)
     return r;
 }
 
-// ---------------------------------------------------------------------------
-// Column sums over the 8 warps of per-thread partials.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void stash(ItemSmem &sm, int vec, float2 a, float2 b)
+__device__ __forceinline__ float2 shfl2(float2 v, int m)
 {
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    *reinterpret_cast<float4 *>(&sm.red[vec][w][4 * l]) = make_float4(a.x, a.y, b.x, b.y);
+    return f2(__shfl_xor_sync(kFull, v.x, m), __shfl_xor_sync(kFull, v.y, m));
 }
 
-__device__ __forceinline__ float sum_partials(const ItemSmem &sm, int vec, int j)
-{
-    float acc = sm.red[vec][0][j];
-#pragma unroll
-    for (int w = 1; w < 8; w++) acc += sm.red[vec][w][j];
-    return acc;
-}
+// Per-item factors, double-buffered by item parity: the factors of the next
+// item are written while the current item's fit still reads its own.
+struct alignas(16) RowFactors {
+    float4 k2[64], l2[64], g2[64];  // a k, a q, gamma (see pslot)
+    float4 a2[64], q2[64];          // alpha, 1/Q (0 on pivot rows); row-wise widths only
+    float4 h2[64], w2[64];          // fit: h = a / r', w = rho r'^2
+    float ra[kDK];                  // a_i = alpha_i r_i (alpha_i on pivot rows), by row
+    int rb[kDK];                    // widths, by sslot
+    float kqp[4];                   // k.q over rows 32m .. 32m+31
+    float beta;
+    int item, head_b;               // the item; its head's common width (0: row-wise)
+};
 
-__device__ __forceinline__ float max_partials(const ItemSmem &sm, int vec, int j)
-{
-    float acc = sm.red[vec][0][j];
-#pragma unroll
-    for (int w = 1; w < 8; w++) acc = fmaxf(acc, sm.red[vec][w][j]);
-    return acc;
-}
+struct alignas(16) ItemSmem {
+    struct {
+        RowFactors rf[2];
+    } u;
+    // per value column; warp w touches only its own 16 columns
+    float cd[kDV], cdt[kDV], cc0[kDV], cnew[kDV], ci[kDV], crat[kDV];
+    // row partials of P^2: [warp][column subgroup][128 rows] in 16-byte
+    // chunks swizzled by row group (rowp_chunk)
+    float rowp[8 * 4 * kDK];
+    uint64_t bar[kMaxSlots];
+    int4 prod_rec;          // producer: staging record of position prod_n
+    int prod_n;             // producer: next position to stage
+    uint32_t prod_issued;   // producer: items staged so far
+};
 
-// Half of a column reduction: the partials of warps 4 half .. 4 half + 3.
-__device__ __forceinline__ float sum_partials4(const ItemSmem &sm, int vec, int j, int half)
-{
-    const float a = sm.red[vec][4 * half][j], b = sm.red[vec][4 * half + 1][j];
-    const float c = sm.red[vec][4 * half + 2][j], d = sm.red[vec][4 * half + 3][j];
-    return (a + b) + (c + d);
-}
+using X2 = float2[kRowsPerGroup][2];  // the thread's 16 x 4 block as float2 pairs
 
-__device__ __forceinline__ float max_partials4(const ItemSmem &sm, int vec, int j, int half)
-{
-    const float a = sm.red[vec][4 * half][j], b = sm.red[vec][4 * half + 1][j];
-    const float c = sm.red[vec][4 * half + 2][j], d = sm.red[vec][4 * half + 3][j];
-    return fmaxf(fmaxf(a, b), fmaxf(c, d));
-}
-
-// The duplicated factors of two consecutive rows (p 16-byte aligned) in one load.
-__device__ __forceinline__ void ld_pairs(const float2 *p, float2 (&out)[2])
-{
-    const float4 v = *reinterpret_cast<const float4 *>(p);
-    out[0] = make_float2(v.x, v.y);
-    out[1] = make_float2(v.z, v.w);
-}
+// Word offset, inside a 128-float row-partial block, of the chunk holding rows
+// 16 rg + 4 q .. +3 (conflict-free for both the writes and the row reads).
+__device__ __forceinline__ int rowp_chunk(int rg, int q) { return 16 * rg + 4 * (q ^ ((rg >> 1) & 3)); }
 
 // ---------------------------------------------------------------------------
-// Decode the thread's column-group stream of its tile into X (code values as
-// floats; pivot rows: their binary16 values).  Fixed width B > 0 keeps the
-// stream in registers; B == 0 reads widths per row from sm.rb.
+// Decode the thread's stream (word m at words[32 m]) into X: code values as
+// floats; pivot rows their binary16 values.  Fixed width B > 0 keeps the
+// stream in registers; B == 0 reads the row widths from rb_lane[8 rr].
 // ---------------------------------------------------------------------------
 template <int B>
-__device__ __forceinline__ void decode_stream(const ItemSmem &sm, const uint32_t *words, int stride, X2 &X)
+__device__ __forceinline__ void decode_stream(const int *rb_lane, const uint32_t *words, X2 &X)
 {
-    const int w = threadIdx.x >> 5;
     if constexpr (B > 0) {
         uint32_t wd[2 * B];
 #pragma unroll
-        for (int m = 0; m < 2 * B; m++) wd[m] = words[m * stride];
+        for (int m = 0; m < 2 * B; m++) wd[m] = words[m * kStreams];
         const float mz = -(kMagic + (float)(1 << (B - 1)));
         const float2 mz2 = f2(mz, mz);
 #pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; rr++)
+        for (int rr = 0; rr < kRowsPerGroup; rr++)
 #pragma unroll
             for (int hh = 0; hh < 2; hh++) {
                 const uint32_t u0 = field_at<B>(wd, 4 * rr + 2 * hh) | kMagicBits;
@@ -161,10 +155,10 @@ __device__ __forceinline__ void decode_stream(const ItemSmem &sm, const uint32_t
             }
     } else {
         BitReader br;
-        br.init(words, stride);
+        br.init(words, kStreams);
 #pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; rr++) {
-            const int b = sm.rb[kRowsPerWarp * w + rr];
+        for (int rr = 0; rr < kRowsPerGroup; rr++) {
+            const int b = rb_lane[8 * rr];
             if (b == kPivotBits) {
 #pragma unroll
                 for (int hh = 0; hh < 2; hh++) {
@@ -187,67 +181,80 @@ __device__ __forceinline__ void decode_stream(const ItemSmem &sm, const uint32_t
     }
 }
 
-// One least-squares round's partial sums over the thread's rows, stashed for
-// the column reduction: with n = rne(p / c) (clipped to the row's range when
-// CLIP), N_j = sum w_i n_ij p_ij and D_j = sum w_i n_ij^2.
-template <int B, bool ROWWISE, bool CLIP>
-__device__ __forceinline__ void ls_partials(ItemSmem &sm, const X2 &X)
+// Sum over the 8 lanes sharing cg of two 4-column vectors (A0|A1 and B0|B1,
+// float2 each), scattered: on return lane rg holds the full sum of vector
+// (rg & 4 ? B : A) at column rg & 3 of the thread's four.
+__device__ __forceinline__ float reduce_scatter_2x4(float2 A0, float2 A1, float2 B0, float2 B1, int rg)
 {
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    const int r0 = kRowsPerWarp * w;
+    const bool hiA = rg & 4, hiB = rg & 2, hiC = rg & 1;
+    float2 k0 = hiA ? B0 : A0, k1 = hiA ? B1 : A1;
+    const float2 s0 = hiA ? A0 : B0, s1 = hiA ? A1 : B1;
+    k0 = __fadd2_rn(k0, shfl2(s0, 4));
+    k1 = __fadd2_rn(k1, shfl2(s1, 4));
+    float2 kk = hiB ? k1 : k0;
+    const float2 ss = hiB ? k0 : k1;
+    kk = __fadd2_rn(kk, shfl2(ss, 2));
+    const float v = hiC ? kk.y : kk.x;
+    const float sv = hiC ? kk.x : kk.y;
+    return v + __shfl_xor_sync(kFull, sv, 1);
+}
+
+// ---------------------------------------------------------------------------
+// One least-squares round: with n = rne(p / c) (clipped to the row's range
+// when CLIP), N_j = sum w_i n_ij p_ij and D_j = sum w_i n_ij^2 over the
+// warp's rows; then c_j = N_j / D_j (kept when D_j = 0), its reciprocal and
+// c0_j / c_j for the warp's 16 columns.
+// ---------------------------------------------------------------------------
+template <int B, bool ROWWISE, bool CLIP>
+__device__ __forceinline__ void ls_round(ItemSmem &sm, const RowFactors &rf, const X2 &X)
+{
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31, rg = l & 7, cg = l >> 3;
+    const int col0 = 16 * w + 4 * cg;
     const float2 rm2 = f2(kRoundMagic, kRoundMagic), nrm2 = f2(-kRoundMagic, -kRoundMagic);
-    const float4 i4 = ld4(&sm.ci[4 * l]);
+    const float4 i4 = ld4(&sm.ci[col0]);
     const float2 ic0 = f2(i4.x, i4.y), ic1 = f2(i4.z, i4.w);
     float2 N0 = f2(0.f, 0.f), N1 = N0, D0 = N0, D1 = N0;
 #pragma unroll
-    for (int rr = 0; rr < kRowsPerWarp; rr += 2) {
+    for (int p = 0; p < kRowsPerGroup / 2; p++) {
         float2 wp[2];
-        ld_pairs(&sm.rw2[r0 + rr], wp);
+        ld_pairs(rf.w2, p, rg, wp);
 #pragma unroll
         for (int u = 0; u < 2; u++) {
-            const int i = r0 + rr + u;
-            if (ROWWISE && sm.rb[i] == kPivotBits) continue;
+            const int rr = 2 * p + u;
+            if (ROWWISE && rf.rb[8 * rr + rg] == kPivotBits) continue;
             // round to the nearest integer, ties to even: x + 1.5 * 2^23 - 1.5 * 2^23;
-            // clipping acts on the biased value (for a fixed width the bounds are
-            // immediates)
-            float2 m0 = __ffma2_rn(X[rr + u][0], ic0, rm2);
-            float2 m1 = __ffma2_rn(X[rr + u][1], ic1, rm2);
+            // clipping acts on the biased value
+            float2 m0 = __ffma2_rn(X[rr][0], ic0, rm2);
+            float2 m1 = __ffma2_rn(X[rr][1], ic1, rm2);
             if (CLIP) {
-                const float Q = (float)qmax_of(ROWWISE ? sm.rb[i] : B);
+                const float Q = (float)qmax_of(ROWWISE ? rf.rb[8 * rr + rg] : B);
                 const float lo = kRoundMagic - Q, hi = kRoundMagic + Q;
                 m0 = f2(fminf(fmaxf(m0.x, lo), hi), fminf(fmaxf(m0.y, lo), hi));
                 m1 = f2(fminf(fmaxf(m1.x, lo), hi), fminf(fmaxf(m1.y, lo), hi));
             }
             const float2 n0 = __fadd2_rn(m0, nrm2), n1 = __fadd2_rn(m1, nrm2);
             const float2 wn0 = __fmul2_rn(wp[u], n0), wn1 = __fmul2_rn(wp[u], n1);
-            N0 = __ffma2_rn(wn0, X[rr + u][0], N0);
-            N1 = __ffma2_rn(wn1, X[rr + u][1], N1);
+            N0 = __ffma2_rn(wn0, X[rr][0], N0);
+            N1 = __ffma2_rn(wn1, X[rr][1], N1);
             D0 = __ffma2_rn(wn0, n0, D0);
             D1 = __ffma2_rn(wn1, n1, D1);
         }
     }
-    stash(sm, 0, N0, N1);
-    stash(sm, 1, D0, D1);
-}
-
-// The least-squares column scales from the stashed partials, two threads per
-// column: c_j = N_j / D_j (kept when D_j = 0), its reciprocal, and c0_j / c_j.
-__device__ __forceinline__ void ls_update_columns(ItemSmem &sm)
-{
-    const int j = threadIdx.x >> 1, half = threadIdx.x & 1;
-    float nn = sum_partials4(sm, 0, j, half), dd = sum_partials4(sm, 1, j, half);
-    nn += __shfl_xor_sync(0xffffffffu, nn, 1);
-    dd += __shfl_xor_sync(0xffffffffu, dd, 1);
-    if (half == 0) {
-        const float c = (dd > 0.f) ? div_approx(nn, dd) : sm.cnew[j];
+    // lane rg: N (rg < 4) or D (rg >= 4) of column col0 + (rg & 3)
+    const float part = reduce_scatter_2x4(N0, N1, D0, D1, rg);
+    const float other = __shfl_xor_sync(kFull, part, 4);
+    if (rg < 4) {
+        const int j = col0 + rg;
+        const float c = (other > 0.f) ? div_approx(part, other) : sm.cnew[j];
         const float icn = rcp_approx(c);
         sm.cnew[j] = c;
         sm.ci[j] = icn;
         sm.crat[j] = sm.cc0[j] * icn;
     }
+    __syncwarp();
 }
 
-// Final codes of a fixed-width tile stream and their store: u = z + clip(rne(p / c))
+// Final codes of a fixed-width stream and their store: u = z + clip(rne(p / c))
 // taken from the low mantissa bits of p / c + 2^23 + z; each 32-bit word is
 // stored as soon as its last code is placed.
 template <int B, bool CLIP>
@@ -260,7 +267,7 @@ __device__ __forceinline__ void pack_fixed(const X2 &X, float2 ic0, float2 ic1, 
 #pragma unroll
     for (int m = 0; m <= 2 * B; m++) ow[m] = 0u;
 #pragma unroll
-    for (int rr = 0; rr < kRowsPerWarp; rr++)
+    for (int rr = 0; rr < kRowsPerGroup; rr++)
 #pragma unroll
         for (int hh = 0; hh < 2; hh++) {
             float2 mm;
@@ -276,139 +283,159 @@ __device__ __forceinline__ void pack_fixed(const X2 &X, float2 ic0, float2 ic1, 
                 const int c = 4 * rr + 2 * hh + e;
                 field_put_bits<B>(ow, c, __float_as_uint(e ? mm.y : mm.x));
 #pragma unroll
-                for (int m = (c * B) / 32; m < ((c + 1) * B) / 32; m++) words[m * kGroups] = ow[m];
+                for (int m = (c * B) / 32; m < ((c + 1) * B) / 32; m++) words[m * kStreams] = ow[m];
             }
         }
 }
 
+// Nothing to do between the two barriers of the fit (pack kernel).
+struct NoMid {
+    __device__ __forceinline__ bool operator()() const { return true; }
+};
+
+enum FitResult { kFitDone = 0, kFitAbortNow = 1, kFitAbortAfter = 2 };
+
 // ---------------------------------------------------------------------------
 // The fit (row scales, column scales, least squares), requantisation and the
 // packed store.  On entry X holds P_ij = S_ij / a_i on quantised rows and S_ij
-// on pivot rows; sm.ra, rs, rrho, rb, rq2 and sm.head_b / head_kind are set.
-// Writes r', c and the item's streams at item_g.  Contains __syncthreads.
-// ROWWISE: rows may differ in width and may be pivots.
+// on pivot rows; rf.ra, rb (and q2 for row-wise widths) are set, rec is the
+// head's record (fit constants).  Writes r', c and the item's streams at
+// item_g (W words per stream).
+//
+// Barrier 1 publishes the row partials of P^2; threads 0..127 then derive row
+// i's scale and fit factors while `mid` runs on threads 128..255 (the fused
+// step prepares the next item there); barrier 2 publishes both, and
+// everything after it is warp-local.  If ok_in is false on any thread the
+// item is abandoned at barrier 1 with nothing stored (kFitAbortNow); if `mid`
+// fails on any thread the item is completed and kFitAbortAfter returned.
 // ---------------------------------------------------------------------------
-template <int B, bool ROWWISE, bool MULTI>
-__device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item_g, int ls_iters,
-                                              bool store_c = true)
+template <int B, bool ROWWISE, bool MULTI, class Mid>
+__device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf, const HeadRec *rec, X2 &X,
+                                                   uint8_t *item_g, int W, int ls_iters, bool store_c,
+                                                   bool ok_in, const Mid &mid)
 {
-    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
-    const int r0 = kRowsPerWarp * w;
-    // read now: the next item's phase 0 may rewrite them while this item's last
-    // phase still runs
-    const uint32_t tile_off = sm.tile_off[w];
-    // ---- row magnitudes: sum over the 128 columns of P^2 -------------------
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31, rg = l & 7, cg = l >> 3;
+    const int col0 = 16 * w + 4 * cg;
+    // ---- row partials of P^2 over the thread's 4 columns -------------------
     {
-        float *t = &sm.rowt[w][0][0];
+        float *T = &sm.rowp[(4 * w + cg) * kDK];
 #pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; rr++) {
-            float2 s2 = __fmul2_rn(X[rr][0], X[rr][0]);
-            s2 = __ffma2_rn(X[rr][1], X[rr][1], s2);
-            t[rr * 36 + l] = s2.x + s2.y;
-        }
-        __syncwarp();
-        const int rr = l >> 1, hf = l & 1;
-        float ss = 0.f;
+        for (int q = 0; q < 4; q++) {
+            float s[4];
 #pragma unroll
-        for (int m = 0; m < 4; m++) {
-            const float4 x = ld4(t + rr * 36 + 16 * hf + 4 * m);
-            ss += (x.x + x.y) + (x.z + x.w);
-        }
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        if (hf == 0) {
-            const int i = r0 + rr;
-            const int b = sm.rb[i];
-            float rnew = 0.f, h = 1.f, wt = 0.f;  // pivot rows: p = S, not part of any fit
-            if (b != kPivotBits) {
-                const float a = sm.ra[i];
-                float m = a * sqrt_approx(ss * (1.0f / kDV));
-                if (m == 0.f) m = 1.f;
-                rnew = (m * sm.rs[i]) * sm.rq2[i].x;
-                h = div_approx(a, rnew);
-                wt = (sm.rrho[i] * rnew) * rnew;
+            for (int e = 0; e < 4; e++) {
+                const int rr = 4 * q + e;
+                float2 s2 = __fmul2_rn(X[rr][0], X[rr][0]);
+                s2 = __ffma2_rn(X[rr][1], X[rr][1], s2);
+                s[e] = s2.x + s2.y;
             }
-            sm.rh2[i] = f2(h, h);
-            sm.rw2[i] = f2(wt, wt);
-            reinterpret_cast<float *>(item_g)[i] = rnew;
+            *reinterpret_cast<float4 *>(T + rowp_chunk(rg, q)) = make_float4(s[0], s[1], s[2], s[3]);
         }
-        __syncwarp();
     }
+    if (__syncthreads_or(!ok_in)) return kFitAbortNow;
+    bool ok_mid = true;
+    if (tid < kDK) {
+        // ---- row i: RMS over the 128 columns, new row scale, fit factors -----
+        const int i = tid, irg = i >> 4, irr = i & 15;
+        const float *src = &sm.rowp[rowp_chunk(irg, irr >> 2) + (irr & 3)];
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+        for (int bk = 0; bk < 32; bk += 4) {
+            s0 += src[(bk + 0) * kDK];
+            s1 += src[(bk + 1) * kDK];
+            s2 += src[(bk + 2) * kDK];
+            s3 += src[(bk + 3) * kDK];
+        }
+        const float ss = (s0 + s1) + (s2 + s3);
+        const int b = ROWWISE ? rec->bits[i] : B;
+        float rnew = 0.f, h = 1.f, wt = 0.f;  // pivot rows: p = S, not part of any fit
+        if (!ROWWISE || b != kPivotBits) {
+            const float a = rf.ra[i];
+            float m = a * sqrt_approx(ss * (1.0f / kDV));
+            if (m == 0.f) m = 1.f;
+            rnew = (m * rec->s[i]) * rec->rq[i];
+            h = div_approx(a, rnew);
+            wt = (rec->rho[i] * rnew) * rnew;
+        }
+        put_pair(rf.h2, i, h);
+        put_pair(rf.w2, i, wt);
+        reinterpret_cast<float *>(item_g)[i] = rnew;
+    } else {
+        ok_mid = mid();
+    }
+    const bool abort_after = __syncthreads_or(!ok_mid);
     // ---- p = P h; column maxima (of |p| / Q_i for row-wise widths) ----------
     {
         float mx[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; rr += 2) {
-            float2 p[2][2], hh[2], qq[2];
-            ld_pairs(&sm.rh2[r0 + rr], hh);
-            if (ROWWISE) ld_pairs(&sm.rq2[r0 + rr], qq);
+        for (int p = 0; p < kRowsPerGroup / 2; p++) {
+            float2 hh[2], qq[2], pv[2][2];
+            ld_pairs(rf.h2, p, rg, hh);
+            if (ROWWISE) ld_pairs(rf.q2, p, rg, qq);
 #pragma unroll
             for (int u = 0; u < 2; u++) {
-                p[u][0] = __fmul2_rn(X[rr + u][0], hh[u]);
-                p[u][1] = __fmul2_rn(X[rr + u][1], hh[u]);
-                X[rr + u][0] = p[u][0];
-                X[rr + u][1] = p[u][1];
-                if (ROWWISE) {  // pivot rows have rq2 = 0 and do not count
-                    p[u][0] = __fmul2_rn(p[u][0], qq[u]);
-                    p[u][1] = __fmul2_rn(p[u][1], qq[u]);
+                const int rr = 2 * p + u;
+                X[rr][0] = __fmul2_rn(X[rr][0], hh[u]);
+                X[rr][1] = __fmul2_rn(X[rr][1], hh[u]);
+                pv[u][0] = X[rr][0];
+                pv[u][1] = X[rr][1];
+                if (ROWWISE) {  // pivot rows have q = 0 and do not count
+                    pv[u][0] = __fmul2_rn(pv[u][0], qq[u]);
+                    pv[u][1] = __fmul2_rn(pv[u][1], qq[u]);
                 }
             }
-            mx[0] = max_abs3(mx[0], p[0][0].x, p[1][0].x);
-            mx[1] = max_abs3(mx[1], p[0][0].y, p[1][0].y);
-            mx[2] = max_abs3(mx[2], p[0][1].x, p[1][1].x);
-            mx[3] = max_abs3(mx[3], p[0][1].y, p[1][1].y);
+            mx[0] = max_abs3(mx[0], pv[0][0].x, pv[1][0].x);
+            mx[1] = max_abs3(mx[1], pv[0][0].y, pv[1][0].y);
+            mx[2] = max_abs3(mx[2], pv[0][1].x, pv[1][1].x);
+            mx[3] = max_abs3(mx[3], pv[0][1].y, pv[1][1].y);
         }
-        stash(sm, 0, f2(mx[0], mx[1]), f2(mx[2], mx[3]));
-    }
-    __syncthreads();
-    {
-        // two threads per column, each over four warps' partials
-        const int j = tid >> 1, half = tid & 1;
-        float m = max_partials4(sm, 0, j, half);
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        if (half == 0) {
-            if (!ROWWISE) m = m * sm.rq2[0].x;  // every row has the head's width
+        // maximum over the 8 lanes sharing cg: lanes rg and rg ^ 1 end with
+        // column col0 + 2 (rg >> 2 & 1) + (rg >> 1 & 1)
+        const bool hiA = rg & 4, hiB = rg & 2;
+        float k0 = hiA ? mx[2] : mx[0], k1 = hiA ? mx[3] : mx[1];
+        const float t0 = hiA ? mx[0] : mx[2], t1 = hiA ? mx[1] : mx[3];
+        k0 = fmaxf(k0, __shfl_xor_sync(kFull, t0, 4));
+        k1 = fmaxf(k1, __shfl_xor_sync(kFull, t1, 4));
+        float m = hiB ? k1 : k0;
+        m = fmaxf(m, __shfl_xor_sync(kFull, hiB ? k0 : k1, 2));
+        m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+        if constexpr (!ROWWISE) m = m * (1.0f / (float)((1 << (B - 1)) - 1));  // every row has width B
+        if ((rg & 1) == 0) {
+            const int j = col0 + 2 * hiA + hiB;
             const float c0 = (m > 0.f) ? m : 1.f;
             sm.cc0[j] = c0;
             sm.cnew[j] = c0;
             sm.ci[j] = rcp_approx(c0);
             sm.crat[j] = 1.f;
         }
+        __syncwarp();
     }
-    __syncthreads();
     // ---- impact-weighted least squares for the column scales ---------------
     // |p / c0| <= Q, so the first round needs no clipping; later rounds clip to
     // the row's range.  More than one round is a separate instantiation (MULTI)
     // so that the one-round code holds a single round body.
     if (!MULTI) {
-        if (ls_iters > 0) {
-            ls_partials<B, ROWWISE, false>(sm, X);
-            __syncthreads();
-            ls_update_columns(sm);
-            __syncthreads();
-        }
+        if (ls_iters > 0) ls_round<B, ROWWISE, false>(sm, rf, X);
     } else {
         for (int it = 0; it < ls_iters; it++) {
             if (it == 0)
-                ls_partials<B, ROWWISE, false>(sm, X);
+                ls_round<B, ROWWISE, false>(sm, rf, X);
             else
-                ls_partials<B, ROWWISE, true>(sm, X);
-            __syncthreads();
-            ls_update_columns(sm);
-            __syncthreads();
+                ls_round<B, ROWWISE, true>(sm, rf, X);
         }
     }
     // ---- requantise, pack, store -------------------------------------------
-    const float4 i4 = ld4(&sm.ci[4 * l]);
+    const float4 i4 = ld4(&sm.ci[col0]);
     const float2 ic0 = f2(i4.x, i4.y), ic1 = f2(i4.z, i4.w);
     float rat;
     {
-        const float4 r = ld4(&sm.crat[4 * l]);
+        const float4 r = ld4(&sm.crat[col0]);
         rat = fmaxf(fmaxf(r.x, r.y), fmaxf(r.z, r.w));
     }
     // the largest |p / c| of a column is at most Q c0 / c: clip only where that
-    // can reach Q + 1/2
-    rat = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(rat)));
-    uint32_t *words = reinterpret_cast<uint32_t *>(item_g + tile_off) + l;
+    // can reach Q + 1/2 (decided per warp)
+    rat = __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(rat)));
+    uint32_t *words = reinterpret_cast<uint32_t *>(item_g + kHeaderBytes) + (kStreams * W) * w + l;
     if constexpr (B > 0) {
         constexpr int Qb = (1 << (B - 1)) - 1;
         if ((float)Qb * (rat - 1.f) >= 0.49f)
@@ -417,10 +444,10 @@ __device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item
             pack_fixed<B, false>(X, ic0, ic1, words);
     } else {
         BitWriter bw;
-        bw.init(words, kGroups);
+        bw.init(words, kStreams);
 #pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; rr++) {
-            const int b = sm.rb[r0 + rr];
+        for (int rr = 0; rr < kRowsPerGroup; rr++) {
+            const int b = rf.rb[8 * rr + rg];
             if (b == kPivotBits) {
 #pragma unroll
                 for (int hh = 0; hh < 2; hh++) {
@@ -451,8 +478,10 @@ __device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item
             }
         }
         bw.flush();
+        for (int m = bw.next; m < W; m++) words[m * kStreams] = 0u;  // the stream's padding words
     }
-    if (tid < kDV) reinterpret_cast<float *>(item_g)[kDK + tid] = store_c ? sm.cnew[tid] : 0.f;
+    if (l < 16) reinterpret_cast<float *>(item_g)[kDK + 16 * w + l] = store_c ? sm.cnew[16 * w + l] : 0.f;
+    return abort_after ? kFitAbortAfter : kFitDone;
 }
 
 // ---------------------------------------------------------------------------
@@ -463,192 +492,234 @@ __device__ __forceinline__ void fit_and_store(ItemSmem &sm, X2 &X, uint8_t *item
 // ahead of the compute.
 // ---------------------------------------------------------------------------
 
-// An item of an all-pivot head: binary16 state, update and readout, no fit.
-__device__ void pivot_item(ItemSmem &sm, const StepArgs &a, int item)
+// An item of an all-pivot head, straight from global memory: binary16 state,
+// update and readout, no fit.  Every row of the item is a pivot row, so each
+// stream holds 16 rows x 4 binary16 values (two words per row), and each
+// thread derives its own rows' factors; no barrier.
+__device__ void pivot_item(const StepArgs &a, int item)
 {
-    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31, rg = l & 7, cg = l >> 3;
+    const int col0 = 16 * w + 4 * cg;
     const int rq = item / a.heads, h = item - rq * a.heads;
-    const HeadRec *rec = a.t.rowrec + h;
     uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + a.t.head_off[h];
-    const long long vec = (long long)item * kDK;
+    const long long vec = (long long)item * kDK + kRowsPerGroup * rg;
     const float beta = a.beta[item];
-    if (tid < kDK) {
-        const int i = tid;
-        const float al = a.kda ? a.alpha[vec + i] : a.alpha[item];
-        const float k = a.k[vec + i], q = a.q[vec + i];
-        sm.rk2[i] = f2(al * k, al * k);
-        sm.rl2[i] = f2(al * q, al * q);
-        sm.rg2[i] = f2(beta * k, beta * k);
-        sm.ra2[i] = f2(al, al);
-        float kq = k * q;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, o);
-        if (l == 0) sm.kq[w] = kq;
-    } else {
-        sm.cv[tid - kDK] = a.v[vec + tid - kDK];
-    }
-    __syncthreads();
-    uint32_t *words = reinterpret_cast<uint32_t *>(item_g + rec->tile_off[w]) + l;
+    uint32_t *words = reinterpret_cast<uint32_t *>(item_g + kHeaderBytes) + (kStreams * 2 * kRowsPerGroup) * w + l;
     X2 X;
     float2 V0 = f2(0.f, 0.f), V1 = V0, U0 = V0, U1 = V0;
+    float kq = 0.f;
 #pragma unroll
-    for (int rr = 0; rr < kRowsPerWarp; rr++) {
-        const int i = kRowsPerWarp * w + rr;
-        const uint32_t w0 = words[(2 * rr) * kGroups], w1 = words[(2 * rr + 1) * kGroups];
-        const float2 h0 = __half22float2(*reinterpret_cast<const __half2 *>(&w0));
-        const float2 h1 = __half22float2(*reinterpret_cast<const __half2 *>(&w1));
-        const float2 kk = ld2(&sm.rk2[i]), ll = ld2(&sm.rl2[i]), aa = ld2(&sm.ra2[i]);
-        X[rr][0] = __fmul2_rn(aa, h0);
-        X[rr][1] = __fmul2_rn(aa, h1);
-        V0 = __ffma2_rn(kk, h0, V0);
-        V1 = __ffma2_rn(kk, h1, V1);
-        U0 = __ffma2_rn(ll, h0, U0);
-        U1 = __ffma2_rn(ll, h1, U1);
-    }
-    stash(sm, 0, V0, V1);
-    stash(sm, 1, U0, U1);
-    __syncthreads();
-    if (tid < kDV) {
-        sm.cd[tid] = sm.cv[tid] - sum_partials(sm, 0, tid);
-    } else {
-        sm.cu[tid - kDK] = sum_partials(sm, 1, tid - kDK);
-    }
-    __syncthreads();
-    if (tid < kDV) {
-        const float kq = (sm.kq[0] + sm.kq[1]) + (sm.kq[2] + sm.kq[3]);
-        a.out[(long long)item * kDV + tid] = fmaf(beta * kq, sm.cd[tid], sm.cu[tid]);
-    }
-    const float4 d4 = ld4(&sm.cd[4 * l]);
-    const float2 d0 = f2(d4.x, d4.y), d1 = f2(d4.z, d4.w);
+    for (int q4 = 0; q4 < kRowsPerGroup / 4; q4++) {
+        const float4 k4 = ld4(a.k + vec + 4 * q4), qv4 = ld4(a.q + vec + 4 * q4);
+        const float4 al4 = a.kda ? ld4(a.alpha + vec + 4 * q4) : make_float4(a.alpha[item], a.alpha[item],
+                                                                             a.alpha[item], a.alpha[item]);
+        const float kk[4] = {k4.x, k4.y, k4.z, k4.w}, qq[4] = {qv4.x, qv4.y, qv4.z, qv4.w};
+        const float aa[4] = {al4.x, al4.y, al4.z, al4.w};
 #pragma unroll
-    for (int rr = 0; rr < kRowsPerWarp; rr++) {
-        const int i = kRowsPerWarp * w + rr;
-        const float2 gg = ld2(&sm.rg2[i]);
-        const float2 s0 = __ffma2_rn(gg, d0, X[rr][0]), s1 = __ffma2_rn(gg, d1, X[rr][1]);
-        const __half2 h0 = __floats2half2_rn(s0.x, s0.y);
-        const __half2 h1 = __floats2half2_rn(s1.x, s1.y);
-        words[(2 * rr) * kGroups] = *reinterpret_cast<const uint32_t *>(&h0);
-        words[(2 * rr + 1) * kGroups] = *reinterpret_cast<const uint32_t *>(&h1);
+        for (int e = 0; e < 4; e++) {
+            const int rr = 4 * q4 + e;
+            const uint32_t w0 = words[(2 * rr) * kStreams], w1 = words[(2 * rr + 1) * kStreams];
+            const float2 h0 = __half22float2(*reinterpret_cast<const __half2 *>(&w0));
+            const float2 h1 = __half22float2(*reinterpret_cast<const __half2 *>(&w1));
+            const float2 a2 = f2(aa[e], aa[e]);
+            const float2 kp = f2(aa[e] * kk[e], aa[e] * kk[e]), lp = f2(aa[e] * qq[e], aa[e] * qq[e]);
+            X[rr][0] = __fmul2_rn(a2, h0);
+            X[rr][1] = __fmul2_rn(a2, h1);
+            V0 = __ffma2_rn(kp, h0, V0);
+            V1 = __ffma2_rn(kp, h1, V1);
+            U0 = __ffma2_rn(lp, h0, U0);
+            U1 = __ffma2_rn(lp, h1, U1);
+            kq = fmaf(kk[e], qq[e], kq);
+        }
     }
-    __syncthreads();
+    // k.q over all rows: the 8 row groups are the lanes sharing cg
+    kq += __shfl_xor_sync(kFull, kq, 1);
+    kq += __shfl_xor_sync(kFull, kq, 2);
+    kq += __shfl_xor_sync(kFull, kq, 4);
+    // lane rg: v_old (rg < 4) or the query projection (rg >= 4) of column col0 + (rg & 3)
+    const float part = reduce_scatter_2x4(V0, V1, U0, U1, rg);
+    const int j = col0 + (rg & 3);
+    const float d = a.v[(long long)item * kDV + j] - part;
+    const float d_col = __shfl_xor_sync(kFull, d, 4);
+    if (rg >= 4) a.out[(long long)item * kDV + j] = fmaf(beta * kq, d_col, part);
+    // d of the thread's four columns: lanes cg*8 + 0..3 hold them
+    float dd[4];
+#pragma unroll
+    for (int e = 0; e < 4; e++) dd[e] = __shfl_sync(kFull, d, 8 * cg + e);
+    const float2 d0 = f2(dd[0], dd[1]), d1 = f2(dd[2], dd[3]);
+#pragma unroll
+    for (int q4 = 0; q4 < kRowsPerGroup / 4; q4++) {
+        const float4 k4 = ld4(a.k + vec + 4 * q4);
+        const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const int rr = 4 * q4 + e;
+            const float2 gg = f2(beta * kk[e], beta * kk[e]);
+            const float2 s0 = __ffma2_rn(gg, d0, X[rr][0]), s1 = __ffma2_rn(gg, d1, X[rr][1]);
+            const __half2 h0 = __floats2half2_rn(s0.x, s0.y);
+            const __half2 h1 = __floats2half2_rn(s1.x, s1.y);
+            words[(2 * rr) * kStreams] = *reinterpret_cast<const uint32_t *>(&h0);
+            words[(2 * rr + 1) * kStreams] = *reinterpret_cast<const uint32_t *>(&h1);
+        }
+    }
 }
 
-// Issue the bulk copies that stage one item into slot buffer sb.  st = the
-// item's staging record {item, item bytes, byte offset in the pool (lo, hi)}.
+// Stage one item into slot buffer sb, on every lane of the producer warp: the
+// packed item and the head record by bulk copies (lane 0), q, k, v (and the
+// KDA gates) as 16-byte asynchronous copies, one per lane and vector, and the
+// per-item scalars (lane 0).  All of it completes on the slot's barrier, which
+// counts lane 0's expect-tx arrival and one arrival per lane for its copies.
 template <bool KDA>
 __device__ __forceinline__ void stage_item(const StepArgs &a, int4 st, uint8_t *sb, uint64_t *bar)
 {
+    const int lane = threadIdx.x & 31;
     const int item = st.x, h = item % a.heads;
-    const uint32_t bytes = (uint32_t)st.y;
-    const uint8_t *src = a.pool + (long long)(((unsigned long long)(uint32_t)st.w << 32) | (uint32_t)st.z);
     const long long vec = (long long)item * kDK;
-    const uint32_t tx = bytes + 3u * 4u * kDK + (KDA ? 4u * kDK : 0u) + (uint32_t)sizeof(HeadRec);
-    mbar_arrive_expect_tx(bar, tx);
-    bulk_g2s(sb, src, bytes, bar);
-    bulk_g2s(sb + a.off_q, a.q + vec, 4 * kDK, bar);
-    bulk_g2s(sb + a.off_k, a.k + vec, 4 * kDK, bar);
-    bulk_g2s(sb + a.off_v, a.v + (long long)item * kDV, 4 * kDV, bar);
-    if (KDA) bulk_g2s(sb + a.off_alpha, a.alpha + vec, 4 * kDK, bar);
-    bulk_g2s(sb + a.off_rec, a.t.rowrec + h, sizeof(HeadRec), bar);
-    // the per-item scalars (GDN alpha, beta) are 4-byte copies tracked by the same barrier
-    const uint32_t dab = smem_addr(sb + a.off_ab);
-    if (!KDA) asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dab), "l"(a.alpha + item) : "memory");
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dab + 4), "l"(a.beta + item) : "memory");
+    if (lane == 0) {
+        const uint32_t bytes = (uint32_t)st.y;
+        const uint8_t *src = a.pool + (long long)(((unsigned long long)(uint32_t)st.w << 32) | (uint32_t)st.z);
+        mbar_arrive_expect_tx(bar, bytes + (uint32_t)sizeof(HeadRec));
+        bulk_g2s(sb, src, bytes, bar);
+        bulk_g2s(sb + a.off_rec, a.t.rowrec + h, sizeof(HeadRec), bar);
+        const uint32_t dab = smem_addr(sb + a.off_ab);
+        if (!KDA) asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dab), "l"(a.alpha + item) : "memory");
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dab + 4), "l"(a.beta + item) : "memory");
+    }
+    const uint32_t o = 16u * lane;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(sb + a.off_q) + o), "l"(a.q + vec + 4 * lane)
+                 : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(sb + a.off_k) + o), "l"(a.k + vec + 4 * lane)
+                 : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(sb + a.off_v) + o),
+                 "l"(a.v + (long long)item * kDV + 4 * lane)
+                 : "memory");
+    if (KDA)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(sb + a.off_alpha) + o),
+                     "l"(a.alpha + vec + 4 * lane)
+                     : "memory");
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// Producer state, used by thread 0 only and kept in shared memory so that it
-// costs no registers in the other threads: the next position to stage, the
-// number staged so far, and that position's staging record, fetched one issue
-// ahead with an asynchronous copy so that no global load stalls the thread.
+// Arrivals that complete one staging: lane 0's expect-tx arrival and the 32
+// lanes' asynchronous-copy arrivals.
+constexpr uint32_t kStageArrivals = 1 + 32;
+
+// Producer state, used by the producer warp only and kept in shared memory so
+// that it costs no registers elsewhere: the next position to stage, the number
+// staged so far, and that position's staging record, fetched one issue ahead
+// by an asynchronous copy (lane 0) so that no global load stalls the warp.
 __device__ __forceinline__ void prefetch_stage_rec(ItemSmem &sm, const StepArgs &a)
 {
-    if (sm.prod_n < a.n_items)
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_addr(&sm.prod_rec)),
-                     "l"(a.t.stage + sm.prod_n)
-                     : "memory");
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// Stage the next position into slot buffer sb (thread 0).
-template <bool KDA>
-__device__ __forceinline__ void produce(ItemSmem &sm, const StepArgs &a, uint8_t *sb, uint64_t *bar)
-{
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    stage_item<KDA>(a, sm.prod_rec, sb, bar);
-    sm.prod_n += gridDim.x;
-    sm.prod_issued++;
-    prefetch_stage_rec(sm, a);
-}
-
-// Phase 0 of a staged item: per-row and per-column factors from the slot.
-template <bool KDA>
-__device__ __forceinline__ void phase0(ItemSmem &sm, const StepArgs &a, const uint8_t *sb)
-{
-    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
-    const HeadRec *rec = reinterpret_cast<const HeadRec *>(sb + a.off_rec);
-    const float *s_r = reinterpret_cast<const float *>(sb);
-    const float *s_c = s_r + kDK;
-    const float beta = *reinterpret_cast<const float *>(sb + a.off_ab + 4);
-    if (tid < kDK) {
-        const int i = tid;
-        const int b = rec->bits[i];
-        const float al = KDA ? reinterpret_cast<const float *>(sb + a.off_alpha)[i]
-                             : *reinterpret_cast<const float *>(sb + a.off_ab);
-        const float k = reinterpret_cast<const float *>(sb + a.off_k)[i];
-        const float q = reinterpret_cast<const float *>(sb + a.off_q)[i];
-        float A, g, qi = 0.f, s = 0.f, rh = 0.f;
-        if (b == kPivotBits) {
-            A = al;
-            g = beta * k;
-        } else {
-            A = al * s_r[i];
-            g = __fdiv_rn(beta * k, A);
-            qi = __frcp_rn((float)qmax_of(b));
-            s = rec->s[i];
-            rh = rec->rho[i];
-        }
-        sm.rk2[i] = f2(A * k, A * k);
-        sm.rl2[i] = f2(A * q, A * q);
-        sm.rg2[i] = f2(g, g);
-        sm.ra2[i] = f2(al, al);
-        sm.rq2[i] = f2(qi, qi);
-        sm.ra[i] = A;
-        sm.rs[i] = s;
-        sm.rrho[i] = rh;
-        sm.rb[i] = b;
-        float kq = k * q;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, o);
-        if (l == 0) sm.kq[w] = kq;
-    } else {
-        const int j = tid - kDK;
-        sm.cc[j] = s_c[j];
-        sm.cv[j] = reinterpret_cast<const float *>(sb + a.off_v)[j];
-        if (j < kTiles) sm.tile_off[j] = rec->tile_off[j];
-        if (j == kTiles) {
-            sm.head_b = rec->head_b;
-            sm.head_kind = rec->head_kind;
-            sm.head_off = rec->head_off;
-            sm.beta_item = beta;
-        }
+    if ((threadIdx.x & 31) == 0) {
+        if (sm.prod_n < a.n_items)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_addr(&sm.prod_rec)),
+                         "l"(a.t.stage + sm.prod_n)
+                         : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
     }
 }
 
-// Phases after phase 0 of a staged item: reconstruct + project, release the
-// slot (stage the next item into it), Delta update, readout, fit, store.
-template <int B, bool KDA, bool MULTI>
-__device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int item, const uint8_t *sb, int slot,
-                                         uint8_t *ring)
+// Stage the next position into slot buffer sb (the whole producer warp; the
+// caller checks sm.prod_n < n_items, a warp-uniform condition).
+template <bool KDA>
+__device__ __forceinline__ void produce(ItemSmem &sm, const StepArgs &a, uint8_t *sb, uint64_t *bar)
 {
-    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
-    const int r0 = kRowsPerWarp * w;
-    constexpr bool ROWWISE = (B == 0);
-    X2 X;
-    // ---- phase A: codes -> floats, key and query projections ---------------
-    decode_stream<B>(sm, reinterpret_cast<const uint32_t *>(sb + sm.tile_off[w]) + l, kGroups, X);
+    if ((threadIdx.x & 31) == 0) asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncwarp();
+    const int4 st = sm.prod_rec;
+    __syncwarp();
+    stage_item<KDA>(a, st, sb, bar);
+    if ((threadIdx.x & 31) == 0) {
+        sm.prod_n += gridDim.x;
+        sm.prod_issued++;
+    }
+    __syncwarp();
+    prefetch_stage_rec(sm, a);
+}
+
+// Phase 0 of a staged item (threads 128..255, row i = tid - 128): per-row
+// factors from the slot into rf.  Runs while the previous item's state is live
+// in registers, hence the call-free quotient.
+template <bool KDA>
+__device__ __forceinline__ void phase0(RowFactors &rf, const StepArgs &a, const uint8_t *sb, int item)
+{
+    const int i = threadIdx.x - kDK;
+    const HeadRec *rec = reinterpret_cast<const HeadRec *>(sb + a.off_rec);
+    const float beta = *reinterpret_cast<const float *>(sb + a.off_ab + 4);
+    const int b = rec->bits[i];
+    const float al = KDA ? reinterpret_cast<const float *>(sb + a.off_alpha)[i]
+                         : *reinterpret_cast<const float *>(sb + a.off_ab);
+    const float k = reinterpret_cast<const float *>(sb + a.off_k)[i];
+    const float q = reinterpret_cast<const float *>(sb + a.off_q)[i];
+    const float r = reinterpret_cast<const float *>(sb)[i];
+    float A, g;
+    if (b == kPivotBits) {
+        A = al;
+        g = beta * k;
+    } else {
+        A = al * r;
+        g = div_approx(beta * k, A);
+    }
+    put_pair(rf.k2, i, A * k);
+    put_pair(rf.l2, i, A * q);
+    put_pair(rf.g2, i, g);
+    if (KDA) {
+        put_pair(rf.a2, i, al);
+        put_pair(rf.q2, i, rec->rq[i]);
+    }
+    rf.ra[i] = A;
+    if (KDA) rf.rb[sslot(i)] = b;
+    float kq = k * q;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(kFull, kq, o);
+    if ((i & 31) == 0) rf.kqp[i >> 5] = kq;
+    if (i == 0) {
+        rf.beta = beta;
+        rf.item = item;
+        rf.head_b = rec->head_b;
+    }
+}
+
+// Work between the fit's two barriers of staged item n, on threads 128..255:
+// phase 0 of the CTA's next staged item into the other factor buffer.
+// Returns false if that item's copy never landed.
+template <bool KDA>
+struct StageNext {
+    ItemSmem &sm;
+    const StepArgs &a;
+    uint8_t *ring;
+    int next_pos;      // position of the next staged item (>= n_items: none)
+    uint32_t n_next;   // its consumption count
+    RowFactors &rf_next;
+    __device__ __forceinline__ bool operator()() const
     {
-        const float4 c4 = ld4(&sm.cc[4 * l]);
+        if (next_pos >= a.n_items) return true;
+        const int s = (int)(n_next % (uint32_t)a.nslots);
+        if (!mbar_wait_bounded(&sm.bar[s], (n_next / (uint32_t)a.nslots) & 1u, kWaitLimit)) return false;
+        phase0<KDA>(rf_next, a, ring + s * a.slot_bytes, a.t.order[next_pos]);
+        return true;
+    }
+};
+
+// A staged item: reconstruct + project (phase A), read out, Delta update
+// (phase B), then the fit, during which the next item is prepared.  The slot
+// sb stays untouched until the fit's second barrier.
+template <int B, bool KDA, bool MULTI>
+__device__ __forceinline__ FitResult run_item(ItemSmem &sm, const StepArgs &a, RowFactors &rf, const uint8_t *sb,
+                                              bool ok_slot, const StageNext<KDA> &next)
+{
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31, rg = l & 7, cg = l >> 3;
+    const int col0 = 16 * w + 4 * cg;
+    constexpr bool ROWWISE = (B == 0);
+    const int item = rf.item;
+    const HeadRec *rec = reinterpret_cast<const HeadRec *>(sb + a.off_rec);
+    const int W = (B > 0) ? 2 * B : rec->slab_words;
+    X2 X;
+    // ---- phase A: codes -> floats, key and query projections, readout -------
+    decode_stream<B>(rf.rb + rg, reinterpret_cast<const uint32_t *>(sb + kHeaderBytes) + (kStreams * W) * w + l, X);
+    const float *s_c = reinterpret_cast<const float *>(sb) + kDK;
+    const float4 c4 = ld4(s_c + col0);
+    {
         float2 V0 = f2(0.f, 0.f), V1 = V0, U0 = V0, U1 = V0;
         float2 ic0 = V0, ic1 = V0;
         if (ROWWISE) {
@@ -656,23 +727,24 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
             ic1 = f2(rcp_approx(c4.z), rcp_approx(c4.w));
         }
 #pragma unroll
-        for (int r2 = 0; r2 < kRowsPerWarp; r2 += 2) {
+        for (int p = 0; p < kRowsPerGroup / 2; p++) {
             float2 kp[2], lp[2];
-            ld_pairs(&sm.rk2[r0 + r2], kp);
-            ld_pairs(&sm.rl2[r0 + r2], lp);
+            ld_pairs(rf.k2, p, rg, kp);
+            ld_pairs(rf.l2, p, rg, lp);
 #pragma unroll
             for (int u = 0; u < 2; u++) {
-                const int rr = r2 + u, i = r0 + rr;
-                if (ROWWISE && sm.rb[i] == kPivotBits) {
+                const int rr = 2 * p + u;
+                if (ROWWISE && rf.rb[8 * rr + rg] == kPivotBits) {
                     // a pivot value enters the projections in units of c_j; S' = alpha h
                     const float2 hs0 = __fmul2_rn(X[rr][0], ic0), hs1 = __fmul2_rn(X[rr][1], ic1);
                     V0 = __ffma2_rn(kp[u], hs0, V0);
                     V1 = __ffma2_rn(kp[u], hs1, V1);
                     U0 = __ffma2_rn(lp[u], hs0, U0);
                     U1 = __ffma2_rn(lp[u], hs1, U1);
-                    const float2 aa = ld2(&sm.ra2[i]);
-                    X[rr][0] = __fmul2_rn(aa, X[rr][0]);
-                    X[rr][1] = __fmul2_rn(aa, X[rr][1]);
+                    float2 aa[2];
+                    ld_pairs(rf.a2, p, rg, aa);
+                    X[rr][0] = __fmul2_rn(aa[u], X[rr][0]);
+                    X[rr][1] = __fmul2_rn(aa[u], X[rr][1]);
                 } else {
                     V0 = __ffma2_rn(kp[u], X[rr][0], V0);
                     V1 = __ffma2_rn(kp[u], X[rr][1], V1);
@@ -681,52 +753,42 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
                 }
             }
         }
-        stash(sm, 0, V0, V1);
-        stash(sm, 1, U0, U1);
-    }
-    __syncthreads();
-    // the slot has been read by every thread: stage the next item into it
-    if (tid == 0 && sm.prod_n < a.n_items) produce<KDA>(sm, a, ring + slot * a.slot_bytes, &sm.bar[slot]);
-    {
-        // two threads per column, each over four warps' partials
-        const int j = tid >> 1, half = tid & 1;
-        float vs = sum_partials4(sm, 0, j, half), us = sum_partials4(sm, 1, j, half);
-        vs += __shfl_xor_sync(0xffffffffu, vs, 1);
-        us += __shfl_xor_sync(0xffffffffu, us, 1);
-        const float c = sm.cc[j];
-        if (half == 0) {
-            const float d = sm.cv[j] - c * vs;
-            sm.cd[j] = d;
+        // lane rg: the key projection (rg < 4) or the query projection (rg >= 4)
+        // of column j, in units of c_j
+        const float part = reduce_scatter_2x4(V0, V1, U0, U1, rg);
+        const int j = col0 + (rg & 3);
+        const float c = s_c[j];
+        const float d = reinterpret_cast<const float *>(sb + a.off_v)[j] - c * part;
+        if (rg < 4) {
             sm.cdt[j] = div_approx(d, c);
-        } else {
-            sm.cu[j] = c * us;
+            if (ROWWISE) sm.cd[j] = d;
         }
-    }
-    __syncthreads();
-    if (tid < kDV) {
-        const float kq = (sm.kq[0] + sm.kq[1]) + (sm.kq[2] + sm.kq[3]);
-        a.out[(long long)item * kDV + tid] = fmaf(sm.beta_item * kq, sm.cd[tid], sm.cu[tid]);
+        const float d_col = __shfl_xor_sync(kFull, d, 4);
+        if (rg >= 4) {
+            const float kq = (rf.kqp[0] + rf.kqp[1]) + (rf.kqp[2] + rf.kqp[3]);
+            a.out[(long long)item * kDV + j] = fmaf(rf.beta * kq, d_col, c * part);
+        }
+        __syncwarp();
     }
     // ---- phase B: Delta update in old-scale units; P = S / a ----------------
     {
-        const float4 c4 = ld4(&sm.cc[4 * l]);
         const float2 c0 = f2(c4.x, c4.y), c1 = f2(c4.z, c4.w);
-        const float4 t4 = ld4(&sm.cdt[4 * l]);
+        const float4 t4 = ld4(&sm.cdt[col0]);
         const float2 dt0 = f2(t4.x, t4.y), dt1 = f2(t4.z, t4.w);
         float2 dd0 = dt0, dd1 = dt1;
         if (ROWWISE) {
-            const float4 d4 = ld4(&sm.cd[4 * l]);
+            const float4 d4 = ld4(&sm.cd[col0]);
             dd0 = f2(d4.x, d4.y);
             dd1 = f2(d4.z, d4.w);
         }
 #pragma unroll
-        for (int r2 = 0; r2 < kRowsPerWarp; r2 += 2) {
+        for (int p = 0; p < kRowsPerGroup / 2; p++) {
             float2 gp[2];
-            ld_pairs(&sm.rg2[r0 + r2], gp);
+            ld_pairs(rf.g2, p, rg, gp);
 #pragma unroll
             for (int u = 0; u < 2; u++) {
-                const int rr = r2 + u, i = r0 + rr;
-                if (ROWWISE && sm.rb[i] == kPivotBits) {
+                const int rr = 2 * p + u;
+                if (ROWWISE && rf.rb[8 * rr + rg] == kPivotBits) {
                     X[rr][0] = __ffma2_rn(gp[u], dd0, X[rr][0]);
                     X[rr][1] = __ffma2_rn(gp[u], dd1, X[rr][1]);
                 } else {
@@ -737,11 +799,23 @@ __device__ __forceinline__ void run_item(ItemSmem &sm, const StepArgs &a, int it
         }
     }
     const int rq = item / a.heads;
-    uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + sm.head_off;
-    fit_and_store<B, ROWWISE, MULTI>(sm, X, item_g, a.ls_iters);
-    // the row-wise store reads the row widths, which the next item's phase 0
-    // rewrites; the fixed-width store reads no shared state phase 0 writes
-    if (ROWWISE) __syncthreads();
+    uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + rec->head_off;
+    return fit_and_store<B, ROWWISE, MULTI>(sm, rf, rec, X, item_g, W, a.ls_iters, true, ok_slot, next);
+}
+
+// After a failed wait: record it, let every copy that may still be in flight
+// (consumption counts first_pending .. issued - 1) land, then the CTA returns.
+__device__ __forceinline__ void abort_drain(ItemSmem &sm, const StepArgs &a, uint32_t first_pending, int code)
+{
+    if ((threadIdx.x >> 5) == kProducerWarp) {
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if ((threadIdx.x & 31) == 0) {
+            atomicExch(a.t.status, code);
+            for (uint32_t m = first_pending; m < sm.prod_issued; m++)
+                mbar_wait_bounded(&sm.bar[m % (uint32_t)a.nslots], (m / (uint32_t)a.nslots) & 1u, kWaitLimit);
+        }
+    }
+    __syncthreads();
 }
 
 template <bool KDA, bool MULTI>
@@ -752,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
     const int tid = threadIdx.x;
     const int G = gridDim.x;
     if (tid == 0) {
-        for (int s = 0; s < a.nslots; s++) mbar_init(&sm.bar[s], 2);
+        for (int s = 0; s < a.nslots; s++) mbar_init(&sm.bar[s], kStageArrivals);
         fence_barrier_init();
     }
     __syncthreads();
@@ -761,55 +835,70 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
     // first staged position of this CTA: the smallest n >= npiv with n = blockIdx.x (mod G)
     int n_first = blockIdx.x;
     if (n_first < npiv) n_first += ((npiv - n_first + G - 1) / G) * G;
-    if (tid == 0) {
-        sm.prod_n = n_first;
-        sm.prod_issued = 0;
+    if ((tid >> 5) == kProducerWarp) {
+        if ((tid & 31) == 0) {
+            sm.prod_n = n_first;
+            sm.prod_issued = 0;
+        }
+        __syncwarp();
         prefetch_stage_rec(sm, a);
         for (int s = 0; s < a.nslots && sm.prod_n < a.n_items; s++)
             produce<KDA>(sm, a, ring + s * a.slot_bytes, &sm.bar[s]);
     }
-    uint32_t n_cons = 0;
-    int next_item = (blockIdx.x < a.n_items) ? a.t.order[blockIdx.x] : 0;
-    for (int n = blockIdx.x; n < a.n_items; n += G) {
-        const int item = next_item;
-        if (n + G < a.n_items) next_item = a.t.order[n + G];
-        if (n < npiv) {
-            pivot_item(sm, a, item);
-            continue;
+    for (int n = blockIdx.x; n < npiv && n < a.n_items; n += G) pivot_item(a, a.t.order[n]);
+    if (n_first >= a.n_items) return;  // nothing was staged
+
+    // phase 0 of the first staged item
+    {
+        bool ok = true;
+        if (tid >= kDK) {
+            ok = mbar_wait_bounded(&sm.bar[0], 0u, kWaitLimit);
+            if (ok) phase0<KDA>(sm.u.rf[0], a, ring, a.t.order[n_first]);
         }
-        const int slot = (int)(n_cons % (uint32_t)a.nslots);
-        const uint32_t parity = (n_cons / (uint32_t)a.nslots) & 1u;
-        n_cons++;
-        const uint8_t *sb = ring + slot * a.slot_bytes;
-        const bool ok = mbar_wait_bounded(&sm.bar[slot], parity, kWaitLimit);
-        if (ok) phase0<KDA>(sm, a, sb);
         if (!__syncthreads_and(ok)) {
-            // a staged copy never completed: record it, drain what is in flight, stop
-            if (tid == 0) {
-                atomicExch(a.t.status, kStatusWaitTimeout);
-                for (uint32_t m = n_cons - 1; m < sm.prod_issued; m++)
-                    mbar_wait_bounded(&sm.bar[m % (uint32_t)a.nslots], (m / (uint32_t)a.nslots) & 1u, kWaitLimit);
-            }
-            __syncthreads();
+            abort_drain(sm, a, 0u, kStatusWaitTimeout);
             return;
         }
+    }
+    uint32_t n_cons = 0;
+    int par = 0;
+    for (int n = n_first; n < a.n_items; n += G, par ^= 1) {
+        RowFactors &rf = sm.u.rf[par];
+        const int slot = (int)(n_cons % (uint32_t)a.nslots);
+        const uint32_t parity = (n_cons / (uint32_t)a.nslots) & 1u;
+        const uint8_t *sb = ring + slot * a.slot_bytes;
+        const bool ok = mbar_wait_bounded(&sm.bar[slot], parity, kWaitLimit);
+        const StageNext<KDA> next{sm, a, ring, n + G, n_cons + 1, sm.u.rf[par ^ 1]};
+        FitResult res = kFitDone;
         if (KDA) {
-            run_item<0, KDA, MULTI>(sm, a, item, sb, slot, ring);
+            res = run_item<0, KDA, MULTI>(sm, a, rf, sb, ok, next);
         } else {
-            switch (sm.head_b) {
-                case 2: run_item<2, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
-                case 3: run_item<3, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
-                case 4: run_item<4, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
-                case 5: run_item<5, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
-                case 6: run_item<6, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
-                case 7: run_item<7, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
-                case 8: run_item<8, KDA, MULTI>(sm, a, item, sb, slot, ring); break;
+            switch (rf.head_b) {
+                case 2: res = run_item<2, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
+                case 3: res = run_item<3, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
+                case 4: res = run_item<4, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
+                case 5: res = run_item<5, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
+                case 6: res = run_item<6, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
+                case 7: res = run_item<7, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
+                case 8: res = run_item<8, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
                 default:  // unreachable: Gated-DeltaNet heads have one width, validated on the host
-                    if (tid == 0) atomicExch(a.t.status, kStatusBadHead);
-                    __syncthreads();
-                    break;
+                    abort_drain(sm, a, n_cons, kStatusBadHead);
+                    return;
             }
         }
+        if (res == kFitAbortNow) {
+            abort_drain(sm, a, n_cons, kStatusWaitTimeout);
+            return;
+        }
+        if (res == kFitAbortAfter) {
+            abort_drain(sm, a, n_cons + 1, kStatusWaitTimeout);
+            return;
+        }
+        // every warp is past the item's second barrier, so the slot is free:
+        // stage the next position into it
+        if ((tid >> 5) == kProducerWarp && sm.prod_n < a.n_items)
+            produce<KDA>(sm, a, ring + slot * a.slot_bytes, &sm.bar[slot]);
+        n_cons++;
     }
 }
 
@@ -817,105 +906,102 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
 // Pack (fit + quantise full-precision states) and unpack (dequantise): one CTA
 // per item, the same thread mapping and the same fit as the decode step.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void load_head(ItemSmem &sm, const StepArgs &a, int h)
+__device__ __forceinline__ void load_head(RowFactors &rf, const HeadRec *rec)
 {
     const int tid = threadIdx.x;
-    const HeadRec *rec = a.t.rowrec + h;
     if (tid < kDK) {
-        const int i = tid, b = rec->bits[i];
-        const float qi = (b == kPivotBits) ? 0.f : __frcp_rn((float)qmax_of(b));
-        sm.rb[i] = b;
-        sm.ra[i] = 1.f;
-        sm.rs[i] = rec->s[i];
-        sm.rrho[i] = rec->rho[i];
-        sm.rq2[i] = f2(qi, qi);
-    } else {
-        const int j = tid - kDK;
-        if (j < kTiles) sm.tile_off[j] = rec->tile_off[j];
-        if (j == kTiles) {
-            sm.head_b = rec->head_b;
-            sm.head_kind = rec->head_kind;
-            sm.head_off = rec->head_off;
-        }
+        const int i = tid;
+        rf.ra[i] = 1.f;
+        rf.rb[sslot(i)] = rec->bits[i];
+        put_pair(rf.q2, i, rec->rq[i]);
     }
 }
 
 template <int B, bool ROWWISE>
-__device__ __forceinline__ void pack_body(ItemSmem &sm, const StepArgs &a, int item, uint8_t *item_g)
+__device__ __forceinline__ void pack_body(ItemSmem &sm, RowFactors &rf, const HeadRec *rec, const StepArgs &a,
+                                          int item, uint8_t *item_g)
 {
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31, rg = l & 7, cg = l >> 3;
+    const int col0 = 16 * w + 4 * cg;
     X2 X;
     const float *src = a.S_in + (long long)item * kDK * kDV;
 #pragma unroll
-    for (int rr = 0; rr < kRowsPerWarp; rr++) {
-        const float4 x = ld4(src + (kRowsPerWarp * w + rr) * kDV + 4 * l);
+    for (int rr = 0; rr < kRowsPerGroup; rr++) {
+        const float4 x = ld4(src + (kRowsPerGroup * rg + rr) * kDV + col0);
         X[rr][0] = f2(x.x, x.y);
         X[rr][1] = f2(x.z, x.w);
     }
-    fit_and_store<B, ROWWISE, true>(sm, X, item_g, a.ls_iters, sm.head_kind != kHeadAllPivot);
+    fit_and_store<B, ROWWISE, true>(sm, rf, rec, X, item_g, (B > 0) ? 2 * B : rec->slab_words, a.ls_iters,
+                                    rec->head_kind != kHeadAllPivot, true, NoMid{});
 }
 
 __global__ void __launch_bounds__(kThreads) k_pack(StepArgs a)
 {
     __shared__ ItemSmem sm;
+    RowFactors &rf = sm.u.rf[0];
     const int item = blockIdx.x;
     const int rq = item / a.heads, h = item - rq * a.heads;
-    load_head(sm, a, h);
+    const HeadRec *rec = a.t.rowrec + h;
+    load_head(rf, rec);
     __syncthreads();
-    uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + sm.head_off;
-    switch (sm.head_kind == kHeadQuant ? sm.head_b : 0) {
-        case 2: pack_body<2, false>(sm, a, item, item_g); break;
-        case 3: pack_body<3, false>(sm, a, item, item_g); break;
-        case 4: pack_body<4, false>(sm, a, item, item_g); break;
-        case 5: pack_body<5, false>(sm, a, item, item_g); break;
-        case 6: pack_body<6, false>(sm, a, item, item_g); break;
-        case 7: pack_body<7, false>(sm, a, item, item_g); break;
-        case 8: pack_body<8, false>(sm, a, item, item_g); break;
-        default: pack_body<0, true>(sm, a, item, item_g); break;
+    uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + rec->head_off;
+    switch (rec->head_kind == kHeadQuant ? rec->head_b : 0) {
+        case 2: pack_body<2, false>(sm, rf, rec, a, item, item_g); break;
+        case 3: pack_body<3, false>(sm, rf, rec, a, item, item_g); break;
+        case 4: pack_body<4, false>(sm, rf, rec, a, item, item_g); break;
+        case 5: pack_body<5, false>(sm, rf, rec, a, item, item_g); break;
+        case 6: pack_body<6, false>(sm, rf, rec, a, item, item_g); break;
+        case 7: pack_body<7, false>(sm, rf, rec, a, item, item_g); break;
+        case 8: pack_body<8, false>(sm, rf, rec, a, item, item_g); break;
+        default: pack_body<0, true>(sm, rf, rec, a, item, item_g); break;
     }
 }
 
 template <int B>
-__device__ __forceinline__ void unpack_body(ItemSmem &sm, const StepArgs &a, int item, const uint8_t *item_g)
+__device__ __forceinline__ void unpack_body(const RowFactors &rf, const HeadRec *rec, const StepArgs &a, int item,
+                                            const uint8_t *item_g)
 {
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31, rg = l & 7, cg = l >> 3;
+    const int col0 = 16 * w + 4 * cg;
     X2 X;
-    decode_stream<B>(sm, reinterpret_cast<const uint32_t *>(item_g + sm.tile_off[w]) + l, kGroups, X);
+    const int W = (B > 0) ? 2 * B : rec->slab_words;
+    decode_stream<B>(rf.rb + rg, reinterpret_cast<const uint32_t *>(item_g + kHeaderBytes) + (kStreams * W) * w + l, X);
     const float *r = reinterpret_cast<const float *>(item_g);
-    const float4 c4 = ld4(r + kDK + 4 * l);
+    const float4 c4 = ld4(r + kDK + col0);
     float *dst = a.S_out + (long long)item * kDK * kDV;
 #pragma unroll
-    for (int rr = 0; rr < kRowsPerWarp; rr++) {
-        const int i = kRowsPerWarp * w + rr;
+    for (int rr = 0; rr < kRowsPerGroup; rr++) {
+        const int i = kRowsPerGroup * rg + rr;
         float4 y;
-        if (B == 0 && sm.rb[i] == kPivotBits) {
+        if (B == 0 && rf.rb[8 * rr + rg] == kPivotBits) {
             y = make_float4(X[rr][0].x, X[rr][0].y, X[rr][1].x, X[rr][1].y);
         } else {
             const float ri = r[i];
             y = make_float4(__fmul_rn(__fmul_rn(ri, c4.x), X[rr][0].x), __fmul_rn(__fmul_rn(ri, c4.y), X[rr][0].y),
                             __fmul_rn(__fmul_rn(ri, c4.z), X[rr][1].x), __fmul_rn(__fmul_rn(ri, c4.w), X[rr][1].y));
         }
-        *reinterpret_cast<float4 *>(dst + i * kDV + 4 * l) = y;
+        *reinterpret_cast<float4 *>(dst + i * kDV + col0) = y;
     }
 }
 
 __global__ void __launch_bounds__(kThreads) k_unpack(StepArgs a)
 {
-    __shared__ ItemSmem sm;
+    __shared__ RowFactors rf;
     const int item = blockIdx.x;
     const int rq = item / a.heads, h = item - rq * a.heads;
-    load_head(sm, a, h);
+    const HeadRec *rec = a.t.rowrec + h;
+    load_head(rf, rec);
     __syncthreads();
-    const uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + sm.head_off;
-    switch (sm.head_kind == kHeadQuant ? sm.head_b : 0) {
-        case 2: unpack_body<2>(sm, a, item, item_g); break;
-        case 3: unpack_body<3>(sm, a, item, item_g); break;
-        case 4: unpack_body<4>(sm, a, item, item_g); break;
-        case 5: unpack_body<5>(sm, a, item, item_g); break;
-        case 6: unpack_body<6>(sm, a, item, item_g); break;
-        case 7: unpack_body<7>(sm, a, item, item_g); break;
-        case 8: unpack_body<8>(sm, a, item, item_g); break;
-        default: unpack_body<0>(sm, a, item, item_g); break;
+    const uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + rec->head_off;
+    switch (rec->head_kind == kHeadQuant ? rec->head_b : 0) {
+        case 2: unpack_body<2>(rf, rec, a, item, item_g); break;
+        case 3: unpack_body<3>(rf, rec, a, item, item_g); break;
+        case 4: unpack_body<4>(rf, rec, a, item, item_g); break;
+        case 5: unpack_body<5>(rf, rec, a, item, item_g); break;
+        case 6: unpack_body<6>(rf, rec, a, item, item_g); break;
+        case 7: unpack_body<7>(rf, rec, a, item, item_g); break;
+        case 8: unpack_body<8>(rf, rec, a, item, item_g); break;
+        default: unpack_body<0>(rf, rec, a, item, item_g); break;
     }
 }
 
@@ -939,11 +1025,11 @@ __global__ void __launch_bounds__(kThreads) k_fp32_step(float *Sg, const float *
     }
     __syncthreads();
     float *Sp = Sg + item * kDK * kDV;
-    float S[kRowsPerWarp][4];
+    float S[kRowsPerGroup][4];
     float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int ii = 0; ii < kRowsPerWarp; ii++) {
-        const int i = kRowsPerWarp * w + ii;
+    for (int ii = 0; ii < kRowsPerGroup; ii++) {
+        const int i = kRowsPerGroup * w + ii;
         const float4 x = *reinterpret_cast<const float4 *>(Sp + i * kDV + 4 * l);
         S[ii][0] = sa[i] * x.x; S[ii][1] = sa[i] * x.y; S[ii][2] = sa[i] * x.z; S[ii][3] = sa[i] * x.w;
 #pragma unroll
@@ -963,8 +1049,8 @@ __global__ void __launch_bounds__(kThreads) k_fp32_step(float *Sg, const float *
     for (int kk = 0; kk < 4; kk++) { d[kk] = scol[4 * l + kk]; part[kk] = 0.f; }
     const float bt = beta[item];
 #pragma unroll
-    for (int ii = 0; ii < kRowsPerWarp; ii++) {
-        const int i = kRowsPerWarp * w + ii;
+    for (int ii = 0; ii < kRowsPerGroup; ii++) {
+        const int i = kRowsPerGroup * w + ii;
         const float g = bt * sk[i];
 #pragma unroll
         for (int kk = 0; kk < 4; kk++) {

@@ -301,21 +301,23 @@ def parity_requests(cfg: Config):
 # packed pool layout (format arithmetic only)
 # ----------------------------------------------------------------------------
 
-TILE_ROWS, GROUP_COLS = 16, 4
+GROUP_ROWS, GROUP_COLS, SLAB_COLS = 16, 4, 16
 
 
-def tile_words(bits: np.ndarray) -> np.ndarray:
-    """32-bit words per column-group stream of each 16-row tile: [H, dk/16]."""
+def stream_words(bits: np.ndarray) -> np.ndarray:
+    """32-bit words per stream of each head, [H]: the most any 16-row group
+    needs for its 4 columns' fields."""
     H, dk = bits.shape
-    per_tile = bits.astype(np.int64).reshape(H, dk // TILE_ROWS, TILE_ROWS).sum(axis=2)
-    return (GROUP_COLS * per_tile + 31) // 32
+    per_group = bits.astype(np.int64).reshape(H, dk // GROUP_ROWS, GROUP_ROWS).sum(axis=2)
+    return ((GROUP_COLS * per_group + 31) // 32).max(axis=1)
 
 
 def head_item_bytes(bits: np.ndarray, dv: int) -> np.ndarray:
-    """Bytes of one packed (request, head) item: r[dk] f32 | c[dv] f32 | tiles,
-    a tile holding dv/4 interleaved streams of tile_words words each."""
+    """Bytes of one packed (request, head) item: r[dk] f32 | c[dv] f32 | slabs,
+    dv/16 slabs of (dk/16) * 4 interleaved streams of stream_words words each."""
     dk = bits.shape[1]
-    return 4 * dk + 4 * dv + 4 * (dv // GROUP_COLS) * tile_words(bits).sum(axis=1)
+    n_streams = (dk // GROUP_ROWS) * GROUP_COLS
+    return 4 * dk + 4 * dv + 4 * n_streams * (dv // SLAB_COLS) * stream_words(bits)
 
 
 def item_offsets(bits: np.ndarray, dv: int, batch: int) -> np.ndarray:

@@ -314,7 +314,7 @@ def stream_words(fields, nwords):
     return [(acc >> (32 * w)) & 0xFFFFFFFF for w in range(nwords)]
 
 
-def test_pack_format_tiled_streams():
+def test_pack_format_slab_streams():
     r = rng(11)
     dk, dv = 128, 128
     bits = r.choice([2, 3, 4, 5, 6, 7, 8, 16], size=dk).astype(np.uint8)
@@ -327,30 +327,29 @@ def test_pack_format_tiled_streams():
             code[i] = r.integers(-Q, Q + 1, dv)
     rr = r.standard_normal(dk).astype(np.float32); cc = r.standard_normal(dv).astype(np.float32)
     item = oracle.pack_item(bits, rr, cc, code, piv)
-    words_per_tile = [(4 * int(bits[16 * T:16 * T + 16].astype(int).sum()) + 31) // 32 for T in range(8)]
-    assert item.size == 4 * dk + 4 * dv + 128 * sum(words_per_tile)
+    # W: the most words any 16-row group needs for 4 columns' fields
+    Wh = max((4 * int(bits[16 * g:16 * g + 16].astype(int).sum()) + 31) // 32 for g in range(8))
+    assert item.size == 4 * dk + 4 * dv + 8 * 32 * 4 * Wh
     assert bytes(item[:4 * dk]) == rr.astype("<f4").tobytes()
     assert bytes(item[4 * dk: 4 * dk + 4 * dv]) == cc.astype("<f4").tobytes()
     words = item[4 * dk + 4 * dv:].view("<u4")
-    base = 0
-    for T in range(8):
-        W_T = words_per_tile[T]
-        tile = words[base: base + 32 * W_T].reshape(W_T, 32)  # word w of stream g at w*32 + g
-        for g in range(32):
+    for s_ in range(8):
+        slab = words[s_ * 32 * Wh:(s_ + 1) * 32 * Wh].reshape(Wh, 32)  # word m of stream l at 32 m + l
+        for l in range(32):
+            g, cg = l % 8, l // 8
             fields = []
             for rho_ in range(16):
-                i = 16 * T + rho_
+                i = 16 * g + rho_
                 b = int(bits[i])
                 for k in range(4):
-                    j = 4 * g + k
+                    j = 16 * s_ + 4 * cg + k
                     if b == 16:
                         fields.append((int(np.array([piv[i, j]], "<f2").view("<u2")[0]), 16))
                     else:
                         u = code[i, j] + (1 << (b - 1))
                         assert 1 <= u <= (1 << b) - 1
                         fields.append((u, b))
-            assert list(tile[:, g]) == stream_words(fields, W_T), (T, g)
-        base += 32 * W_T
+            assert list(slab[:, l]) == stream_words(fields, Wh), (s_, l)
     back = oracle.unpack_item(bits, item, dk, dv)
     np.testing.assert_array_equal(back["code"], code)
     np.testing.assert_array_equal(back["piv"], piv)
@@ -358,7 +357,7 @@ def test_pack_format_tiled_streams():
 
 
 def test_golden_pack_streams():
-    """Hand-derived column-group streams (tests/golden/pack_streams.txt)."""
+    """Hand-derived streams (tests/golden/pack_streams.txt)."""
     import os
     path = os.path.join(os.path.dirname(__file__), "golden", "pack_streams.txt")
     n = 0
@@ -378,12 +377,12 @@ def test_golden_pack_streams():
         item = oracle.pack_item(bits, np.zeros(128), np.zeros(128), code, np.zeros((128, 128)))
         want = [int(x, 16) for x in hex_s.split()]
         words = item[1024:].view("<u4")
-        W_T = len(want)
-        assert words.size == 8 * 32 * W_T
-        for T in range(8):
-            tile = words[T * 32 * W_T:(T + 1) * 32 * W_T].reshape(W_T, 32)
-            for g in (0, 7, 31):
-                assert list(tile[:, g]) == want, (line, T, g)
+        Wh = len(want)
+        assert words.size == 8 * 32 * Wh
+        for s_ in range(8):
+            slab = words[s_ * 32 * Wh:(s_ + 1) * 32 * Wh].reshape(Wh, 32)
+            for l in (0, 7, 13, 31):
+                assert list(slab[:, l]) == want, (line, s_, l)
         n += 1
     assert n >= 5
 
