@@ -83,47 +83,10 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 constexpr float kMagic = 8388608.0f;
 constexpr uint32_t kMagicBits = 0x4B000000u;
 
-// The code u (< 2^22) of a float built as 0x4B000000 | u, minus the offset z:
-// exact in fp32.
-__device__ __forceinline__ float code_to_float(uint32_t u, float magic_plus_z)
-{
-    return __fsub_rn(__uint_as_float(kMagicBits | u), magic_plus_z);
-}
-
 // ---------------------------------------------------------------------------
-// packed stream codec: a column-group stream is a little-endian sequence of
-// fields; the fixed-width form keeps the stream words in registers.
+// packed stream codec for row-wise widths: a stream is a little-endian sequence
+// of fields (the fixed-width forms live with the kernels).
 // ---------------------------------------------------------------------------
-
-// Field number c (width B) of a stream held in words w[].
-template <int B>
-__device__ __forceinline__ uint32_t field_at(const uint32_t *w, int c)
-{
-    const int pos = c * B, lo = pos >> 5, sh = pos & 31;
-    constexpr uint32_t mask = (1u << B) - 1u;
-    if (sh + B <= 32) return (w[lo] >> sh) & mask;
-    return __funnelshift_r(w[lo], w[lo + 1], sh) & mask;
-}
-
-// OR field value u (< 2^B) into position c of words w[].
-template <int B>
-__device__ __forceinline__ void field_put(uint32_t *w, int c, uint32_t u)
-{
-    const int pos = c * B, lo = pos >> 5, sh = pos & 31;
-    w[lo] |= u << sh;
-    if (sh + B > 32) w[lo + 1] |= u >> (32 - sh);
-}
-
-// OR the low B bits of `bits` into position c of words w[] (the masking and
-// the merge are one logic operation per word touched).
-template <int B>
-__device__ __forceinline__ void field_put_bits(uint32_t *w, int c, uint32_t bits)
-{
-    const int pos = c * B, lo = pos >> 5, sh = pos & 31;
-    constexpr uint32_t mask = (1u << B) - 1u;
-    w[lo] |= (bits << sh) & (mask << sh);
-    if (sh + B > 32) w[lo + 1] |= (bits & mask) >> (32 - sh);
-}
 
 // Variable-width reader over stream words fetched on demand from shared memory
 // (word m of the stream at base[m * stride]).

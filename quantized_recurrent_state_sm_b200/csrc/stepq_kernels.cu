@@ -132,6 +132,55 @@ using X2 = float2[kRowsPerGroup][2];  // the thread's 16 x 4 block as float2 pai
 __device__ __forceinline__ int rowp_chunk(int rg, int q) { return 16 * rg + 4 * (q ^ ((rg >> 1) & 3)); }
 
 // ---------------------------------------------------------------------------
+// Field extraction without shifting: a b-bit field at bit sh of a word, kept in
+// place and given the exponent 150 - sh, is the float 2^(23 - sh) + u exactly
+// (its mantissa bits sh .. sh+b-1 weigh 1 .. 2^(b-1)); subtracting 2^(23 - sh)
+// + z leaves the code.  Fields that end above bit 23 are taken from the word's
+// upper half (shifted down by 16 once per word); fields that straddle two
+// words are funnel-shifted to bit 0.
+// ---------------------------------------------------------------------------
+template <int B>
+__device__ __forceinline__ constexpr int field_mode(int pos)
+{
+    return ((pos & 31) + B <= 23) ? 0 : (((pos & 31) + B <= 32) ? 1 : 2);
+}
+
+template <int B>
+__device__ __forceinline__ void field_raw(const uint32_t *wd, const uint32_t *hw, int pos, int mode, uint32_t &bits,
+                                          float &sub)
+{
+    constexpr uint32_t mask = (1u << B) - 1u;
+    const int lo = pos >> 5, sh = pos & 31;
+    const float z = (float)(1 << (B - 1));
+    if (mode == 0) {
+        bits = (wd[lo] & (mask << sh)) | ((150u - (uint32_t)sh) << 23);
+        sub = (float)(1 << (23 - sh)) + z;
+    } else if (mode == 1) {
+        bits = (hw[lo] & (mask << (sh - 16))) | ((150u - (uint32_t)(sh - 16)) << 23);
+        sub = (float)(1 << (23 - (sh - 16))) + z;
+    } else {
+        bits = (__funnelshift_r(wd[lo], wd[lo + 1], sh) & mask) | (150u << 23);
+        sub = kMagic + z;
+    }
+}
+
+// Fields c and c+1 as a float2 of codes.
+template <int B>
+__device__ __forceinline__ float2 decode_pair(const uint32_t *wd, const uint32_t *hw, int c)
+{
+    const int p0 = c * B, p1 = p0 + B;
+    int m0 = field_mode<B>(p0);
+    const int m1 = field_mode<B>(p1);
+    // a field that fits either way joins its partner in the upper half
+    if (m0 == 0 && m1 == 1 && (p0 >> 5) == (p1 >> 5) && (p0 & 31) >= 16) m0 = 1;
+    uint32_t b0, b1;
+    float s0, s1;
+    field_raw<B>(wd, hw, p0, m0, b0, s0);
+    field_raw<B>(wd, hw, p1, m1, b1, s1);
+    return __fadd2_rn(f2(__uint_as_float(b0), __uint_as_float(b1)), f2(-s0, -s1));
+}
+
+// ---------------------------------------------------------------------------
 // Decode the thread's stream (word m at words[32 m]) into X: code values as
 // floats; pivot rows their binary16 values.  Fixed width B > 0 keeps the
 // stream in registers; B == 0 reads the row widths from rb_lane[8 rr].
@@ -140,19 +189,16 @@ template <int B>
 __device__ __forceinline__ void decode_stream(const int *rb_lane, const uint32_t *words, X2 &X)
 {
     if constexpr (B > 0) {
-        uint32_t wd[2 * B];
+        uint32_t wd[2 * B + 1], hw[2 * B];
 #pragma unroll
         for (int m = 0; m < 2 * B; m++) wd[m] = words[m * kStreams];
-        const float mz = -(kMagic + (float)(1 << (B - 1)));
-        const float2 mz2 = f2(mz, mz);
+        wd[2 * B] = 0u;
+#pragma unroll
+        for (int m = 0; m < 2 * B; m++) hw[m] = wd[m] >> 16;
 #pragma unroll
         for (int rr = 0; rr < kRowsPerGroup; rr++)
 #pragma unroll
-            for (int hh = 0; hh < 2; hh++) {
-                const uint32_t u0 = field_at<B>(wd, 4 * rr + 2 * hh) | kMagicBits;
-                const uint32_t u1 = field_at<B>(wd, 4 * rr + 2 * hh + 1) | kMagicBits;
-                X[rr][hh] = __fadd2_rn(f2(__uint_as_float(u0), __uint_as_float(u1)), mz2);
-            }
+            for (int hh = 0; hh < 2; hh++) X[rr][hh] = decode_pair<B>(wd, hw, 4 * rr + 2 * hh);
     } else {
         BitReader br;
         br.init(words, kStreams);
@@ -257,6 +303,21 @@ __device__ __forceinline__ void ls_round(ItemSmem &sm, const RowFactors &rf, con
 // Final codes of a fixed-width stream and their store: u = z + clip(rne(p / c))
 // taken from the low mantissa bits of p / c + 2^23 + z; each 32-bit word is
 // stored as soon as its last code is placed.
+// Word m of a fixed-width stream is the sum over its fields of y << sh, y =
+// 0x4B000000 | u the float bits of 2^23 + u (fields that straddle into the next
+// word enter as u alone), minus the words' share of 0x4B000000 << sh, a
+// constant: the sum has no carries between fields.
+template <int B>
+__device__ __forceinline__ constexpr uint32_t magic_share(int m)
+{
+    uint32_t acc = 0u;
+    for (int c = 0; c < 64; c++) {
+        const int pos = c * B;
+        if ((pos >> 5) == m && (pos & 31) + B <= 32) acc += kMagicBits << (pos & 31);
+    }
+    return acc;
+}
+
 template <int B, bool CLIP>
 __device__ __forceinline__ void pack_fixed(const X2 &X, float2 ic0, float2 ic1, uint32_t *words)
 {
@@ -265,7 +326,7 @@ __device__ __forceinline__ void pack_fixed(const X2 &X, float2 ic0, float2 ic1, 
     const float2 mz2 = f2(mz, mz);
     uint32_t ow[2 * B + 1];
 #pragma unroll
-    for (int m = 0; m <= 2 * B; m++) ow[m] = 0u;
+    for (int m = 0; m <= 2 * B; m++) ow[m] = 0u - magic_share<B>(m);
 #pragma unroll
     for (int rr = 0; rr < kRowsPerGroup; rr++)
 #pragma unroll
@@ -281,7 +342,15 @@ __device__ __forceinline__ void pack_fixed(const X2 &X, float2 ic0, float2 ic1, 
 #pragma unroll
             for (int e = 0; e < 2; e++) {
                 const int c = 4 * rr + 2 * hh + e;
-                field_put_bits<B>(ow, c, __float_as_uint(e ? mm.y : mm.x));
+                const uint32_t y = __float_as_uint(e ? mm.y : mm.x);
+                const int pos = c * B, lo = pos >> 5, sh = pos & 31;
+                if (sh + B <= 32) {
+                    ow[lo] += y << sh;
+                } else {
+                    const uint32_t u = y & ((1u << B) - 1u);
+                    ow[lo] += u << sh;
+                    ow[lo + 1] += u >> (32 - sh);
+                }
 #pragma unroll
                 for (int m = (c * B) / 32; m < ((c + 1) * B) / 32; m++) words[m * kStreams] = ow[m];
             }
