@@ -120,7 +120,8 @@ struct alignas(16) ItemSmem {
     // chunks swizzled by row group (rowp_chunk)
     float rowp[8 * 4 * kDK];
     uint64_t bar[kMaxSlots];
-    int4 prod_rec;          // producer: staging record of position prod_n
+    int4 recs[2][32];       // producer: staging records, 32 stagings per chunk
+    int prod_first;         // producer: the CTA's first staged position
     int prod_n;             // producer: next position to stage
     uint32_t prod_issued;   // producer: items staged so far
 };
@@ -675,35 +676,41 @@ constexpr uint32_t kStageArrivals = 1 + 32;
 
 // Producer state, used by the producer warp only and kept in shared memory so
 // that it costs no registers elsewhere: the next position to stage, the number
-// staged so far, and that position's staging record, fetched one issue ahead
-// by an asynchronous copy (lane 0) so that no global load stalls the warp.
-__device__ __forceinline__ void prefetch_stage_rec(ItemSmem &sm, const StepArgs &a)
+// staged so far, and the staging records of the CTA's positions, fetched 32 at
+// a time (one 16-byte asynchronous copy per lane) a chunk ahead of use.
+// Staging number k stages position n_first + k G and reads recs[k/32 % 2][k%32].
+__device__ __forceinline__ void fetch_rec_chunk(ItemSmem &sm, const StepArgs &a, uint32_t chunk)
 {
-    if ((threadIdx.x & 31) == 0) {
-        if (sm.prod_n < a.n_items)
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_addr(&sm.prod_rec)),
-                         "l"(a.t.stage + sm.prod_n)
-                         : "memory");
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    }
+    const int lane = threadIdx.x & 31;
+    const long long n = (long long)sm.prod_first + (long long)(32 * chunk + lane) * gridDim.x;
+    if (n < a.n_items)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(&sm.recs[chunk & 1][lane])),
+                     "l"(a.t.stage + n)
+                     : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
 // Stage the next position into slot buffer sb (the whole producer warp; the
-// caller checks sm.prod_n < n_items, a warp-uniform condition).
+// caller checks sm.prod_n < n_items, a warp-uniform condition).  At the start
+// of every chunk of 32 stagings the warp waits for that chunk's records and
+// fetches the next chunk's.
 template <bool KDA>
 __device__ __forceinline__ void produce(ItemSmem &sm, const StepArgs &a, uint8_t *sb, uint64_t *bar)
 {
-    if ((threadIdx.x & 31) == 0) asm volatile("cp.async.wait_all;" ::: "memory");
-    __syncwarp();
-    const int4 st = sm.prod_rec;
+    const uint32_t k = sm.prod_issued;
+    if ((k & 31u) == 0) {
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncwarp();
+        fetch_rec_chunk(sm, a, (k >> 5) + 1);
+    }
+    const int4 st = sm.recs[(k >> 5) & 1][k & 31];
     __syncwarp();
     stage_item<KDA>(a, st, sb, bar);
     if ((threadIdx.x & 31) == 0) {
         sm.prod_n += gridDim.x;
-        sm.prod_issued++;
+        sm.prod_issued = k + 1;
     }
     __syncwarp();
-    prefetch_stage_rec(sm, a);
 }
 
 // Phase 0 of a staged item (threads 128..255, row i = tid - 128): per-row
@@ -906,11 +913,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
     if (n_first < npiv) n_first += ((npiv - n_first + G - 1) / G) * G;
     if ((tid >> 5) == kProducerWarp) {
         if ((tid & 31) == 0) {
+            sm.prod_first = n_first;
             sm.prod_n = n_first;
             sm.prod_issued = 0;
         }
         __syncwarp();
-        prefetch_stage_rec(sm, a);
+        fetch_rec_chunk(sm, a, 0);
         for (int s = 0; s < a.nslots && sm.prod_n < a.n_items; s++)
             produce<KDA>(sm, a, ring + s * a.slot_bytes, &sm.bar[s]);
     }
