@@ -188,6 +188,42 @@ STEPQ_API stepq_status stepq_fp32_step(const stepq_desc *desc, float *S, const f
  */
 STEPQ_API stepq_status stepq_pool_check(stepq_pool *pool);
 
+/*
+ * The fused decode step of stepq_decode_step without a pool, allocating
+ * nothing.  The pages describe no counterpart: it is a deployment variant of
+ * the same kernel and computes exactly what stepq_decode_step computes.
+ *
+ * For callers that keep the packed states in memory they manage themselves
+ * and may not allocate at decode time -- e.g. a serving runtime that gives all
+ * free HBM to its own caching allocator, where a cudaMalloc would fail or
+ * synchronise the device.  The kernel's scratch tables (per-head records, item
+ * order, staging records, status word) live in a fixed file-scope device
+ * array of 256 KiB inside the library instead of a pool buffer's tail; every
+ * call rebuilds them on the host and uploads them on the stream before its
+ * launch.  No device or host memory is allocated on the success path (an
+ * error message may be formatted into the library's per-thread error string).
+ *
+ * desc: as for stepq_pool_create, with heads <= 64 and tables that fit the
+ * scratch (about 10 000 items at 32 heads, 7 500 at 64); larger descriptors
+ * return STEPQ_ERR_UNSUPPORTED with the sizes in stepq_last_error().
+ * states: device, state_bytes >= stepq_state_bytes(desc), 16-byte aligned,
+ * laid out as a pool's packed states (e.g. packed by stepq_pack of a pool
+ * with the same descriptor, then copied); updated in place.  q, k, v, alpha,
+ * beta, out: as for stepq_decode_step.  cuda_stream: cudaStream_t or NULL.
+ *
+ * Calls share the one scratch array per device: two calls in flight at the
+ * same time (on different streams or threads) race on it, so order them on
+ * one stream.  The first call on a device looks up the scratch address
+ * (cudaGetSymbolAddress) and should come before any stream capture.  The
+ * status word the kernel writes when a staged copy never lands is cleared by
+ * the next call and not reported here; use a pool and stepq_pool_check where
+ * that report is needed.
+ */
+STEPQ_API stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *states, size_t state_bytes,
+                                                 const float *q, const float *k, const float *v,
+                                                 const float *alpha, const float *beta, float *out,
+                                                 void *cuda_stream);
+
 /* Human-readable name of a status; never NULL. */
 STEPQ_API const char *stepq_status_string(stepq_status s);
 

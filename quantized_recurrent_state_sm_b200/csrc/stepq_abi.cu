@@ -183,6 +183,35 @@ stepq::StepArgs base_args(const stepq_pool *p)
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Decode step without a pool, allocating nothing.  The fused decode kernel
+// needs scratch tables next to the packed states: per-head records, the item
+// order, one staging record per item and a status word.  A pool keeps them in
+// the tail of the caller's buffer; this variant keeps them in a fixed
+// file-scope device array instead and builds them on every call into a fixed
+// host image.  It serves callers that hold the packed states in memory they
+// manage themselves and may not allocate at decode time: a serving runtime
+// that gives all free HBM to its own caching allocator (a cudaMalloc there
+// fails or synchronises the device), or one whose state buffer has no room
+// for a pool's table tail.  No cudaMalloc, cudaFree, host heap or other
+// allocating call is made on the success path.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 256 * 1024;  // the largest table image this variant accepts
+constexpr int kNoAllocMaxHeads = 64;
+constexpr int kNoAllocMaxDevices = 64;
+
+// Device scratch.  Only its status word must start at zero; every call uploads
+// the whole table image, status word (zero) included, before its launch.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;                             // guards the two arrays below
+unsigned char g_noalloc_host[kNoAllocScratchBytes];  // host image of the scratch
+void *g_noalloc_dev[kNoAllocMaxDevices];             // scratch address per device (first call)
+
+}  // namespace
+
 extern "C" {
 
 size_t stepq_pool_bytes(const stepq_desc *desc)
@@ -466,5 +495,185 @@ const char *stepq_status_string(stepq_status s)
 }
 
 const char *stepq_last_error(void) { return g_err.c_str(); }
+
+stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *states, size_t state_bytes, const float *q,
+                                       const float *k, const float *v, const float *alpha, const float *beta,
+                                       float *out, void *cuda_stream)
+{
+    stepq_status st = check_desc(desc, true, nullptr);
+    if (st != STEPQ_OK) return st;
+    const int H = desc->heads, B = desc->batch;
+    if (H > kNoAllocMaxHeads)
+        return fail(STEPQ_ERR_UNSUPPORTED, "stepq_decode_step_noalloc takes at most %d heads (got %d)",
+                    kNoAllocMaxHeads, H);
+    const size_t n = (size_t)B * H;
+    // per-head item layout, as in a pool
+    long long item_bytes[kNoAllocMaxHeads], head_off[kNoAllocMaxHeads];
+    int slab_words[kNoAllocMaxHeads], kind[kNoAllocMaxHeads];
+    long long req = 0, max_staged = 0;
+    int n_pivot_items = 0;
+    for (int h = 0; h < H; h++) {
+        int W = 0, npiv = 0;
+        for (int g = 0; g < stepq::kRowGroups; g++) {
+            int bitsum = 0;
+            for (int rr = 0; rr < stepq::kRowsPerGroup; rr++)
+                bitsum += desc->bits[h * kDK + g * stepq::kRowsPerGroup + rr];
+            W = std::max(W, (4 * bitsum + 31) / 32);
+        }
+        for (int i = 0; i < kDK; i++) npiv += desc->bits[h * kDK + i] == STEPQ_PIVOT_BITS;
+        slab_words[h] = W;
+        item_bytes[h] = stepq::kHeaderBytes + 4LL * W * stepq::kStreams * stepq::kSlabs;
+        kind[h] = npiv == 0 ? stepq::kHeadQuant : (npiv == kDK ? stepq::kHeadAllPivot : stepq::kHeadMixed);
+        head_off[h] = req;
+        req += item_bytes[h];
+        if (kind[h] == stepq::kHeadAllPivot)
+            n_pivot_items += B;
+        else
+            max_staged = std::max(max_staged, item_bytes[h]);
+    }
+    // scratch image layout
+    size_t o = 0;
+    const size_t off_rec = o;        o = align_up(o + sizeof(stepq::HeadRec) * (size_t)H, 256);
+    const size_t off_head_off = o;   o = align_up(o + 8 * (size_t)H, 16);
+    const size_t off_head_bytes = o; o = align_up(o + 4 * (size_t)H, 16);
+    const size_t off_status = o;     o = align_up(o + 16, 16);
+    const size_t off_order = o;      o = align_up(o + 4 * n, 16);
+    const size_t off_stage = o;      o = align_up(o + 16 * n, 16);
+    if (o > kNoAllocScratchBytes)
+        return fail(STEPQ_ERR_UNSUPPORTED,
+                    "stepq_decode_step_noalloc: the tables of %d requests x %d heads take %zu bytes, more than "
+                    "its fixed %zu-byte scratch; use a pool", B, H, o, kNoAllocScratchBytes);
+    if (state_bytes < (size_t)req * (size_t)B)
+        return fail(STEPQ_ERR_INVALID_ARG, "states holds %zu bytes < %zu required", state_bytes,
+                    (size_t)req * (size_t)B);
+    if (n == 0) return STEPQ_OK;
+    if ((st = check_dev(states, "states", 16)) != STEPQ_OK) return st;
+    if ((st = check_step_tensors(desc->variant, n, q, k, v, alpha, beta, out)) != STEPQ_OK) return st;
+    if (overlaps(out, n * kDV * 4, states, (size_t)req * (size_t)B))
+        return fail(STEPQ_ERR_INVALID_ARG, "out overlaps the packed states");
+    // staging slot geometry, as in a pool
+    const int kda = desc->variant == STEPQ_KDA;
+    int off = (int)align_up((size_t)max_staged, 16);
+    const int off_q = off; off += 4 * kDK;
+    const int off_k = off; off += 4 * kDK;
+    const int off_v = off; off += 4 * kDV;
+    const int off_alpha = off; off += kda ? 4 * kDK : 0;
+    const int off_ab = off; off += 16;
+    const int off_rec_slot = off; off += (int)sizeof(stepq::HeadRec);
+    const int slot_bytes = (int)align_up((size_t)off, 128);
+    int nslots = 0;
+    for (int ns = stepq::kMaxSlots; ns >= 2 && nslots == 0; ns--)
+        if (stepq::decode_ctas_per_sm(ns, slot_bytes) >= 2) nslots = ns;
+    for (int ns = stepq::kMaxSlots; ns >= 2 && nslots == 0; ns--)
+        if (stepq::decode_ctas_per_sm(ns, slot_bytes) >= 1) nslots = ns;
+    if (nslots == 0 && max_staged > 0) return fail(STEPQ_ERR_CUDA, "no staging ring fits in shared memory");
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "stepq_decode_step_noalloc: current device");
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return fail(STEPQ_ERR_UNSUPPORTED, "stepq_decode_step_noalloc supports device ordinals below %d",
+                    kNoAllocMaxDevices);
+    std::lock_guard<std::mutex> guard(g_noalloc_mu);
+    if (!g_noalloc_dev[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "stepq_decode_step_noalloc: scratch address");
+        g_noalloc_dev[dev] = p;
+    }
+    uint8_t *img = g_noalloc_host;
+    std::memset(img, 0, o);
+    stepq::HeadRec *rec = reinterpret_cast<stepq::HeadRec *>(img + off_rec);
+    long long *t_head_off = reinterpret_cast<long long *>(img + off_head_off);
+    int *t_head_bytes = reinterpret_cast<int *>(img + off_head_bytes);
+    int *order = reinterpret_cast<int *>(img + off_order);
+    int *stage = reinterpret_cast<int *>(img + off_stage);
+    for (int h = 0; h < H; h++) {
+        stepq::HeadRec &R = rec[h];
+        int b0 = desc->bits[h * kDK], same = 1;
+        for (int i = 0; i < kDK; i++) {
+            const int b = desc->bits[h * kDK + i];
+            R.bits[i] = (uint8_t)b;
+            same &= (b == b0);
+            if (b != STEPQ_PIVOT_BITS) {
+                R.s[i] = (float)(1.0 / std::sqrt((double)desc->rho[h * kDK + i]));
+                R.rho[i] = desc->rho[h * kDK + i];
+                R.rq[i] = (float)(1.0 / (double)((1 << (b - 1)) - 1));
+            }
+        }
+        R.head_off = head_off[h];
+        R.head_b = (same && b0 != STEPQ_PIVOT_BITS) ? b0 : 0;
+        R.head_kind = kind[h];
+        R.head_bytes = (int)item_bytes[h];
+        R.slab_words = slab_words[h];
+        t_head_off[h] = head_off[h];
+        t_head_bytes[h] = (int)item_bytes[h];
+    }
+    // item order: all-pivot heads' items first, then the others, heaviest
+    // heads first; items of equal weight in item order
+    int hs[kNoAllocMaxHeads];
+    for (int h = 0; h < H; h++) hs[h] = h;
+    for (int x = 1; x < H; x++) {  // stable insertion sort of the heads
+        const int hx = hs[x];
+        int y = x;
+        for (; y > 0; y--) {
+            const int hy = hs[y - 1];
+            const int px = kind[hx] == stepq::kHeadAllPivot, py = kind[hy] == stepq::kHeadAllPivot;
+            const bool before = (px != py) ? (px > py) : (item_bytes[hx] > item_bytes[hy]);
+            if (!before) break;
+            hs[y] = hy;
+        }
+        hs[y] = hx;
+    }
+    size_t pos = 0;
+    for (int c0 = 0; c0 < H;) {
+        int c1 = c0 + 1;  // heads hs[c0 .. c1) share one key
+        while (c1 < H && (kind[hs[c1]] == stepq::kHeadAllPivot) == (kind[hs[c0]] == stepq::kHeadAllPivot) &&
+               item_bytes[hs[c1]] == item_bytes[hs[c0]])
+            c1++;
+        int lo = c0, hi = c1;  // within the class, item order: request-major, then head
+        for (int x = lo + 1; x < hi; x++)
+            for (int y = x; y > lo && hs[y] < hs[y - 1]; y--) std::swap(hs[y], hs[y - 1]);
+        for (int b = 0; b < B; b++)
+            for (int c = lo; c < hi; c++) {
+                const int h = hs[c], item = b * H + h;
+                const unsigned long long offb = (unsigned long long)b * (unsigned long long)req +
+                                                (unsigned long long)head_off[h];
+                order[pos] = item;
+                stage[4 * pos + 0] = item;
+                stage[4 * pos + 1] = (int)item_bytes[h];
+                stage[4 * pos + 2] = (int)(uint32_t)(offb & 0xFFFFFFFFull);
+                stage[4 * pos + 3] = (int)(uint32_t)(offb >> 32);
+                pos++;
+            }
+        c0 = c1;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(cuda_stream);
+    uint8_t *dsc = static_cast<uint8_t *>(g_noalloc_dev[dev]);
+    e = cudaMemcpyAsync(dsc, img, o, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "stepq_decode_step_noalloc: table upload");
+    stepq::StepArgs a{};
+    a.pool = static_cast<uint8_t *>(states);
+    a.t.rowrec = reinterpret_cast<const stepq::HeadRec *>(dsc + off_rec);
+    a.t.head_off = reinterpret_cast<const long long *>(dsc + off_head_off);
+    a.t.head_bytes = reinterpret_cast<const int *>(dsc + off_head_bytes);
+    a.t.order = reinterpret_cast<const int *>(dsc + off_order);
+    a.t.stage = reinterpret_cast<const int4 *>(dsc + off_stage);
+    a.t.status = reinterpret_cast<int *>(dsc + off_status);
+    a.req_bytes = req;
+    a.heads = H;
+    a.n_items = (int)n;
+    a.ls_iters = desc->ls_iters;
+    a.kda = kda;
+    a.nslots = nslots;
+    a.slot_bytes = slot_bytes;
+    a.off_q = off_q; a.off_k = off_k; a.off_v = off_v;
+    a.off_alpha = off_alpha; a.off_ab = off_ab; a.off_rec = off_rec_slot;
+    a.n_pivot_items = n_pivot_items;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.out = out;
+    e = stepq::launch_decode_step(a, s);
+    return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "stepq_decode_step_noalloc launch");
+}
+
 
 }  // extern "C"

@@ -37,7 +37,8 @@ class Desc(C.Structure):
 
 EXPORTS = ("stepq_pool_bytes", "stepq_state_bytes", "stepq_pool_create", "stepq_pool_destroy",
            "stepq_pool_set_stream", "stepq_pack", "stepq_unpack", "stepq_decode_step",
-           "stepq_fp32_step", "stepq_pool_check", "stepq_status_string", "stepq_last_error")
+           "stepq_fp32_step", "stepq_pool_check", "stepq_status_string", "stepq_last_error",
+           "stepq_decode_step_noalloc")
 
 
 def _load():
@@ -56,8 +57,9 @@ def _load():
     L.stepq_unpack.argtypes = [P, P]
     L.stepq_decode_step.argtypes = [P, P, P, P, P, P, P]
     L.stepq_fp32_step.argtypes = [D, P, P, P, P, P, P, P, P]
+    L.stepq_decode_step_noalloc.argtypes = [D, P, C.c_size_t, P, P, P, P, P, P, P]
     for fn in ("stepq_pool_create", "stepq_pool_destroy", "stepq_pool_set_stream", "stepq_pool_check", "stepq_pack",
-               "stepq_unpack", "stepq_decode_step", "stepq_fp32_step"):
+               "stepq_unpack", "stepq_decode_step", "stepq_fp32_step", "stepq_decode_step_noalloc"):
         getattr(L, fn).restype = C.c_int
     L.stepq_status_string.argtypes = [C.c_int]; L.stepq_status_string.restype = C.c_char_p
     L.stepq_last_error.argtypes = []; L.stepq_last_error.restype = C.c_char_p
@@ -192,4 +194,29 @@ def fp32_step(variant: int, S: torch.Tensor, q, k, v, alpha, beta, out=None) -> 
                                _dev(k, "k", (B, H, DK)), _dev(v, "v", (B, H, DV)),
                                _dev(alpha, "alpha", ash), _dev(beta, "beta", (B, H)),
                                _dev(out, "out", (B, H, DV)), _stream_ptr()))
+    return out
+
+
+def decode_step_noalloc(variant: int, bits, rho, states: torch.Tensor, q, k, v, alpha, beta, out=None,
+                        ls_iters: int = 1) -> torch.Tensor:
+    """The fused decode step on packed states held in `states` (a uint8 CUDA
+    tensor laid out as a pool's packed states), without a pool: the library
+    keeps the kernel's tables in its own fixed device scratch and allocates
+    nothing.  Calls must not overlap (one stream); see include/stepq.h."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint8)
+    H = bits.shape[0]
+    B = q.shape[0]
+    d, keep = make_desc(variant, B, H, bits, rho, ls_iters)
+    if not isinstance(states, torch.Tensor) or states.dtype != torch.uint8 or not states.is_cuda:
+        raise TypeError("states must be a uint8 CUDA tensor")
+    if not states.is_contiguous():
+        raise ValueError("states must be contiguous")
+    if out is None:
+        out = torch.empty((B, H, DV), dtype=torch.float32, device=states.device)
+    ash = (B, H, DK) if variant == KDA else (B, H)
+    _check(lib.stepq_decode_step_noalloc(C.byref(d), C.c_void_p(states.data_ptr()), states.numel(),
+                                         _dev(q, "q", (B, H, DK)), _dev(k, "k", (B, H, DK)),
+                                         _dev(v, "v", (B, H, DV)), _dev(alpha, "alpha", ash),
+                                         _dev(beta, "beta", (B, H)), _dev(out, "out", (B, H, DV)),
+                                         _stream_ptr()))
     return out
