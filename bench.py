@@ -148,6 +148,29 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time: every rank passes its own, all get the maximum
+    (one all-reduce; a no-op on a single rank)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, items_per_rank, steps, ms):
+    """Items all ranks processed per second, timed by the slowest rank."""
+    return world * items_per_rank * steps / (ms * 1e-3)
+
+
+def rank_step_offset(rank):
+    """Step-index offset of a rank's synthetic inputs: each rank serves its own
+    requests (different inputs, same shapes)."""
+    return 1000 * rank
+
+
 def cpu_oracle_rate(cfg, seconds):
     """The CPU oracle as it stands (single thread) on a bounded sample of the
     workload: the parity requests {0, 1, B/2, B-1} x all heads, consecutive
@@ -227,12 +250,8 @@ def run_e2e(args, cfg, pool, host, out, stream, world):
         e2e_step(i)
     g1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = g0.elapsed_time(g1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    value = world * cfg.items * args.e2e_steps / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks(g0.elapsed_time(g1), world, "cuda")
+    value = whole_job_rate(world, cfg.items, args.e2e_steps, e2e_ms)
 
     return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": args.e2e_steps}
@@ -265,7 +284,7 @@ def main():
     # input ring: RING pre-generated steps resident in HBM
     ring = []
     for t in range(RING):
-        x = W.step_inputs(cfg, t + 1000 * rank)
+        x = W.step_inputs(cfg, t + rank_step_offset(rank))
         ring.append({k: torch.from_numpy(v).cuda() for k, v in x.items()})
     out = torch.empty((B, H, cfg.dv), device="cuda")
     stream = torch.cuda.current_stream()
@@ -313,20 +332,16 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
     ms_per_step = ms / args.steps
-    value = world * cfg.items * args.steps / (ms * 1e-3)
+    value = whole_job_rate(world, cfg.items, args.steps, ms)
 
     # end to end through the public API with host buffers: pinned H2D of the
     # step's inputs, the decode step, D2H of the readout, every step
     e2e = None
     host = []
     for t in range(RING if not args.profile else 0):
-        x = W.step_inputs(cfg, t + 1000 * rank)
+        x = W.step_inputs(cfg, t + rank_step_offset(rank))
         host.append({k: torch.from_numpy(v).pin_memory() for k, v in x.items()})
     if not args.profile:
         e2e = run_e2e(args, cfg, pool, host, out, stream, world)
