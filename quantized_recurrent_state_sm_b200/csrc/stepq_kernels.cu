@@ -103,9 +103,9 @@ struct alignas(16) RowFactors {
     float4 k2[64], l2[64], g2[64];  // a k, a q, gamma (see pslot)
     float4 a2[64], q2[64];          // alpha, 1/Q (0 on pivot rows); row-wise widths only
     float4 h2[64], w2[64];          // fit: h = a / r', w = rho r'^2
+    float kqp[4];
     float ra[kDK];                  // a_i = alpha_i r_i (alpha_i on pivot rows), by row
     int rb[kDK];                    // widths, by sslot
-    float kqp[4];                   // k.q over rows 32m .. 32m+31
     float beta;
     int item, head_b;               // the item; its head's common width (0: row-wise)
 };
@@ -361,6 +361,7 @@ __device__ __forceinline__ void pack_fixed(const X2 &X, float2 ic0, float2 ic1, 
 // Nothing to do between the two barriers of the fit (pack kernel).
 struct NoMid {
     __device__ __forceinline__ bool operator()() const { return true; }
+    __device__ __forceinline__ bool rowside(int) const { return true; }
 };
 
 enum FitResult { kFitDone = 0, kFitAbortNow = 1, kFitAbortAfter = 2 };
@@ -373,9 +374,9 @@ enum FitResult { kFitDone = 0, kFitAbortNow = 1, kFitAbortAfter = 2 };
 // item_g (W words per stream).
 //
 // Barrier 1 publishes the row partials of P^2; threads 0..127 then derive row
-// i's scale and fit factors while `mid` runs on threads 128..255 (the fused
-// step prepares the next item there); barrier 2 publishes both, and
-// everything after it is warp-local.  If ok_in is false on any thread the
+// i's scale and fit factors and run mid.rowside(i), while mid() runs on
+// threads 128..255 (the fused step prepares the next item there); barrier 2
+// publishes both, and everything after it is warp-local.  If ok_in is false on any thread the
 // item is abandoned at barrier 1 with nothing stored (kFitAbortNow); if `mid`
 // fails on any thread the item is completed and kFitAbortAfter returned.
 // ---------------------------------------------------------------------------
@@ -430,6 +431,7 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
         put_pair(rf.h2, i, h);
         put_pair(rf.w2, i, wt);
         reinterpret_cast<float *>(item_g)[i] = rnew;
+        ok_mid = mid.rowside(i);
     } else {
         ok_mid = mid();
     }
@@ -745,10 +747,6 @@ __device__ __forceinline__ void phase0(RowFactors &rf, const StepArgs &a, const 
     }
     rf.ra[i] = A;
     if (KDA) rf.rb[sslot(i)] = b;
-    float kq = k * q;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(kFull, kq, o);
-    if ((i & 31) == 0) rf.kqp[i >> 5] = kq;
     if (i == 0) {
         rf.beta = beta;
         rf.item = item;
@@ -756,23 +754,37 @@ __device__ __forceinline__ void phase0(RowFactors &rf, const StepArgs &a, const 
     }
 }
 
-// Work between the fit's two barriers of staged item n, on threads 128..255:
-// phase 0 of the CTA's next staged item into the other factor buffer.
-// Returns false if that item's copy never landed.
+// Work between the fit's two barriers of staged item n for the CTA's next
+// staged item, written to the other factor buffer: phase 0 on threads
+// 128..255 (operator()), its k.q on threads 0..127 after their row factors
+// (rowside).  Both return false if that item's copy never landed.
 template <bool KDA>
 struct StageNext {
     ItemSmem &sm;
     const StepArgs &a;
     uint8_t *ring;
     int next_pos;      // position of the next staged item (>= n_items: none)
-    uint32_t n_next;   // its consumption count
+    int next_slot;     // its slot and the barrier phase parity it completes
+    uint32_t next_parity;
     RowFactors &rf_next;
     __device__ __forceinline__ bool operator()() const
     {
         if (next_pos >= a.n_items) return true;
-        const int s = (int)(n_next % (uint32_t)a.nslots);
-        if (!mbar_wait_bounded(&sm.bar[s], (n_next / (uint32_t)a.nslots) & 1u, kWaitLimit)) return false;
-        phase0<KDA>(rf_next, a, ring + s * a.slot_bytes, a.t.order[next_pos]);
+        if (!mbar_wait_bounded(&sm.bar[next_slot], next_parity, kWaitLimit)) return false;
+        phase0<KDA>(rf_next, a, ring + next_slot * a.slot_bytes, a.t.order[next_pos]);
+        return true;
+    }
+    // on threads 0..127, after their row factors: row i's k.q of the next
+    // item, summed per 32 rows (the readout's scalar)
+    __device__ __forceinline__ bool rowside(int i) const
+    {
+        if (next_pos >= a.n_items) return true;
+        if (!mbar_wait_bounded(&sm.bar[next_slot], next_parity, kWaitLimit)) return false;
+        const uint8_t *sb = ring + next_slot * a.slot_bytes;
+        float kq = reinterpret_cast<const float *>(sb + a.off_k)[i] * reinterpret_cast<const float *>(sb + a.off_q)[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(kFull, kq, o);
+        if ((i & 31) == 0) rf_next.kqp[i >> 5] = kq;
         return true;
     }
 };
@@ -927,25 +939,23 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
 
     // phase 0 of the first staged item
     {
-        bool ok = true;
-        if (tid >= kDK) {
-            ok = mbar_wait_bounded(&sm.bar[0], 0u, kWaitLimit);
-            if (ok) phase0<KDA>(sm.u.rf[0], a, ring, a.t.order[n_first]);
-        }
+        const StageNext<KDA> first{sm, a, ring, n_first, 0, 0u, sm.u.rf[0]};
+        const bool ok = (tid >= kDK) ? first() : first.rowside(tid);
         if (!__syncthreads_and(ok)) {
             abort_drain(sm, a, 0u, kStatusWaitTimeout);
             return;
         }
     }
-    uint32_t n_cons = 0;
-    int par = 0;
+    uint32_t n_cons = 0;  // consumption count of the item; its slot and barrier parity below
+    int par = 0, slot = 0;
+    uint32_t parity = 0;
     for (int n = n_first; n < a.n_items; n += G, par ^= 1) {
         RowFactors &rf = sm.u.rf[par];
-        const int slot = (int)(n_cons % (uint32_t)a.nslots);
-        const uint32_t parity = (n_cons / (uint32_t)a.nslots) & 1u;
         const uint8_t *sb = ring + slot * a.slot_bytes;
         const bool ok = mbar_wait_bounded(&sm.bar[slot], parity, kWaitLimit);
-        const StageNext<KDA> next{sm, a, ring, n + G, n_cons + 1, sm.u.rf[par ^ 1]};
+        const int slot_next = (slot + 1 == a.nslots) ? 0 : slot + 1;
+        const uint32_t parity_next = (slot_next == 0) ? (parity ^ 1u) : parity;
+        const StageNext<KDA> next{sm, a, ring, n + G, slot_next, parity_next, sm.u.rf[par ^ 1]};
         FitResult res = kFitDone;
         if (KDA) {
             res = run_item<0, KDA, MULTI>(sm, a, rf, sb, ok, next);
@@ -976,6 +986,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
         if ((tid >> 5) == kProducerWarp && sm.prod_n < a.n_items)
             produce<KDA>(sm, a, ring + slot * a.slot_bytes, &sm.bar[slot]);
         n_cons++;
+        slot = slot_next;
+        parity = parity_next;
     }
 }
 
