@@ -71,6 +71,7 @@ stepq_status check_desc(const stepq_desc *d, bool need_tables, Layout *L)
         return fail(STEPQ_ERR_INVALID_ARG, "variant %d is neither STEPQ_GDN nor STEPQ_KDA", d->variant);
     if (d->batch < 0) return fail(STEPQ_ERR_INVALID_ARG, "batch %d < 0", d->batch);
     if (d->heads < 1) return fail(STEPQ_ERR_INVALID_ARG, "heads %d < 1", d->heads);
+    if (d->heads > 65535) return fail(STEPQ_ERR_UNSUPPORTED, "heads %d > 65535", d->heads);
     if (d->dk < 1 || d->dv < 1) return fail(STEPQ_ERR_INVALID_ARG, "dk, dv must be positive");
     if (d->dk != kDK || d->dv != kDV)
         return fail(STEPQ_ERR_UNSUPPORTED, "only dk = dv = 128 is implemented (got %d x %d)", d->dk, d->dv);
@@ -294,7 +295,7 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
         const unsigned long long off = (unsigned long long)(item / H) * (unsigned long long)L.req_bytes +
                                        (unsigned long long)head_off[h];
         stage[4 * n + 0] = item;
-        stage[4 * n + 1] = (int)L.item_bytes[h];
+        stage[4 * n + 1] = (int)L.item_bytes[h] | (h << 16);
         stage[4 * n + 2] = (int)(uint32_t)(off & 0xFFFFFFFFull);
         stage[4 * n + 3] = (int)(uint32_t)(off >> 32);
     }
@@ -641,7 +642,7 @@ stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *states, siz
                                                 (unsigned long long)head_off[h];
                 order[pos] = item;
                 stage[4 * pos + 0] = item;
-                stage[4 * pos + 1] = (int)item_bytes[h];
+                stage[4 * pos + 1] = (int)item_bytes[h] | (h << 16);
                 stage[4 * pos + 2] = (int)(uint32_t)(offb & 0xFFFFFFFFull);
                 stage[4 * pos + 3] = (int)(uint32_t)(offb >> 32);
                 pos++;

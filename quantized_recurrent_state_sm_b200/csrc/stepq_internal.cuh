@@ -47,7 +47,7 @@ struct Tables {
     const long long *head_off;  // [H] byte offset of head h's item inside a request
     const int *head_bytes;      // [H] bytes of an item of head h
     const int *order;           // [B*H] item processing order: all-pivot heads' items first
-    const int4 *stage;          // [B*H] per position: {item, item bytes, pool offset lo, hi}
+    const int4 *stage;          // [B*H] per position: {item, item bytes | head << 16, pool offset lo, hi}
     int *status;                // device status word: 0 ok, else an error code
 };
 

@@ -121,9 +121,6 @@ struct alignas(16) ItemSmem {
     float rowp[8 * 4 * kDK];
     uint64_t bar[kMaxSlots];
     int4 recs[2][32];       // producer: staging records, 32 stagings per chunk
-    int prod_first;         // producer: the CTA's first staged position
-    int prod_n;             // producer: next position to stage
-    uint32_t prod_issued;   // producer: items staged so far
 };
 
 using X2 = float2[kRowsPerGroup][2];  // the thread's 16 x 4 block as float2 pairs
@@ -496,6 +493,8 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
                 ls_round<B, ROWWISE, true>(sm, rf, X);
         }
     }
+    // the column scales are final: store them before the codes
+    if (l < 16) reinterpret_cast<float *>(item_g)[kDK + 16 * w + l] = store_c ? sm.cnew[16 * w + l] : 0.f;
     // ---- requantise, pack, store -------------------------------------------
     const float4 i4 = ld4(&sm.ci[col0]);
     const float2 ic0 = f2(i4.x, i4.y), ic1 = f2(i4.z, i4.w);
@@ -552,7 +551,6 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
         bw.flush();
         for (int m = bw.next; m < W; m++) words[m * kStreams] = 0u;  // the stream's padding words
     }
-    if (l < 16) reinterpret_cast<float *>(item_g)[kDK + 16 * w + l] = store_c ? sm.cnew[16 * w + l] : 0.f;
     return abort_after ? kFitAbortAfter : kFitDone;
 }
 
@@ -645,10 +643,10 @@ template <bool KDA>
 __device__ __forceinline__ void stage_item(const StepArgs &a, int4 st, uint8_t *sb, uint64_t *bar)
 {
     const int lane = threadIdx.x & 31;
-    const int item = st.x, h = item % a.heads;
+    const int item = st.x, h = (int)((uint32_t)st.y >> 16);
     const long long vec = (long long)item * kDK;
     if (lane == 0) {
-        const uint32_t bytes = (uint32_t)st.y;
+        const uint32_t bytes = (uint32_t)st.y & 0xFFFFu;
         const uint8_t *src = a.pool + (long long)(((unsigned long long)(uint32_t)st.w << 32) | (uint32_t)st.z);
         mbar_arrive_expect_tx(bar, bytes + (uint32_t)sizeof(HeadRec));
         bulk_g2s(sb, src, bytes, bar);
@@ -676,15 +674,13 @@ __device__ __forceinline__ void stage_item(const StepArgs &a, int4 st, uint8_t *
 // lanes' asynchronous-copy arrivals.
 constexpr uint32_t kStageArrivals = 1 + 32;
 
-// Producer state, used by the producer warp only and kept in shared memory so
-// that it costs no registers elsewhere: the next position to stage, the number
-// staged so far, and the staging records of the CTA's positions, fetched 32 at
-// a time (one 16-byte asynchronous copy per lane) a chunk ahead of use.
-// Staging number k stages position n_first + k G and reads recs[k/32 % 2][k%32].
-__device__ __forceinline__ void fetch_rec_chunk(ItemSmem &sm, const StepArgs &a, uint32_t chunk)
+// Staging records: staging number k of the CTA stages position n_first + k G
+// (if it exists) from recs[k / 32 % 2][k % 32].  The producer warp fetches
+// them 32 at a time (one 16-byte async copy per lane) a chunk ahead of use.
+__device__ __forceinline__ void fetch_rec_chunk(ItemSmem &sm, const StepArgs &a, int n_first, uint32_t chunk)
 {
     const int lane = threadIdx.x & 31;
-    const long long n = (long long)sm.prod_first + (long long)(32 * chunk + lane) * gridDim.x;
+    const long long n = (long long)n_first + (long long)(32 * chunk + lane) * gridDim.x;
     if (n < a.n_items)
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(&sm.recs[chunk & 1][lane])),
                      "l"(a.t.stage + n)
@@ -692,27 +688,20 @@ __device__ __forceinline__ void fetch_rec_chunk(ItemSmem &sm, const StepArgs &a,
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-// Stage the next position into slot buffer sb (the whole producer warp; the
-// caller checks sm.prod_n < n_items, a warp-uniform condition).  At the start
-// of every chunk of 32 stagings the warp waits for that chunk's records and
-// fetches the next chunk's.
+// Issue staging k into slot buffer sb (the whole producer warp; the caller
+// checks that the position exists).  At the start of every chunk of 32
+// stagings the warp waits for that chunk's records and fetches the next
+// chunk's.
 template <bool KDA>
-__device__ __forceinline__ void produce(ItemSmem &sm, const StepArgs &a, uint8_t *sb, uint64_t *bar)
+__device__ __forceinline__ void produce(ItemSmem &sm, const StepArgs &a, int n_first, uint32_t k, uint8_t *sb,
+                                        uint64_t *bar)
 {
-    const uint32_t k = sm.prod_issued;
     if ((k & 31u) == 0) {
         asm volatile("cp.async.wait_all;" ::: "memory");
         __syncwarp();
-        fetch_rec_chunk(sm, a, (k >> 5) + 1);
+        fetch_rec_chunk(sm, a, n_first, (k >> 5) + 1);
     }
-    const int4 st = sm.recs[(k >> 5) & 1][k & 31];
-    __syncwarp();
-    stage_item<KDA>(a, st, sb, bar);
-    if ((threadIdx.x & 31) == 0) {
-        sm.prod_n += gridDim.x;
-        sm.prod_issued = k + 1;
-    }
-    __syncwarp();
+    stage_item<KDA>(a, sm.recs[(k >> 5) & 1][k & 31], sb, bar);
 }
 
 // Phase 0 of a staged item (threads 128..255, row i = tid - 128): per-row
@@ -892,14 +881,15 @@ __device__ __forceinline__ FitResult run_item(ItemSmem &sm, const StepArgs &a, R
 }
 
 // After a failed wait: record it, let every copy that may still be in flight
-// (consumption counts first_pending .. issued - 1) land, then the CTA returns.
-__device__ __forceinline__ void abort_drain(ItemSmem &sm, const StepArgs &a, uint32_t first_pending, int code)
+// (stagings first_pending .. issued - 1) land, then the CTA returns.
+__device__ __forceinline__ void abort_drain(ItemSmem &sm, const StepArgs &a, uint32_t first_pending, uint32_t issued,
+                                            int code)
 {
     if ((threadIdx.x >> 5) == kProducerWarp) {
         asm volatile("cp.async.wait_all;" ::: "memory");
         if ((threadIdx.x & 31) == 0) {
             atomicExch(a.t.status, code);
-            for (uint32_t m = first_pending; m < sm.prod_issued; m++)
+            for (uint32_t m = first_pending; m < issued; m++)
                 mbar_wait_bounded(&sm.bar[m % (uint32_t)a.nslots], (m / (uint32_t)a.nslots) & 1u, kWaitLimit);
         }
     }
@@ -923,31 +913,31 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
     // first staged position of this CTA: the smallest n >= npiv with n = blockIdx.x (mod G)
     int n_first = blockIdx.x;
     if (n_first < npiv) n_first += ((npiv - n_first + G - 1) / G) * G;
+    // stagings of this CTA: positions n_first, n_first + G, ...
+    const uint32_t n_stage = (n_first < a.n_items) ? (uint32_t)((a.n_items - n_first + G - 1) / G) : 0u;
+    const uint32_t in_flight0 = (n_stage < (uint32_t)a.nslots) ? n_stage : (uint32_t)a.nslots;
     if ((tid >> 5) == kProducerWarp) {
-        if ((tid & 31) == 0) {
-            sm.prod_first = n_first;
-            sm.prod_n = n_first;
-            sm.prod_issued = 0;
-        }
-        __syncwarp();
-        fetch_rec_chunk(sm, a, 0);
-        for (int s = 0; s < a.nslots && sm.prod_n < a.n_items; s++)
-            produce<KDA>(sm, a, ring + s * a.slot_bytes, &sm.bar[s]);
+        fetch_rec_chunk(sm, a, n_first, 0);
+        for (uint32_t k = 0; k < in_flight0; k++) produce<KDA>(sm, a, n_first, k, ring + k * a.slot_bytes, &sm.bar[k]);
     }
     for (int n = blockIdx.x; n < npiv && n < a.n_items; n += G) pivot_item(a, a.t.order[n]);
-    if (n_first >= a.n_items) return;  // nothing was staged
+    if (n_stage == 0) {  // nothing was staged
+        if ((tid >> 5) == kProducerWarp) asm volatile("cp.async.wait_all;" ::: "memory");
+        return;
+    }
 
     // phase 0 of the first staged item
     {
         const StageNext<KDA> first{sm, a, ring, n_first, 0, 0u, sm.u.rf[0]};
         const bool ok = (tid >= kDK) ? first() : first.rowside(tid);
         if (!__syncthreads_and(ok)) {
-            abort_drain(sm, a, 0u, kStatusWaitTimeout);
+            abort_drain(sm, a, 0u, in_flight0, kStatusWaitTimeout);
             return;
         }
     }
     uint32_t n_cons = 0;  // consumption count of the item; its slot and barrier parity below
     int par = 0, slot = 0;
+    const uint32_t nsl = (uint32_t)a.nslots;
     uint32_t parity = 0;
     for (int n = n_first; n < a.n_items; n += G, par ^= 1) {
         RowFactors &rf = sm.u.rf[par];
@@ -969,26 +959,27 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
                 case 7: res = run_item<7, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
                 case 8: res = run_item<8, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
                 default:  // unreachable: Gated-DeltaNet heads have one width, validated on the host
-                    abort_drain(sm, a, n_cons, kStatusBadHead);
+                    abort_drain(sm, a, n_cons, min(n_cons + nsl, n_stage), kStatusBadHead);
                     return;
             }
         }
         if (res == kFitAbortNow) {
-            abort_drain(sm, a, n_cons, kStatusWaitTimeout);
+            abort_drain(sm, a, n_cons, min(n_cons + nsl, n_stage), kStatusWaitTimeout);
             return;
         }
         if (res == kFitAbortAfter) {
-            abort_drain(sm, a, n_cons + 1, kStatusWaitTimeout);
+            abort_drain(sm, a, n_cons + 1, min(n_cons + nsl, n_stage), kStatusWaitTimeout);
             return;
         }
         // every warp is past the item's second barrier, so the slot is free:
-        // stage the next position into it
-        if ((tid >> 5) == kProducerWarp && sm.prod_n < a.n_items)
-            produce<KDA>(sm, a, ring + slot * a.slot_bytes, &sm.bar[slot]);
+        // stage the position n_cons + nslots stagings on into it
+        if ((tid >> 5) == kProducerWarp && n_cons + nsl < n_stage)
+            produce<KDA>(sm, a, n_first, n_cons + nsl, ring + slot * a.slot_bytes, &sm.bar[slot]);
         n_cons++;
         slot = slot_next;
         parity = parity_next;
     }
+    if ((tid >> 5) == kProducerWarp) asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
