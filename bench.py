@@ -257,6 +257,37 @@ def run_e2e(args, cfg, pool, host, out, stream, world):
             "steps": args.e2e_steps}
 
 
+def run_split(args, cfg, pool, ring, out, stream, world):
+    """The pages' split pipeline on the same pool and inputs: update + readout
+    into an fp32 work buffer, then fit + packed writeback on a side stream
+    (context for the fused step; not the headline)."""
+    import torch
+    import torch.distributed as dist
+    work = torch.empty((cfg.batch, cfg.heads, cfg.dk, cfg.dv), device="cuda")
+    side = torch.cuda.Stream()
+    n = max(10, args.steps // 50)
+
+    def split_step(i):
+        d = ring[i % RING]
+        pool.decode_step_split(d["q"], d["k"], d["v"], d["alpha"], d["beta"], work, out, side_stream=side)
+
+    for i in range(3):
+        split_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for i in range(n):
+        split_step(i)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s0.elapsed_time(s1), world, "cuda") / n
+    del work
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "steps": n, "work_buffer_bytes": cfg.items * cfg.dk * cfg.dv * 4}
+
+
 def main():
     args = parse()
     cfg = W.CONFIGS[args.config]
@@ -345,6 +376,7 @@ def main():
         host.append({k: torch.from_numpy(v).pin_memory() for k, v in x.items()})
     if not args.profile:
         e2e = run_e2e(args, cfg, pool, host, out, stream, world)
+    split = None if args.profile else run_split(args, cfg, pool, ring, out, stream, world)
 
     ring_bytes = sum(v.numel() * v.element_size() for v in ring[0].values())
     if rank == 0:
@@ -371,6 +403,9 @@ def main():
                 "state_bytes": cfg.items * cfg.dk * cfg.dv * 4},
             "clocks": clocks.summary(),
         }
+        if split is not None:
+            split["fused_speedup"] = split["ms_per_step"] / ms_per_step
+            line["split_pipeline"] = split
         if not (args.no_cpu_baseline or args.profile):
             rate, meta = cpu_oracle_rate(cfg, args.cpu_seconds)
             line["cpu_baseline"] = dict(value=rate, unit=UNIT, **meta)

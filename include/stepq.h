@@ -136,6 +136,25 @@ STEPQ_API stepq_status stepq_pool_destroy(stepq_pool *pool);
 STEPQ_API stepq_status stepq_pool_set_stream(stepq_pool *pool, void *cuda_stream);
 
 /*
+ * Restrict the pool's later decode steps to the requests active[0 ..
+ * n_active) (host array of distinct request indices in 0 .. batch-1, read
+ * during the call; NULL = every request, n_active ignored) -- the slot-indexed
+ * pool of a serving runtime, where requests come and go between steps and
+ * each keeps its slot of the state pool, as in a KV-cache allocation
+ * (ai.info summary, "Why This Matters": the packed state replaces the
+ * runtime's per-request state storage).  stepq_decode_step keeps its
+ * [batch, heads, ...] tensor shapes, indexed by request slot: it reads the
+ * rows of q, k, v, alpha, beta and writes the rows of out of the active
+ * requests only, and updates only their states; the other rows and states
+ * are neither read nor written.  The item order and staging tables in the
+ * pool buffer's tail are rebuilt on the host (heaviest heads first) and
+ * uploaded on the pool's stream (no sync).  stepq_pack, stepq_unpack and
+ * stepq_decode_step_split always cover every request (split returns
+ * STEPQ_ERR_UNSUPPORTED while a subset is active).
+ */
+STEPQ_API stepq_status stepq_pool_set_active(stepq_pool *pool, const int *active, int n_active);
+
+/*
  * Fit and quantise full-precision states into the pool (the initial state of
  * every item, or a restore from a checkpoint).  S: device fp32
  * [batch, heads, dk, dv].  Per item: row scales from the row's root-mean-square
@@ -166,6 +185,25 @@ STEPQ_API stepq_status stepq_unpack(stepq_pool *pool, float *S_out);
  */
 STEPQ_API stepq_status stepq_decode_step(stepq_pool *pool, const float *q, const float *k, const float *v,
                                const float *alpha, const float *beta, float *out);
+
+/*
+ * The same decode step as stepq_decode_step computed the way the pages'
+ * serving kernels split it (ai.info summary, "Key Contributions": the
+ * reconstruction, Delta update and readout fused, with scale fitting and
+ * packed writeback on a separate CUDA stream): one kernel reconstructs,
+ * updates and reads out, writing the updated unquantised state to S_work;
+ * then the fit and packed writeback (the stepq_pack kernel on S_work) run on
+ * side_stream, which waits for the first kernel, and the pool's stream waits
+ * for them.  Kept to measure the split against the single fused pass; the
+ * results agree with stepq_decode_step within rounding.  S_work: device fp32
+ * [batch, heads, dk, dv], 16-byte aligned, caller-owned, overwritten; must not
+ * overlap the pool or the step tensors.  side_stream: cudaStream_t; NULL or the
+ * pool's stream runs both halves on the pool's stream.  Other arguments as in
+ * stepq_decode_step.
+ */
+STEPQ_API stepq_status stepq_decode_step_split(stepq_pool *pool, float *S_work, const float *q, const float *k,
+                                               const float *v, const float *alpha, const float *beta, float *out,
+                                               void *side_stream);
 
 /*
  * The same update and readout on an unquantised fp32 state, in place: the

@@ -30,6 +30,12 @@ struct stepq_pool {
     int n_pivot_items = 0;
     int nslots = 0, slot_bytes = 0;
     int off_q = 0, off_k = 0, off_v = 0, off_alpha = 0, off_ab = 0, off_rec = 0;
+    // the active request set: decode steps update requests active[0..n_active)
+    int n_active = 0;
+    std::vector<int> kind;               // per head: kHeadQuant / kHeadAllPivot / kHeadMixed
+    std::vector<long long> item_bytes;   // per head
+    std::vector<long long> head_off;     // per head
+    std::vector<int> active_tables;      // host copy of the uploaded order and staging records
 };
 
 namespace {
@@ -182,6 +188,36 @@ stepq::StepArgs base_args(const stepq_pool *p)
     return a;
 }
 
+// Item order and staging records of a decode step over the requests
+// active[0 .. n_active) (all requests in order when active is NULL): position
+// list of the items b * H + h of the listed requests b.  Items of all-pivot
+// heads come first (processed from global memory), then the staged items,
+// heaviest heads first, equal weights in list order.
+void build_order_stage(int H, const int *active, int n_active, const std::vector<int> &kind,
+                       const std::vector<long long> &item_bytes, const long long *head_off, long long req_bytes,
+                       int *order, int *stage)
+{
+    std::vector<int> idx((size_t)n_active * H);
+    std::iota(idx.begin(), idx.end(), 0);
+    std::stable_sort(idx.begin(), idx.end(), [&](int x, int y) {
+        const int hx = x % H, hy = y % H;
+        const int px = kind[hx] == stepq::kHeadAllPivot, py = kind[hy] == stepq::kHeadAllPivot;
+        if (px != py) return px > py;
+        return item_bytes[hx] > item_bytes[hy];
+    });
+    for (size_t n = 0; n < idx.size(); n++) {
+        const int x = idx[n], h = x % H, r = x / H;
+        const int b = active ? active[r] : r;
+        const unsigned long long off = (unsigned long long)b * (unsigned long long)req_bytes +
+                                       (unsigned long long)head_off[h];
+        order[n] = b * H + h;
+        stage[4 * n + 0] = b * H + h;
+        stage[4 * n + 1] = (int)item_bytes[h] | (h << 16);
+        stage[4 * n + 2] = (int)(uint32_t)(off >> 10);  // items start at multiples of 1024 bytes
+        stage[4 * n + 3] = b;
+    }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -278,27 +314,8 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
         R.slab_words = L.slab_words[h];
         if (kind[h] != stepq::kHeadAllPivot) max_staged = std::max(max_staged, L.item_bytes[h]);
     }
-    // order: items of all-pivot heads first (processed from global memory), then
-    // the staged items, heaviest first
-    std::vector<int> idx((size_t)B * H);
-    std::iota(idx.begin(), idx.end(), 0);
-    std::stable_sort(idx.begin(), idx.end(), [&](int x, int y) {
-        const int hx = x % H, hy = y % H;
-        const int px = kind[hx] == stepq::kHeadAllPivot, py = kind[hy] == stepq::kHeadAllPivot;
-        if (px != py) return px > py;
-        return L.item_bytes[hx] > L.item_bytes[hy];
-    });
-    std::memcpy(order, idx.data(), idx.size() * sizeof(int));
-    int *stage = reinterpret_cast<int *>(at(L.off_stage));
-    for (size_t n = 0; n < idx.size(); n++) {
-        const int item = idx[n], h = item % H;
-        const unsigned long long off = (unsigned long long)(item / H) * (unsigned long long)L.req_bytes +
-                                       (unsigned long long)head_off[h];
-        stage[4 * n + 0] = item;
-        stage[4 * n + 1] = (int)L.item_bytes[h] | (h << 16);
-        stage[4 * n + 2] = (int)(uint32_t)(off & 0xFFFFFFFFull);
-        stage[4 * n + 3] = (int)(uint32_t)(off >> 32);
-    }
+    build_order_stage(H, nullptr, B, kind, L.item_bytes, head_off, L.req_bytes, order,
+                      reinterpret_cast<int *>(at(L.off_stage)));
     int n_pivot_items = 0;
     for (int h = 0; h < H; h++) n_pivot_items += (kind[h] == stepq::kHeadAllPivot) ? B : 0;
 
@@ -352,6 +369,10 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
     p->slot_bytes = slot_bytes;
     p->off_q = off_q; p->off_k = off_k; p->off_v = off_v;
     p->off_alpha = off_alpha; p->off_ab = off_ab; p->off_rec = off_rec;
+    p->n_active = B;
+    p->kind = kind;
+    p->item_bytes = L.item_bytes;
+    p->head_off.assign(head_off, head_off + H);
     {
         std::lock_guard<std::mutex> g(g_live_mu);
         g_live.insert(p);
@@ -378,6 +399,40 @@ stepq_status stepq_pool_set_stream(stepq_pool *pool, void *cuda_stream)
     stepq_status st = check_pool(pool);
     if (st != STEPQ_OK) return st;
     pool->stream = reinterpret_cast<cudaStream_t>(cuda_stream);
+    return STEPQ_OK;
+}
+
+stepq_status stepq_pool_set_active(stepq_pool *pool, const int *active, int n_active)
+{
+    stepq_status st = check_pool(pool);
+    if (st != STEPQ_OK) return st;
+    const int B = pool->desc.batch, H = pool->desc.heads;
+    if (!active) n_active = B;
+    if (n_active < 0 || n_active > B)
+        return fail(STEPQ_ERR_INVALID_ARG, "n_active = %d is outside 0 .. batch = %d", n_active, B);
+    if (active) {
+        std::vector<char> seen((size_t)B, 0);
+        for (int r = 0; r < n_active; r++) {
+            const int b = active[r];
+            if (b < 0 || b >= B) return fail(STEPQ_ERR_INVALID_ARG, "active[%d] = %d is not a request of the pool", r, b);
+            if (seen[b]) return fail(STEPQ_ERR_INVALID_ARG, "request %d is listed twice", b);
+            seen[b] = 1;
+        }
+    }
+    const size_t n = (size_t)n_active * H;
+    std::vector<int> &tb = pool->active_tables;
+    tb.assign(5 * n, 0);
+    build_order_stage(H, active, n_active, pool->kind, pool->item_bytes, pool->head_off.data(), pool->req_bytes,
+                      tb.data(), tb.data() + n);
+    if (n > 0) {
+        cudaError_t e = cudaMemcpyAsync(const_cast<int *>(pool->t.order), tb.data(), 4 * n, cudaMemcpyHostToDevice,
+                                        pool->stream);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(const_cast<int4 *>(pool->t.stage), tb.data() + n, 16 * n, cudaMemcpyHostToDevice,
+                                pool->stream);
+        if (e != cudaSuccess) return cuda_fail(e, "stepq_pool_set_active upload");
+    }
+    pool->n_active = n_active;
     return STEPQ_OK;
 }
 
@@ -436,15 +491,68 @@ stepq_status stepq_decode_step(stepq_pool *pool, const float *q, const float *k,
 {
     stepq_status st = check_pool(pool);
     if (st != STEPQ_OK) return st;
-    const size_t n = (size_t)pool->desc.batch * pool->desc.heads;
-    if (n == 0) return STEPQ_OK;
+    const size_t n = (size_t)pool->desc.batch * pool->desc.heads;  // rows of the step tensors
+    if (n == 0 || pool->n_active == 0) return STEPQ_OK;
     if ((st = check_step_tensors(pool->desc.variant, n, q, k, v, alpha, beta, out)) != STEPQ_OK) return st;
     if (overlaps(out, n * kDV * 4, pool->dev, pool->bytes))
         return fail(STEPQ_ERR_INVALID_ARG, "out overlaps the pool buffer");
     stepq::StepArgs a = base_args(pool);
+    // the active requests' items: the tables hold n_active * heads positions
+    a.n_items = pool->n_active * pool->desc.heads;
+    a.n_pivot_items = 0;
+    for (int h = 0; h < pool->desc.heads; h++)
+        a.n_pivot_items += (pool->kind[h] == stepq::kHeadAllPivot) ? pool->n_active : 0;
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.out = out;
     cudaError_t e = stepq::launch_decode_step(a, pool->stream);
     return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "stepq_decode_step launch");
+}
+
+stepq_status stepq_decode_step_split(stepq_pool *pool, float *S_work, const float *q, const float *k,
+                                     const float *v, const float *alpha, const float *beta, float *out,
+                                     void *side_stream)
+{
+    stepq_status st = check_pool(pool);
+    if (st != STEPQ_OK) return st;
+    if (pool->n_active != pool->desc.batch)
+        return fail(STEPQ_ERR_UNSUPPORTED, "stepq_decode_step_split needs every request active");
+    const size_t n = (size_t)pool->desc.batch * pool->desc.heads;
+    if (n == 0) return STEPQ_OK;
+    if ((st = check_step_tensors(pool->desc.variant, n, q, k, v, alpha, beta, out)) != STEPQ_OK) return st;
+    if ((st = check_dev(S_work, "S_work", 16)) != STEPQ_OK) return st;
+    const size_t nw = n * kDK * kDV * 4;
+    if (overlaps(out, n * kDV * 4, pool->dev, pool->bytes))
+        return fail(STEPQ_ERR_INVALID_ARG, "out overlaps the pool buffer");
+    if (overlaps(S_work, nw, pool->dev, pool->bytes) || overlaps(S_work, nw, out, n * kDV * 4) ||
+        overlaps(S_work, nw, q, n * kDK * 4) || overlaps(S_work, nw, k, n * kDK * 4) ||
+        overlaps(S_work, nw, v, n * kDV * 4))
+        return fail(STEPQ_ERR_INVALID_ARG, "S_work overlaps the pool or a step tensor");
+    stepq::StepArgs a = base_args(pool);
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.out = out;
+    a.S_in = S_work;
+    cudaError_t e = stepq::launch_split_update(a, pool->stream);
+    if (e != cudaSuccess) return cuda_fail(e, "stepq_decode_step_split update launch");
+    cudaStream_t side = reinterpret_cast<cudaStream_t>(side_stream);
+    if (side == nullptr || side == pool->stream) {
+        e = stepq::launch_pack(a, pool->stream);
+        return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "stepq_decode_step_split pack launch");
+    }
+    // fit + writeback on the side stream, ordered after the update and before
+    // the pool stream's later work
+    cudaEvent_t ev[2] = {nullptr, nullptr};
+    for (int i = 0; i < 2; i++) {
+        e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            if (ev[0]) cudaEventDestroy(ev[0]);
+            return cuda_fail(e, "stepq_decode_step_split event");
+        }
+    }
+    if ((e = cudaEventRecord(ev[0], pool->stream)) == cudaSuccess &&
+        (e = cudaStreamWaitEvent(side, ev[0], 0)) == cudaSuccess &&
+        (e = stepq::launch_pack(a, side)) == cudaSuccess && (e = cudaEventRecord(ev[1], side)) == cudaSuccess)
+        e = cudaStreamWaitEvent(pool->stream, ev[1], 0);
+    cudaEventDestroy(ev[0]);
+    cudaEventDestroy(ev[1]);
+    return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "stepq_decode_step_split side stream");
 }
 
 stepq_status stepq_fp32_step(const stepq_desc *desc, float *S, const float *q, const float *k,
@@ -643,8 +751,8 @@ stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *states, siz
                 order[pos] = item;
                 stage[4 * pos + 0] = item;
                 stage[4 * pos + 1] = (int)item_bytes[h] | (h << 16);
-                stage[4 * pos + 2] = (int)(uint32_t)(offb & 0xFFFFFFFFull);
-                stage[4 * pos + 3] = (int)(uint32_t)(offb >> 32);
+                stage[4 * pos + 2] = (int)(uint32_t)(offb >> 10);  // items start at multiples of 1024 bytes
+                stage[4 * pos + 3] = b;
                 pos++;
             }
         c0 = c1;

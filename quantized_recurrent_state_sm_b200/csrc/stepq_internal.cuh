@@ -47,7 +47,8 @@ struct Tables {
     const long long *head_off;  // [H] byte offset of head h's item inside a request
     const int *head_bytes;      // [H] bytes of an item of head h
     const int *order;           // [B*H] item processing order: all-pivot heads' items first
-    const int4 *stage;          // [B*H] per position: {item, item bytes | head << 16, pool offset lo, hi}
+    // [B*H] per position: {item, item bytes | head << 16, state offset / 1024, request}
+    const int4 *stage;
     int *status;                // device status word: 0 ok, else an error code
 };
 
@@ -77,6 +78,9 @@ constexpr int kStatusBadHead = 2;
 cudaError_t launch_decode_step(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_pack(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_unpack(const StepArgs &a, cudaStream_t s);
+// The pages' split pipeline, first half: reconstruct, update, read out; the
+// updated unquantised state goes to a.S_in (a work buffer), for launch_pack.
+cudaError_t launch_split_update(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_fp32_step(float *S, const float *q, const float *k, const float *v,
                              const float *alpha, const float *beta, float *out, int n_items,
                              int kda, cudaStream_t s);

@@ -566,12 +566,13 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
 // update and readout, no fit.  Every row of the item is a pivot row, so each
 // stream holds 16 rows x 4 binary16 values (two words per row), and each
 // thread derives its own rows' factors; no barrier.
-__device__ void pivot_item(const StepArgs &a, int item)
+__device__ void pivot_item(const StepArgs &a, int pos)
 {
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31, rg = l & 7, cg = l >> 3;
     const int col0 = 16 * w + 4 * cg;
-    const int rq = item / a.heads, h = item - rq * a.heads;
-    uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + a.t.head_off[h];
+    const int4 st = a.t.stage[pos];  // {item, bytes | head << 16, state offset / 1024, request}
+    const int item = st.x;
+    uint8_t *item_g = a.pool + ((long long)(uint32_t)st.z << 10);
     const long long vec = (long long)item * kDK + kRowsPerGroup * rg;
     const float beta = a.beta[item];
     uint32_t *words = reinterpret_cast<uint32_t *>(item_g + kHeaderBytes) + (kStreams * 2 * kRowsPerGroup) * w + l;
@@ -647,7 +648,7 @@ __device__ __forceinline__ void stage_item(const StepArgs &a, int4 st, uint8_t *
     const long long vec = (long long)item * kDK;
     if (lane == 0) {
         const uint32_t bytes = (uint32_t)st.y & 0xFFFFu;
-        const uint8_t *src = a.pool + (long long)(((unsigned long long)(uint32_t)st.w << 32) | (uint32_t)st.z);
+        const uint8_t *src = a.pool + ((long long)(uint32_t)st.z << 10);
         mbar_arrive_expect_tx(bar, bytes + (uint32_t)sizeof(HeadRec));
         bulk_g2s(sb, src, bytes, bar);
         bulk_g2s(sb + a.off_rec, a.t.rowrec + h, sizeof(HeadRec), bar);
@@ -740,6 +741,7 @@ __device__ __forceinline__ void phase0(RowFactors &rf, const StepArgs &a, const 
         rf.beta = beta;
         rf.item = item;
         rf.head_b = rec->head_b;
+
     }
 }
 
@@ -920,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
         fetch_rec_chunk(sm, a, n_first, 0);
         for (uint32_t k = 0; k < in_flight0; k++) produce<KDA>(sm, a, n_first, k, ring + k * a.slot_bytes, &sm.bar[k]);
     }
-    for (int n = blockIdx.x; n < npiv && n < a.n_items; n += G) pivot_item(a, a.t.order[n]);
+    for (int n = blockIdx.x; n < npiv && n < a.n_items; n += G) pivot_item(a, n);
     if (n_stage == 0) {  // nothing was staged
         if ((tid >> 5) == kProducerWarp) asm volatile("cp.async.wait_all;" ::: "memory");
         return;
@@ -1085,6 +1087,107 @@ __global__ void __launch_bounds__(kThreads) k_unpack(StepArgs a)
     }
 }
 
+// ---------------------------------------------------------------------------
+// The pages' own pipeline, kept for comparison with the fused step: a kernel
+// that reconstructs the state, applies the gated Delta update and reads out
+// (writing the updated unquantised state to a work buffer), followed by the
+// fit and packed writeback (k_pack on that buffer) on a second stream.  One
+// CTA per item, the decode mapping; the state is formed in absolute units in
+// the order of the recurrence: S' = alpha S, v_old = S'^T k,
+// S = S' + beta k (v - v_old)^T, o = S^T q.
+// ---------------------------------------------------------------------------
+template <int B>
+__device__ __forceinline__ void split_update_body(const RowFactors &rf, const HeadRec *rec, const StepArgs &a,
+                                                  int item, const uint8_t *item_g, float *S_work)
+{
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31, rg = l & 7, cg = l >> 3;
+    const int col0 = 16 * w + 4 * cg;
+    const int W = (B > 0) ? 2 * B : rec->slab_words;
+    X2 X;
+    decode_stream<B>(rf.rb + rg, reinterpret_cast<const uint32_t *>(item_g + kHeaderBytes) + (kStreams * W) * w + l, X);
+    const float *r = reinterpret_cast<const float *>(item_g);
+    const float4 c4 = ld4(r + kDK + col0);
+    const long long vec = (long long)item * kDK + kRowsPerGroup * rg;
+    float2 V0 = f2(0.f, 0.f), V1 = V0;
+    float kk[kRowsPerGroup], qq[kRowsPerGroup];
+#pragma unroll
+    for (int q4 = 0; q4 < kRowsPerGroup / 4; q4++) {
+        const float4 k4 = ld4(a.k + vec + 4 * q4), v4 = ld4(a.q + vec + 4 * q4);
+        const float4 al4 = a.kda ? ld4(a.alpha + vec + 4 * q4)
+                                 : make_float4(a.alpha[item], a.alpha[item], a.alpha[item], a.alpha[item]);
+        const float ka[4] = {k4.x, k4.y, k4.z, k4.w}, qa[4] = {v4.x, v4.y, v4.z, v4.w};
+        const float aa[4] = {al4.x, al4.y, al4.z, al4.w};
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const int rr = 4 * q4 + e, i = kRowsPerGroup * rg + rr;
+            kk[rr] = ka[e];
+            qq[rr] = qa[e];
+            float2 s0, s1;
+            if (B == 0 && rf.rb[8 * rr + rg] == kPivotBits) {
+                s0 = X[rr][0];
+                s1 = X[rr][1];
+            } else {
+                const float ri = r[i];
+                s0 = f2(__fmul_rn(__fmul_rn(ri, c4.x), X[rr][0].x), __fmul_rn(__fmul_rn(ri, c4.y), X[rr][0].y));
+                s1 = f2(__fmul_rn(__fmul_rn(ri, c4.z), X[rr][1].x), __fmul_rn(__fmul_rn(ri, c4.w), X[rr][1].y));
+            }
+            const float2 a2 = f2(aa[e], aa[e]);
+            X[rr][0] = __fmul2_rn(a2, s0);
+            X[rr][1] = __fmul2_rn(a2, s1);
+            const float2 k2 = f2(ka[e], ka[e]);
+            V0 = __ffma2_rn(k2, X[rr][0], V0);
+            V1 = __ffma2_rn(k2, X[rr][1], V1);
+        }
+    }
+    // v_old over the 8 row groups (butterfly), then d for the thread's columns
+    V0 = __fadd2_rn(V0, shfl2(V0, 1)); V1 = __fadd2_rn(V1, shfl2(V1, 1));
+    V0 = __fadd2_rn(V0, shfl2(V0, 2)); V1 = __fadd2_rn(V1, shfl2(V1, 2));
+    V0 = __fadd2_rn(V0, shfl2(V0, 4)); V1 = __fadd2_rn(V1, shfl2(V1, 4));
+    const float4 v4 = ld4(a.v + (long long)item * kDV + col0);
+    const float2 d0 = f2(v4.x - V0.x, v4.y - V0.y), d1 = f2(v4.z - V1.x, v4.w - V1.y);
+    const float beta = a.beta[item];
+    float2 U0 = f2(0.f, 0.f), U1 = U0;
+    float *dst = S_work + (long long)item * kDK * kDV;
+#pragma unroll
+    for (int rr = 0; rr < kRowsPerGroup; rr++) {
+        const float g = beta * kk[rr];
+        const float2 g2 = f2(g, g), q2 = f2(qq[rr], qq[rr]);
+        X[rr][0] = __ffma2_rn(g2, d0, X[rr][0]);
+        X[rr][1] = __ffma2_rn(g2, d1, X[rr][1]);
+        U0 = __ffma2_rn(q2, X[rr][0], U0);
+        U1 = __ffma2_rn(q2, X[rr][1], U1);
+        *reinterpret_cast<float4 *>(dst + (kRowsPerGroup * rg + rr) * kDV + col0) =
+            make_float4(X[rr][0].x, X[rr][0].y, X[rr][1].x, X[rr][1].y);
+    }
+    U0 = __fadd2_rn(U0, shfl2(U0, 1)); U1 = __fadd2_rn(U1, shfl2(U1, 1));
+    U0 = __fadd2_rn(U0, shfl2(U0, 2)); U1 = __fadd2_rn(U1, shfl2(U1, 2));
+    U0 = __fadd2_rn(U0, shfl2(U0, 4)); U1 = __fadd2_rn(U1, shfl2(U1, 4));
+    if (rg == 0)
+        *reinterpret_cast<float4 *>(a.out + (long long)item * kDV + col0) = make_float4(U0.x, U0.y, U1.x, U1.y);
+}
+
+__global__ void __launch_bounds__(kThreads) k_split_update(StepArgs a)
+{
+    __shared__ RowFactors rf;
+    const int item = blockIdx.x;
+    const int rq = item / a.heads, h = item - rq * a.heads;
+    const HeadRec *rec = a.t.rowrec + h;
+    load_head(rf, rec);
+    __syncthreads();
+    const uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + rec->head_off;
+    float *S_work = const_cast<float *>(a.S_in);
+    switch (rec->head_kind == kHeadQuant ? rec->head_b : 0) {
+        case 2: split_update_body<2>(rf, rec, a, item, item_g, S_work); break;
+        case 3: split_update_body<3>(rf, rec, a, item, item_g, S_work); break;
+        case 4: split_update_body<4>(rf, rec, a, item, item_g, S_work); break;
+        case 5: split_update_body<5>(rf, rec, a, item, item_g, S_work); break;
+        case 6: split_update_body<6>(rf, rec, a, item, item_g, S_work); break;
+        case 7: split_update_body<7>(rf, rec, a, item, item_g, S_work); break;
+        case 8: split_update_body<8>(rf, rec, a, item, item_g, S_work); break;
+        default: split_update_body<0>(rf, rec, a, item, item_g, S_work); break;
+    }
+}
+
 // Unquantised fp32 state: the same update and readout, state read and written
 // in full precision (the baseline the packed state is compared with).
 __global__ void __launch_bounds__(kThreads) k_fp32_step(float *Sg, const float *q, const float *k,
@@ -1204,6 +1307,13 @@ cudaError_t launch_pack(const StepArgs &a, cudaStream_t s)
 {
     if (a.n_items == 0) return cudaSuccess;
     k_pack<<<a.n_items, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_split_update(const StepArgs &a, cudaStream_t s)
+{
+    if (a.n_items == 0) return cudaSuccess;
+    k_split_update<<<a.n_items, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -38,7 +38,7 @@ class Desc(C.Structure):
 EXPORTS = ("stepq_pool_bytes", "stepq_state_bytes", "stepq_pool_create", "stepq_pool_destroy",
            "stepq_pool_set_stream", "stepq_pack", "stepq_unpack", "stepq_decode_step",
            "stepq_fp32_step", "stepq_pool_check", "stepq_status_string", "stepq_last_error",
-           "stepq_decode_step_noalloc")
+           "stepq_decode_step_noalloc", "stepq_decode_step_split", "stepq_pool_set_active")
 
 
 def _load():
@@ -58,8 +58,11 @@ def _load():
     L.stepq_decode_step.argtypes = [P, P, P, P, P, P, P]
     L.stepq_fp32_step.argtypes = [D, P, P, P, P, P, P, P, P]
     L.stepq_decode_step_noalloc.argtypes = [D, P, C.c_size_t, P, P, P, P, P, P, P]
+    L.stepq_decode_step_split.argtypes = [P, P, P, P, P, P, P, P, P]
+    L.stepq_pool_set_active.argtypes = [P, P, C.c_int]
     for fn in ("stepq_pool_create", "stepq_pool_destroy", "stepq_pool_set_stream", "stepq_pool_check", "stepq_pack",
-               "stepq_unpack", "stepq_decode_step", "stepq_fp32_step", "stepq_decode_step_noalloc"):
+               "stepq_unpack", "stepq_decode_step", "stepq_fp32_step", "stepq_decode_step_noalloc",
+               "stepq_decode_step_split", "stepq_pool_set_active"):
         getattr(L, fn).restype = C.c_int
     L.stepq_status_string.argtypes = [C.c_int]; L.stepq_status_string.restype = C.c_char_p
     L.stepq_last_error.argtypes = []; L.stepq_last_error.restype = C.c_char_p
@@ -131,10 +134,30 @@ class PackedStatePool:
         _check(lib.stepq_pool_create(C.byref(self._desc), C.c_void_p(self.buffer.data_ptr()),
                                      self.nbytes, _stream_ptr(), C.byref(h)))
         self._h = h
+        self.n_active = batch
 
     @property
     def n_items(self) -> int:
         return self.batch * self.heads
+
+    def set_active(self, requests=None):
+        """Restrict later decode steps to the listed requests (distinct slot
+        indices in 0 .. batch-1); None = all.  decode_step keeps its
+        [batch, heads, ...] shapes: it reads and writes only the listed
+        requests' rows and updates only their states."""
+        if requests is None:
+            self._check_active(lib.stepq_pool_set_active(self._h, None, 0))
+            self.n_active = self.batch
+            return
+        arr = np.ascontiguousarray(np.asarray(requests, dtype=np.int32).reshape(-1))
+        self._sync_stream()
+        self._check_active(lib.stepq_pool_set_active(self._h, arr.ctypes.data_as(C.c_void_p), int(arr.size)))
+        self._active_host = arr  # the upload reads it on the stream
+        self.n_active = int(arr.size)
+
+    @staticmethod
+    def _check_active(status):
+        _check(status)
 
     @property
     def state(self) -> torch.Tensor:
@@ -164,6 +187,23 @@ class PackedStatePool:
         _check(lib.stepq_decode_step(self._h, _dev(q, "q", (B, H, DK)), _dev(k, "k", (B, H, DK)),
                                      _dev(v, "v", (B, H, DV)), _dev(alpha, "alpha", ash),
                                      _dev(beta, "beta", (B, H)), _dev(out, "out", (B, H, DV))))
+        return out
+
+    def decode_step_split(self, q, k, v, alpha, beta, S_work, out=None, side_stream=None) -> torch.Tensor:
+        """The same step as decode_step, split the way the pages' kernels split
+        it: update + readout into S_work (fp32 [B, H, 128, 128]), then fit and
+        packed writeback on side_stream (a torch.cuda.Stream; None = the
+        current stream)."""
+        B, H = self.batch, self.heads
+        if out is None:
+            out = torch.empty((B, H, DV), dtype=torch.float32, device=self.buffer.device)
+        ash = (B, H, DK) if self.variant == KDA else (B, H)
+        self._sync_stream()
+        side = None if side_stream is None else C.c_void_p(side_stream.cuda_stream)
+        _check(lib.stepq_decode_step_split(self._h, _dev(S_work, "S_work", (B, H, DK, DV)),
+                                           _dev(q, "q", (B, H, DK)), _dev(k, "k", (B, H, DK)),
+                                           _dev(v, "v", (B, H, DV)), _dev(alpha, "alpha", ash),
+                                           _dev(beta, "beta", (B, H)), _dev(out, "out", (B, H, DV)), side))
         return out
 
     def check(self):

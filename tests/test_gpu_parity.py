@@ -65,7 +65,7 @@ class Setup:
         return self.bits[self.slots[s] % self.cfg.heads]
 
 
-def lockstep(setup, steps, t0=0, full_inputs=True):
+def lockstep(setup, steps, t0=0, full_inputs=True, step=None):
     cfg = setup.cfg
     cmp = PoolComparison()
     S0 = oracle.initial_state(cfg, setup.req)
@@ -75,7 +75,10 @@ def lockstep(setup, steps, t0=0, full_inputs=True):
         setup.push_oracle_bytes()
         x = W.step_inputs(cfg, t) if full_inputs else None
         d = to_dev(x)
-        out = setup.gpu.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+        if step is None:
+            out = setup.gpu.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+        else:
+            out = step(setup.gpu, d)
         torch.cuda.synchronize()
         o_ref, dg = setup.ref.step(*setup.slot_inputs(x), diag=True)
         o = out.cpu().numpy()[setup.req].reshape(len(setup.slots), -1)
