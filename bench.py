@@ -171,35 +171,65 @@ def rank_step_offset(rank):
     return 1000 * rank
 
 
-def cpu_oracle_rate(cfg, seconds):
-    """The CPU oracle as it stands (single thread) on a bounded sample of the
-    workload: the parity requests {0, 1, B/2, B-1} x all heads, consecutive
-    steps until `seconds` of CPU time have been spent.  Returns items/s."""
+def _oracle_worker(cfg_index, overrides, part, n_parts, seconds, start):
+    """One process of the CPU baseline: the oracle, single-threaded, stepping
+    its share of the sample (every n_parts-th item) until `seconds` of wall time
+    after the shared start instant.  Returns (items, busy seconds, steps)."""
     import oracle
+    cfg = W.with_overrides(W.CONFIGS[cfg_index], **overrides)
     req = W.parity_requests(cfg)
     H = cfg.heads
     slots = (np.asarray(req)[:, None] * H + np.arange(H)[None, :]).reshape(-1)
+    mine = np.arange(len(slots))[part::n_parts]
     bits, rho = W.bit_table(cfg), W.rho(cfg)
     kda = cfg.variant == W.KDA
-    pool = oracle.SlotPool(slots % H, bits, rho, ls_iters=cfg.ls_iters, kda=kda)
-    rng = np.random.default_rng(0)
-    pool.pack((rng.standard_normal((len(slots), 128, 128)) * 0.1).astype(np.float32))
-    n = len(slots)
-    items = 0
-    busy = 0.0
-    t = 0
-    while busy < seconds:
+    pool = oracle.SlotPool(slots[mine] % H, bits, rho, ls_iters=cfg.ls_iters, kda=kda)
+    rng = np.random.default_rng(part)
+    pool.pack((rng.standard_normal((len(mine), 128, 128)) * 0.1).astype(np.float32))
+    n = len(mine)
+    while time.time() < start:
+        time.sleep(0.001)
+    items, busy, t = 0, 0.0, 0
+    while time.time() < start + seconds:
         x = W.step_inputs(cfg, t, req)
-        args = (x["q"].reshape(n, -1), x["k"].reshape(n, -1), x["v"].reshape(n, -1),
-                x["alpha"].reshape(n, -1) if kda else x["alpha"].reshape(-1), x["beta"].reshape(-1))
+        f = {k: v.reshape(len(slots), -1)[mine] for k, v in x.items()}
+        args = (f["q"], f["k"], f["v"], f["alpha"] if kda else f["alpha"].reshape(-1), f["beta"].reshape(-1))
         t0 = time.perf_counter()
         pool.step(*args)
         busy += time.perf_counter() - t0
         items += n
         t += 1
-    return items / busy, {"kind": "oracle", "cores": 1,
-                          "sample": f"{n} items (requests {req} x {H} heads) x {t} steps of {cfg.name}, "
-                                    f"single-threaded C oracle, {busy:.1f} s"}
+    return items, busy, t
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_rate(cfg, seconds, cores=None):
+    """The CPU oracle as it stands, on the host's cores: the bounded sample is
+    the parity requests {0, 1, B/2, B-1} x all heads, split over `cores`
+    single-threaded processes (spawned, so safe after CUDA use), each stepping
+    its items for `seconds`.  Returns (items/s over the whole sample, meta)."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    req = W.parity_requests(cfg)
+    n_items = len(req) * cfg.heads
+    P = max(1, min(cores or host_cores(), n_items))
+    overrides = {k: getattr(cfg, k) for k in ("batch", "heads", "ls_iters")}
+    start = time.time() + 15.0 + 0.05 * P  # after every process has imported and packed
+    with cf.ProcessPoolExecutor(max_workers=P, mp_context=mp.get_context("spawn")) as ex:
+        futs = [ex.submit(_oracle_worker, cfg.index, overrides, p, P, seconds, start) for p in range(P)]
+        res = [f.result() for f in futs]
+    steps = min(r[2] for r in res)
+    rate = sum(r[0] / r[1] for r in res if r[1] > 0)  # the processes run side by side
+    return rate, {"kind": "oracle", "cores": P,
+                  "sample": f"{n_items} items (requests {req} x {cfg.heads} heads) of {cfg.name}, "
+                            f"split over {P} single-threaded C-oracle processes, {seconds:.0f} s each, "
+                            f">= {steps} steps per process"}
 
 
 def run_reference(args, cfg):
@@ -409,6 +439,8 @@ def main():
         if not (args.no_cpu_baseline or args.profile):
             rate, meta = cpu_oracle_rate(cfg, args.cpu_seconds)
             line["cpu_baseline"] = dict(value=rate, unit=UNIT, **meta)
+            rate1, meta1 = cpu_oracle_rate(cfg, max(1.0, args.cpu_seconds / 2), cores=1)
+            line["cpu_baseline_single_thread"] = dict(value=rate1, unit=UNIT, **meta1)
         print(json.dumps(line), flush=True)
     pool.close()
     if world > 1:
