@@ -101,7 +101,11 @@ typedef struct stepq_pool stepq_pool; /* opaque handle */
  *   W (one value per head) is the largest over the 8 row groups of
  *   ceil(4 * sum of the group's widths / 32); for a head of one width b,
  *   W = 2b.  Word m of stream l sits at slab byte offset 4 * (32 m + l), so
- *   a slab takes 128 W bytes and an item 4 dk + 4 dv + 1024 W bytes.  A field
+ *   a slab takes 128 W bytes and an item 4 dk + 4 dv + 1024 W bytes.
+ *   "Key row" above means storage row: a head whose rows all have one width
+ *   stores them in key order; otherwise the key rows are sorted by width
+ *   (widest first, ties by key index) and the j-th sorted row is storage row
+ *   16 (j % (dk/16)) + j / (dk/16).  r[] is in storage order too.  A field
  *   of a quantised row holds the offset-binary code (code + 2^(b_i - 1), in
  *   1 .. 2^b_i - 1); a field of a pivot row holds the binary16 bits of the
  *   element.  The stored element is r_i * c_j * code_ij (ai-papers.net,

@@ -80,18 +80,48 @@ double oracle_column_error_f64(int dk, int dv, int j, const double *S, const uin
  * binary16 bits on a pivot row), concatenated into one little-endian bit
  * stream that is zero-padded to W 32-bit words.  W is one number per head: the
  * largest over the row groups of the words the group's fields need.  Word m of
- * stream l is stored at word m * NS + l of the slab. */
+ * stream l is stored at word m * NS + l of the slab.
+ *
+ * Storage rows.  "Row" above means a storage row.  If every key row of the
+ * head has the same width, storage row s is key row s.  Otherwise the key
+ * rows are sorted by width, widest first (a pivot row counts 16), ties by key
+ * index, and the j-th of them is stored as storage row 16 (j % RG) + j / RG:
+ * the rows are dealt to the RG row groups in turn, so every group receives
+ * rows of the same widths (and the streams of a slab nearly the same length).
+ * The row scales r[] of the header are stored in storage order. */
 
 enum { GROUP_ROWS = 16, GROUP_COLS = 4, SLAB_COLS = 16 };
 
 static int field_bits(int b) { return b; } /* a pivot row's field is its 16 binary16 bits */
 
+/* key_of[s] = the key row stored as storage row s (rule above). */
+static void storage_rows(int dk, const uint8_t *bits, int *key_of)
+{
+    int uniform = 1;
+    for (int i = 1; i < dk; i++) uniform &= bits[i] == bits[0];
+    if (uniform || dk < GROUP_ROWS) {
+        for (int s = 0; s < dk; s++) key_of[s] = s;
+        return;
+    }
+    const int RG = dk / GROUP_ROWS;
+    int j = 0;
+    for (int b = 16; b >= 1; b--) /* widths from widest down; key order within a width */
+        for (int i = 0; i < dk; i++)
+            if (bits[i] == b) {
+                key_of[GROUP_ROWS * (j % RG) + j / RG] = i;
+                j++;
+            }
+}
+
 static size_t stream_words(int dk, const uint8_t *bits)
 {
+    int key_of[1024];
+    storage_rows(dk, bits, key_of);
     size_t W = 0;
     for (int g = 0; g < dk / GROUP_ROWS; g++) {
         size_t nbits = 0;
-        for (int rr = 0; rr < GROUP_ROWS; rr++) nbits += (size_t)GROUP_COLS * field_bits(bits[g * GROUP_ROWS + rr]);
+        for (int rr = 0; rr < GROUP_ROWS; rr++)
+            nbits += (size_t)GROUP_COLS * field_bits(bits[key_of[g * GROUP_ROWS + rr]]);
         const size_t w = (nbits + 31) / 32;
         if (w > W) W = w;
     }
@@ -117,7 +147,9 @@ void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const
     uint8_t *p = item;
     const int RG = dk / GROUP_ROWS, NS = GROUP_COLS * RG;
     const size_t W = stream_words(dk, bits);
-    for (int i = 0; i < dk; i++, p += 4) put_f32(p, r[i]);
+    int key_of[1024];
+    storage_rows(dk, bits, key_of);
+    for (int s = 0; s < dk; s++, p += 4) put_f32(p, r[key_of[s]]);
     for (int j = 0; j < dv; j++, p += 4) put_f32(p, c[j]);
     for (int sl = 0; sl < dv / SLAB_COLS; sl++) {
         memset(p, 0, 4 * W * NS);
@@ -125,7 +157,7 @@ void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const
             const int g = l % RG, cg = l / RG;
             size_t pos = 0; /* bit position in stream l */
             for (int rr = 0; rr < GROUP_ROWS; rr++) {
-                const int i = g * GROUP_ROWS + rr, b = bits[i];
+                const int i = key_of[g * GROUP_ROWS + rr], b = bits[i];
                 for (int kk = 0; kk < GROUP_COLS; kk++) {
                     const int j = sl * SLAB_COLS + cg * GROUP_COLS + kk;
                     const uint32_t u = (b == ORACLE_PIVOT_BITS)
@@ -146,14 +178,16 @@ void oracle_unpack_item(int dk, int dv, const uint8_t *bits, const uint8_t *item
     const uint8_t *p = item;
     const int RG = dk / GROUP_ROWS, NS = GROUP_COLS * RG;
     const size_t W = stream_words(dk, bits);
-    for (int i = 0; i < dk; i++, p += 4) r[i] = get_f32(p);
+    int key_of[1024];
+    storage_rows(dk, bits, key_of);
+    for (int s = 0; s < dk; s++, p += 4) r[key_of[s]] = get_f32(p);
     for (int j = 0; j < dv; j++, p += 4) c[j] = get_f32(p);
     for (int sl = 0; sl < dv / SLAB_COLS; sl++) {
         for (int l = 0; l < NS; l++) {
             const int g = l % RG, cg = l / RG;
             size_t pos = 0;
             for (int rr = 0; rr < GROUP_ROWS; rr++) {
-                const int i = g * GROUP_ROWS + rr, b = bits[i];
+                const int i = key_of[g * GROUP_ROWS + rr], b = bits[i];
                 for (int kk = 0; kk < GROUP_COLS; kk++) {
                     const int j = sl * SLAB_COLS + cg * GROUP_COLS + kk;
                     uint32_t u = 0;

@@ -109,7 +109,10 @@ double oracle_from_fp16(uint16_t h);
  * column by column, the row's b-bit offset-binary code (or 16 binary16 bits on
  * a pivot row), little-endian, zero-padded to W words, W per head = the most
  * any row group needs; word m of stream l sits at word m * NS + l of the slab.
- * Requires dk % 16 == 0 and dv % 16 == 0. */
+ * Storage rows: key order when the head has one width; otherwise the key rows
+ * sorted by width (widest first, ties by index), the j-th stored as row
+ * 16 (j % (dk/16)) + j / (dk/16); r[] is stored in storage order.
+ * Requires dk % 16 == 0, dk <= 1024 and dv % 16 == 0. */
 size_t oracle_item_bytes(int dk, int dv, const uint8_t *bits);
 void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
                       const int32_t *code, const float *piv, uint8_t *item);

@@ -60,6 +60,69 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// key_of[s]: the key row stored as storage row s.  Key order when the head's
+// rows share one width; otherwise the key rows sorted by width (widest first,
+// ties by key index), the j-th stored as row 16 (j % 8) + j / 8, so that every
+// row group holds rows of the same widths.
+void storage_rows(const uint8_t *bits, int *key_of)
+{
+    bool uniform = true;
+    for (int i = 1; i < kDK; i++) uniform &= bits[i] == bits[0];
+    if (uniform) {
+        for (int s = 0; s < kDK; s++) key_of[s] = s;
+        return;
+    }
+    int j = 0;
+    for (int b = STEPQ_PIVOT_BITS; b >= 1; b--)
+        for (int i = 0; i < kDK; i++)
+            if (bits[i] == b) {
+                key_of[stepq::kRowsPerGroup * (j % stepq::kRowGroups) + j / stepq::kRowGroups] = i;
+                j++;
+            }
+}
+
+// 32-bit words per stream (W): the most any row group of storage rows needs.
+int stream_words(const uint8_t *bits)
+{
+    int key_of[kDK];
+    storage_rows(bits, key_of);
+    int W = 0;
+    for (int g = 0; g < stepq::kRowGroups; g++) {
+        int bitsum = 0;
+        for (int rr = 0; rr < stepq::kRowsPerGroup; rr++) bitsum += bits[key_of[g * stepq::kRowsPerGroup + rr]];
+        W = std::max(W, (4 * bitsum + 31) / 32);
+    }
+    return W;
+}
+
+// The fit constants of head h in storage order (rec fields bits, s, rho, rq,
+// key_row, head_b); returns the number of pivot rows.
+int fill_rows(const stepq_desc *d, int h, stepq::HeadRec &R)
+{
+    const uint8_t *bits = d->bits + (size_t)h * kDK;
+    int key_of[kDK];
+    storage_rows(bits, key_of);
+    int npiv = 0, same = 1;
+    for (int s = 0; s < kDK; s++) {
+        const int i = key_of[s], b = bits[i];
+        R.key_row[s] = (uint8_t)i;
+        R.bits[s] = (uint8_t)b;
+        same &= (b == bits[0]);
+        if (b == STEPQ_PIVOT_BITS) {
+            npiv++;
+            R.s[s] = 0.f;
+            R.rho[s] = 0.f;
+            R.rq[s] = 0.f;
+        } else {
+            R.s[s] = (float)(1.0 / std::sqrt((double)d->rho[(size_t)h * kDK + i]));
+            R.rho[s] = d->rho[(size_t)h * kDK + i];
+            R.rq[s] = (float)(1.0 / (double)((1 << (b - 1)) - 1));
+        }
+    }
+    R.head_b = (same && bits[0] != STEPQ_PIVOT_BITS) ? bits[0] : 0;
+    return npiv;
+}
+
 struct Layout {
     size_t state = 0;
     size_t off_rec = 0, off_head_off = 0, off_head_bytes = 0, off_order = 0, off_stage = 0, off_status = 0,
@@ -108,13 +171,7 @@ stepq_status check_desc(const stepq_desc *d, bool need_tables, Layout *L)
         L->slab_words.assign(H, 0);
         long long req = 0;
         for (int h = 0; h < H; h++) {
-            int W = 0;
-            for (int g = 0; g < stepq::kRowGroups; g++) {
-                int bitsum = 0;
-                for (int rr = 0; rr < stepq::kRowsPerGroup; rr++)
-                    bitsum += d->bits[h * kDK + g * stepq::kRowsPerGroup + rr];
-                W = std::max(W, (4 * bitsum + 31) / 32);
-            }
+            const int W = stream_words(d->bits + (size_t)h * kDK);
             L->slab_words[h] = W;
             const long long n = stepq::kHeaderBytes + 4LL * W * stepq::kStreams * stepq::kSlabs;
             L->item_bytes[h] = n;
@@ -292,25 +349,9 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
         R.head_off = pre;
         R.head_bytes = (int)L.item_bytes[h];
         pre += L.item_bytes[h];
-        int npiv = 0, b0 = desc->bits[h * kDK], same = 1;
-        for (int i = 0; i < kDK; i++) {
-            const int b = desc->bits[h * kDK + i];
-            R.bits[i] = (uint8_t)b;
-            same &= (b == b0);
-            if (b == STEPQ_PIVOT_BITS) {
-                npiv++;
-                R.s[i] = 0.f;
-                R.rho[i] = 0.f;
-                R.rq[i] = 0.f;
-            } else {
-                R.s[i] = (float)(1.0 / std::sqrt((double)desc->rho[h * kDK + i]));
-                R.rho[i] = desc->rho[h * kDK + i];
-                R.rq[i] = (float)(1.0 / (double)((1 << (b - 1)) - 1));
-            }
-        }
+        const int npiv = fill_rows(desc, h, R);
         kind[h] = npiv == 0 ? stepq::kHeadQuant : (npiv == kDK ? stepq::kHeadAllPivot : stepq::kHeadMixed);
         R.head_kind = kind[h];
-        R.head_b = (same && b0 != STEPQ_PIVOT_BITS) ? b0 : 0;
         R.slab_words = L.slab_words[h];
         if (kind[h] != stepq::kHeadAllPivot) max_staged = std::max(max_staged, L.item_bytes[h]);
     }
@@ -622,13 +663,8 @@ stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *states, siz
     long long req = 0, max_staged = 0;
     int n_pivot_items = 0;
     for (int h = 0; h < H; h++) {
-        int W = 0, npiv = 0;
-        for (int g = 0; g < stepq::kRowGroups; g++) {
-            int bitsum = 0;
-            for (int rr = 0; rr < stepq::kRowsPerGroup; rr++)
-                bitsum += desc->bits[h * kDK + g * stepq::kRowsPerGroup + rr];
-            W = std::max(W, (4 * bitsum + 31) / 32);
-        }
+        const int W = stream_words(desc->bits + (size_t)h * kDK);
+        int npiv = 0;
         for (int i = 0; i < kDK; i++) npiv += desc->bits[h * kDK + i] == STEPQ_PIVOT_BITS;
         slab_words[h] = W;
         item_bytes[h] = stepq::kHeaderBytes + 4LL * W * stepq::kStreams * stepq::kSlabs;
@@ -699,19 +735,8 @@ stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *states, siz
     int *stage = reinterpret_cast<int *>(img + off_stage);
     for (int h = 0; h < H; h++) {
         stepq::HeadRec &R = rec[h];
-        int b0 = desc->bits[h * kDK], same = 1;
-        for (int i = 0; i < kDK; i++) {
-            const int b = desc->bits[h * kDK + i];
-            R.bits[i] = (uint8_t)b;
-            same &= (b == b0);
-            if (b != STEPQ_PIVOT_BITS) {
-                R.s[i] = (float)(1.0 / std::sqrt((double)desc->rho[h * kDK + i]));
-                R.rho[i] = desc->rho[h * kDK + i];
-                R.rq[i] = (float)(1.0 / (double)((1 << (b - 1)) - 1));
-            }
-        }
+        fill_rows(desc, h, R);
         R.head_off = head_off[h];
-        R.head_b = (same && b0 != STEPQ_PIVOT_BITS) ? b0 : 0;
         R.head_kind = kind[h];
         R.head_bytes = (int)item_bytes[h];
         R.slab_words = slab_words[h];

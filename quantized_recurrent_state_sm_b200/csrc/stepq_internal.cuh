@@ -27,10 +27,13 @@ constexpr int kHeadMixed = 2;     // some rows pivots
 // Per-head record (host-built, staged with every item): the fit constants and
 // the tile layout of the head's items.
 struct HeadRec {
-    float s[kDK];                // fp32(rho_i^-1/2), rounded once from fp64 (0 on pivot rows)
+    float s[kDK];                // fp32(rho_i^-1/2), rounded once from fp64 (0 on pivot rows), by storage row
     float rho[kDK];              // row-impact weights (0 on pivot rows)
     float rq[kDK];               // fp32(1 / Q_i), Q_i = 2^(b_i - 1) - 1 (0 on pivot rows)
+    // per storage row (key order for a one-width head; otherwise the key rows
+    // sorted by width and dealt to the row groups in turn):
     uint8_t bits[kDK];           // row widths (16 = pivot)
+    uint8_t key_row[kDK];        // the key row stored as this row
     long long head_off;          // byte offset of the head's item inside a request
     int head_b;                  // common row width, 0 if the rows differ
     int head_kind;               // kHeadQuant / kHeadAllPivot / kHeadMixed

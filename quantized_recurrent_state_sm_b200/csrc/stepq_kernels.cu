@@ -711,14 +711,14 @@ __device__ __forceinline__ void produce(ItemSmem &sm, const StepArgs &a, int n_f
 template <bool KDA>
 __device__ __forceinline__ void phase0(RowFactors &rf, const StepArgs &a, const uint8_t *sb, int item)
 {
-    const int i = threadIdx.x - kDK;
+    const int i = threadIdx.x - kDK;  // storage row
     const HeadRec *rec = reinterpret_cast<const HeadRec *>(sb + a.off_rec);
     const float beta = *reinterpret_cast<const float *>(sb + a.off_ab + 4);
-    const int b = rec->bits[i];
-    const float al = KDA ? reinterpret_cast<const float *>(sb + a.off_alpha)[i]
+    const int b = rec->bits[i], key = rec->key_row[i];
+    const float al = KDA ? reinterpret_cast<const float *>(sb + a.off_alpha)[key]
                          : *reinterpret_cast<const float *>(sb + a.off_ab);
-    const float k = reinterpret_cast<const float *>(sb + a.off_k)[i];
-    const float q = reinterpret_cast<const float *>(sb + a.off_q)[i];
+    const float k = reinterpret_cast<const float *>(sb + a.off_k)[key];
+    const float q = reinterpret_cast<const float *>(sb + a.off_q)[key];
     const float r = reinterpret_cast<const float *>(sb)[i];
     float A, g;
     if (b == kPivotBits) {
@@ -1009,7 +1009,7 @@ __device__ __forceinline__ void pack_body(ItemSmem &sm, RowFactors &rf, const He
     const float *src = a.S_in + (long long)item * kDK * kDV;
 #pragma unroll
     for (int rr = 0; rr < kRowsPerGroup; rr++) {
-        const float4 x = ld4(src + (kRowsPerGroup * rg + rr) * kDV + col0);
+        const float4 x = ld4(src + rec->key_row[kRowsPerGroup * rg + rr] * kDV + col0);
         X[rr][0] = f2(x.x, x.y);
         X[rr][1] = f2(x.z, x.w);
     }
@@ -1062,7 +1062,7 @@ __device__ __forceinline__ void unpack_body(const RowFactors &rf, const HeadRec 
             y = make_float4(__fmul_rn(__fmul_rn(ri, c4.x), X[rr][0].x), __fmul_rn(__fmul_rn(ri, c4.y), X[rr][0].y),
                             __fmul_rn(__fmul_rn(ri, c4.z), X[rr][1].x), __fmul_rn(__fmul_rn(ri, c4.w), X[rr][1].y));
         }
-        *reinterpret_cast<float4 *>(dst + i * kDV + col0) = y;
+        *reinterpret_cast<float4 *>(dst + rec->key_row[i] * kDV + col0) = y;
     }
 }
 
@@ -1107,16 +1107,19 @@ __device__ __forceinline__ void split_update_body(const RowFactors &rf, const He
     decode_stream<B>(rf.rb + rg, reinterpret_cast<const uint32_t *>(item_g + kHeaderBytes) + (kStreams * W) * w + l, X);
     const float *r = reinterpret_cast<const float *>(item_g);
     const float4 c4 = ld4(r + kDK + col0);
-    const long long vec = (long long)item * kDK + kRowsPerGroup * rg;
+    const long long vec = (long long)item * kDK;
     float2 V0 = f2(0.f, 0.f), V1 = V0;
     float kk[kRowsPerGroup], qq[kRowsPerGroup];
 #pragma unroll
     for (int q4 = 0; q4 < kRowsPerGroup / 4; q4++) {
-        const float4 k4 = ld4(a.k + vec + 4 * q4), v4 = ld4(a.q + vec + 4 * q4);
-        const float4 al4 = a.kda ? ld4(a.alpha + vec + 4 * q4)
-                                 : make_float4(a.alpha[item], a.alpha[item], a.alpha[item], a.alpha[item]);
-        const float ka[4] = {k4.x, k4.y, k4.z, k4.w}, qa[4] = {v4.x, v4.y, v4.z, v4.w};
-        const float aa[4] = {al4.x, al4.y, al4.z, al4.w};
+        float ka[4], qa[4], aa[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {  // the inputs of the key rows this thread's storage rows hold
+            const int key = rec->key_row[kRowsPerGroup * rg + 4 * q4 + e];
+            ka[e] = a.k[vec + key];
+            qa[e] = a.q[vec + key];
+            aa[e] = a.kda ? a.alpha[vec + key] : a.alpha[item];
+        }
 #pragma unroll
         for (int e = 0; e < 4; e++) {
             const int rr = 4 * q4 + e, i = kRowsPerGroup * rg + rr;
@@ -1156,7 +1159,7 @@ __device__ __forceinline__ void split_update_body(const RowFactors &rf, const He
         X[rr][1] = __ffma2_rn(g2, d1, X[rr][1]);
         U0 = __ffma2_rn(q2, X[rr][0], U0);
         U1 = __ffma2_rn(q2, X[rr][1], U1);
-        *reinterpret_cast<float4 *>(dst + (kRowsPerGroup * rg + rr) * kDV + col0) =
+        *reinterpret_cast<float4 *>(dst + rec->key_row[kRowsPerGroup * rg + rr] * kDV + col0) =
             make_float4(X[rr][0].x, X[rr][0].y, X[rr][1].x, X[rr][1].y);
     }
     U0 = __fadd2_rn(U0, shfl2(U0, 1)); U1 = __fadd2_rn(U1, shfl2(U1, 1));

@@ -304,12 +304,33 @@ def parity_requests(cfg: Config):
 GROUP_ROWS, GROUP_COLS, SLAB_COLS = 16, 4, 16
 
 
+def storage_rows(bits_head: np.ndarray) -> np.ndarray:
+    """key_of[s]: the key row stored as storage row s.  Key order when the head
+    has one width; otherwise the key rows sorted by width (widest first, ties
+    by key index), the j-th stored as row 16 (j % RG) + j // RG (RG = dk/16),
+    so that every row group holds rows of the same widths."""
+    bits_head = np.asarray(bits_head)
+    dk = bits_head.shape[0]
+    if np.all(bits_head == bits_head[0]):
+        return np.arange(dk)
+    rg = dk // GROUP_ROWS
+    order = np.lexsort((np.arange(dk), -bits_head.astype(np.int64)))
+    key_of = np.empty(dk, dtype=np.int64)
+    j = np.arange(dk)
+    key_of[GROUP_ROWS * (j % rg) + j // rg] = order
+    return key_of
+
+
 def stream_words(bits: np.ndarray) -> np.ndarray:
-    """32-bit words per stream of each head, [H]: the most any 16-row group
-    needs for its 4 columns' fields."""
+    """32-bit words per stream of each head, [H]: the most any 16-row group of
+    storage rows needs for its 4 columns' fields."""
     H, dk = bits.shape
-    per_group = bits.astype(np.int64).reshape(H, dk // GROUP_ROWS, GROUP_ROWS).sum(axis=2)
-    return ((GROUP_COLS * per_group + 31) // 32).max(axis=1)
+    out = np.zeros(H, dtype=np.int64)
+    for h in range(H):
+        sb = bits[h][storage_rows(bits[h])].astype(np.int64)
+        per_group = sb.reshape(dk // GROUP_ROWS, GROUP_ROWS).sum(axis=1)
+        out[h] = ((GROUP_COLS * per_group + 31) // 32).max()
+    return out
 
 
 def head_item_bytes(bits: np.ndarray, dv: int) -> np.ndarray:

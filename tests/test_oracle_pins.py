@@ -314,6 +314,20 @@ def stream_words(fields, nwords):
     return [(acc >> (32 * w)) & 0xFFFFFFFF for w in range(nwords)]
 
 
+def test_storage_rows_balance_widths():
+    """Every row group of a mixed-width head holds rows of nearly the same
+    widths (the deal of the sorted rows), and a one-width head keeps key order."""
+    assert list(W.storage_rows(np.full(128, 5, np.uint8))) == list(range(128))
+    r = rng(5)
+    bits = r.choice([3, 4, 5, 6, 7, 8, 16], size=128).astype(np.uint8)
+    key_of = W.storage_rows(bits)
+    assert sorted(key_of) == list(range(128))
+    groups = bits[key_of].astype(int).reshape(8, 16)
+    # row rr of every group: consecutive ranks, so widths differ by at most one step
+    assert np.all(groups.max(axis=0) - groups.min(axis=0) <= 16 - 8)
+    assert groups.sum(axis=1).max() - groups.sum(axis=1).min() <= 16
+
+
 def test_pack_format_slab_streams():
     r = rng(11)
     dk, dv = 128, 128
@@ -327,10 +341,16 @@ def test_pack_format_slab_streams():
             code[i] = r.integers(-Q, Q + 1, dv)
     rr = r.standard_normal(dk).astype(np.float32); cc = r.standard_normal(dv).astype(np.float32)
     item = oracle.pack_item(bits, rr, cc, code, piv)
+    # storage rows: widths differ, so the key rows sorted (widest first, ties
+    # by index) are dealt to the 8 row groups in turn
+    ranked = sorted(range(dk), key=lambda i: (-int(bits[i]), i))
+    key_of = [0] * dk
+    for j, i in enumerate(ranked):
+        key_of[16 * (j % 8) + j // 8] = i
     # W: the most words any 16-row group needs for 4 columns' fields
-    Wh = max((4 * int(bits[16 * g:16 * g + 16].astype(int).sum()) + 31) // 32 for g in range(8))
+    Wh = max((4 * sum(int(bits[key_of[16 * g + t]]) for t in range(16)) + 31) // 32 for g in range(8))
     assert item.size == 4 * dk + 4 * dv + 8 * 32 * 4 * Wh
-    assert bytes(item[:4 * dk]) == rr.astype("<f4").tobytes()
+    assert bytes(item[:4 * dk]) == rr[key_of].astype("<f4").tobytes()
     assert bytes(item[4 * dk: 4 * dk + 4 * dv]) == cc.astype("<f4").tobytes()
     words = item[4 * dk + 4 * dv:].view("<u4")
     for s_ in range(8):
@@ -339,7 +359,7 @@ def test_pack_format_slab_streams():
             g, cg = l % 8, l // 8
             fields = []
             for rho_ in range(16):
-                i = 16 * g + rho_
+                i = key_of[16 * g + rho_]
                 b = int(bits[i])
                 for k in range(4):
                     j = 16 * s_ + 4 * cg + k
