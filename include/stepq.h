@@ -96,18 +96,20 @@ typedef struct stepq_pool stepq_pool; /* opaque handle */
  *   Slab s covers value columns 16s .. 16s+15 of all dk key rows and holds
  *   32 interleaved streams: stream l (rg = l % 8, cg = l / 8) carries the
  *   fields of key rows 16rg .. 16rg+15 and value columns 16s + 4cg .. +3,
- *   row-major (row 16rg, its 4 columns first), each field b_i bits wide,
- *   packed little-endian into 32-bit words and zero-padded to W words, where
- *   W (one value per head) is the largest over the 8 row groups of
- *   ceil(4 * sum of the group's widths / 32); for a head of one width b,
- *   W = 2b.  Word m of stream l sits at slab byte offset 4 * (32 m + l), so
- *   a slab takes 128 W bytes and an item 4 dk + 4 dv + 1024 W bytes.
- *   "Key row" above means storage row: a head whose rows all have one width
- *   stores them in key order; otherwise the key rows are sorted by width
- *   (widest first, ties by key index) and the j-th sorted row is storage row
+ *   row-major (row 16rg, its 4 columns first), packed little-endian into
+ *   32-bit words and zero-padded to W words.  The fields of row 16rg + p
+ *   (position p) are F_p bits wide, F_p = the largest width at position p
+ *   over the 8 row groups, so every stream of a head has the same layout and
+ *   W = ceil(4 * (F_0 + ... + F_15) / 32); for a head of one width b,
+ *   F_p = b and W = 2b.  Word m of stream l sits at slab byte offset
+ *   4 * (32 m + l), so a slab takes 128 W bytes and an item
+ *   4 dk + 4 dv + 1024 W bytes.  "Key row" above means storage row: a head
+ *   whose rows all have one width stores them in key order; otherwise the key
+ *   rows are sorted by width (widest first, a pivot row counting 16, ties by
+ *   key index) and the j-th sorted row is storage row
  *   16 (j % (dk/16)) + j / (dk/16).  r[] is in storage order too.  A field
- *   of a quantised row holds the offset-binary code (code + 2^(b_i - 1), in
- *   1 .. 2^b_i - 1); a field of a pivot row holds the binary16 bits of the
+ *   of a quantised row holds the offset-binary code (code + 2^(F_p - 1));
+ *   a field of a pivot row (F_p = 16) holds the binary16 bits of the
  *   element.  The stored element is r_i * c_j * code_ij (ai-papers.net,
  *   "STEPQuantの仕組み"); pivot rows keep r_i = 0, and a Gated-DeltaNet
  *   pivot head keeps c_j = 0 as well.  The interleave lets the 32 lanes of a

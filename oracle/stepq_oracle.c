@@ -75,20 +75,26 @@ double oracle_column_error_f64(int dk, int dv, int j, const double *S, const uin
  * Slab s holds value columns 16s .. 16s+15 of every key row as NS = 4 dk/16
  * streams.  Stream l covers the key rows of row group l % (dk/16) (rows
  * 16 (l % (dk/16)) .. +15) and the value columns 16s + 4 (l / (dk/16)) .. +3:
- * its codes are taken row by row, and within a row column by column, as fields
- * of the row's width (the offset-binary code u = code + 2^(b-1), or the
- * binary16 bits on a pivot row), concatenated into one little-endian bit
- * stream that is zero-padded to W 32-bit words.  W is one number per head: the
- * largest over the row groups of the words the group's fields need.  Word m of
- * stream l is stored at word m * NS + l of the slab.
+ * its codes are taken row by row, and within a row column by column, as
+ * fields concatenated into one little-endian bit stream that is zero-padded
+ * to W 32-bit words.  Word m of stream l is stored at word m * NS + l of the
+ * slab.
  *
  * Storage rows.  "Row" above means a storage row.  If every key row of the
  * head has the same width, storage row s is key row s.  Otherwise the key
  * rows are sorted by width, widest first (a pivot row counts 16), ties by key
  * index, and the j-th of them is stored as storage row 16 (j % RG) + j / RG:
  * the rows are dealt to the RG row groups in turn, so every group receives
- * rows of the same widths (and the streams of a slab nearly the same length).
- * The row scales r[] of the header are stored in storage order. */
+ * rows of nearly the same widths.  The row scales r[] of the header are
+ * stored in storage order.
+ *
+ * Field widths.  The fields of storage row 16 g + p (position p of group g)
+ * are F_p bits wide, F_p = the largest width at position p over all row
+ * groups; a row narrower than its field is stored in the wider field.  A
+ * quantised row's field holds the offset-binary code u = code + 2^(F_p - 1),
+ * a pivot row's field (F_p = 16 then) the binary16 bits of the element.  Every
+ * stream of a head therefore has the same layout, and W = ceil(4 sum_p F_p /
+ * 32).  For a head of one width b, F_p = b and W = 2b. */
 
 enum { GROUP_ROWS = 16, GROUP_COLS = 4, SLAB_COLS = 16 };
 
@@ -113,19 +119,26 @@ static void storage_rows(int dk, const uint8_t *bits, int *key_of)
             }
 }
 
+/* fw[p] = F_p, the field width of position p (rule above), p < 16. */
+static void position_widths(int dk, const uint8_t *bits, const int *key_of, int *fw)
+{
+    for (int p = 0; p < GROUP_ROWS; p++) {
+        fw[p] = 0;
+        for (int g = 0; g < dk / GROUP_ROWS; g++) {
+            const int b = field_bits(bits[key_of[g * GROUP_ROWS + p]]);
+            if (b > fw[p]) fw[p] = b;
+        }
+    }
+}
+
 static size_t stream_words(int dk, const uint8_t *bits)
 {
-    int key_of[1024];
+    int key_of[1024], fw[GROUP_ROWS];
     storage_rows(dk, bits, key_of);
-    size_t W = 0;
-    for (int g = 0; g < dk / GROUP_ROWS; g++) {
-        size_t nbits = 0;
-        for (int rr = 0; rr < GROUP_ROWS; rr++)
-            nbits += (size_t)GROUP_COLS * field_bits(bits[key_of[g * GROUP_ROWS + rr]]);
-        const size_t w = (nbits + 31) / 32;
-        if (w > W) W = w;
-    }
-    return W;
+    position_widths(dk, bits, key_of, fw);
+    size_t nbits = 0;
+    for (int p = 0; p < GROUP_ROWS; p++) nbits += (size_t)GROUP_COLS * fw[p];
+    return (nbits + 31) / 32;
 }
 
 size_t oracle_item_bytes(int dk, int dv, const uint8_t *bits)
@@ -147,8 +160,9 @@ void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const
     uint8_t *p = item;
     const int RG = dk / GROUP_ROWS, NS = GROUP_COLS * RG;
     const size_t W = stream_words(dk, bits);
-    int key_of[1024];
+    int key_of[1024], fw[GROUP_ROWS];
     storage_rows(dk, bits, key_of);
+    position_widths(dk, bits, key_of, fw);
     for (int s = 0; s < dk; s++, p += 4) put_f32(p, r[key_of[s]]);
     for (int j = 0; j < dv; j++, p += 4) put_f32(p, c[j]);
     for (int sl = 0; sl < dv / SLAB_COLS; sl++) {
@@ -157,13 +171,13 @@ void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const
             const int g = l % RG, cg = l / RG;
             size_t pos = 0; /* bit position in stream l */
             for (int rr = 0; rr < GROUP_ROWS; rr++) {
-                const int i = key_of[g * GROUP_ROWS + rr], b = bits[i];
+                const int i = key_of[g * GROUP_ROWS + rr], b = bits[i], F = fw[rr];
                 for (int kk = 0; kk < GROUP_COLS; kk++) {
                     const int j = sl * SLAB_COLS + cg * GROUP_COLS + kk;
                     const uint32_t u = (b == ORACLE_PIVOT_BITS)
                                            ? oracle_to_fp16((double)piv[i * dv + j])
-                                           : (uint32_t)(code[i * dv + j] + (1 << (b - 1)));
-                    for (int t = 0; t < field_bits(b); t++, pos++)
+                                           : (uint32_t)(code[i * dv + j] + (1 << (F - 1)));
+                    for (int t = 0; t < F; t++, pos++)
                         if ((u >> t) & 1u) set_bit(p, (pos / 32) * NS + l, (int)(pos % 32));
                 }
             }
@@ -178,8 +192,9 @@ void oracle_unpack_item(int dk, int dv, const uint8_t *bits, const uint8_t *item
     const uint8_t *p = item;
     const int RG = dk / GROUP_ROWS, NS = GROUP_COLS * RG;
     const size_t W = stream_words(dk, bits);
-    int key_of[1024];
+    int key_of[1024], fw[GROUP_ROWS];
     storage_rows(dk, bits, key_of);
+    position_widths(dk, bits, key_of, fw);
     for (int s = 0; s < dk; s++, p += 4) r[key_of[s]] = get_f32(p);
     for (int j = 0; j < dv; j++, p += 4) c[j] = get_f32(p);
     for (int sl = 0; sl < dv / SLAB_COLS; sl++) {
@@ -187,17 +202,17 @@ void oracle_unpack_item(int dk, int dv, const uint8_t *bits, const uint8_t *item
             const int g = l % RG, cg = l / RG;
             size_t pos = 0;
             for (int rr = 0; rr < GROUP_ROWS; rr++) {
-                const int i = key_of[g * GROUP_ROWS + rr], b = bits[i];
+                const int i = key_of[g * GROUP_ROWS + rr], b = bits[i], F = fw[rr];
                 for (int kk = 0; kk < GROUP_COLS; kk++) {
                     const int j = sl * SLAB_COLS + cg * GROUP_COLS + kk;
                     uint32_t u = 0;
-                    for (int t = 0; t < field_bits(b); t++, pos++)
+                    for (int t = 0; t < F; t++, pos++)
                         u |= (uint32_t)get_bit(p, (pos / 32) * NS + l, (int)(pos % 32)) << t;
                     if (b == ORACLE_PIVOT_BITS) {
                         piv[i * dv + j] = (float)oracle_from_fp16((uint16_t)u);
                         code[i * dv + j] = 0;
                     } else {
-                        code[i * dv + j] = (int32_t)u - (1 << (b - 1));
+                        code[i * dv + j] = (int32_t)u - (1 << (F - 1));
                         piv[i * dv + j] = 0;
                     }
                 }

@@ -106,13 +106,16 @@ double oracle_from_fp16(uint16_t h);
  * item = r[dk] fp32 | c[dv] fp32 | slab 0 | ... | slab dv/16 - 1; slab s holds
  * value columns 16s..16s+15 as NS = 4 dk/16 streams.  Stream l covers key rows
  * 16 (l % (dk/16)) .. +15 and columns 16s + 4 (l / (dk/16)) .. +3: row by row,
- * column by column, the row's b-bit offset-binary code (or 16 binary16 bits on
- * a pivot row), little-endian, zero-padded to W words, W per head = the most
- * any row group needs; word m of stream l sits at word m * NS + l of the slab.
- * Storage rows: key order when the head has one width; otherwise the key rows
- * sorted by width (widest first, ties by index), the j-th stored as row
- * 16 (j % (dk/16)) + j / (dk/16); r[] is stored in storage order.
- * Requires dk % 16 == 0, dk <= 1024 and dv % 16 == 0. */
+ * column by column, an F_p-bit field per element (offset-binary code
+ * u = code + 2^(F_p - 1), or the 16 binary16 bits on a pivot row),
+ * little-endian, zero-padded to W = ceil(4 sum_p F_p / 32) words; F_p, the
+ * field width of position p (row 16 g + p of any group g), is the widest row
+ * at that position over the groups.  Word m of stream l sits at word
+ * m * NS + l of the slab.  Storage rows: key order when the head has one
+ * width; otherwise the key rows sorted by width (widest first, ties by
+ * index), the j-th stored as row 16 (j % (dk/16)) + j / (dk/16); r[] is
+ * stored in storage order.  Requires dk % 16 == 0, dk <= 1024 and
+ * dv % 16 == 0. */
 size_t oracle_item_bytes(int dk, int dv, const uint8_t *bits);
 void oracle_pack_item(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
                       const int32_t *code, const float *piv, uint8_t *item);

@@ -28,6 +28,7 @@ struct stepq_pool {
     cudaStream_t stream = nullptr;
     stepq::Tables t{};
     int n_pivot_items = 0;
+    int max_n16 = 0;  // the most leading 16-bit field positions of a staged head
     int nslots = 0, slot_bytes = 0;
     int off_q = 0, off_k = 0, off_v = 0, off_alpha = 0, off_ab = 0, off_rec = 0;
     // the active request set: decode steps update requests active[0..n_active)
@@ -81,18 +82,26 @@ void storage_rows(const uint8_t *bits, int *key_of)
             }
 }
 
-// 32-bit words per stream (W): the most any row group of storage rows needs.
+// F[p]: the field width of row position p (storage rows 16 g + p), the widest
+// row at that position over the row groups.
+void position_widths(const uint8_t *bits, const int *key_of, int *F)
+{
+    for (int p = 0; p < stepq::kRowsPerGroup; p++) {
+        F[p] = 0;
+        for (int g = 0; g < stepq::kRowGroups; g++)
+            F[p] = std::max(F[p], (int)bits[key_of[g * stepq::kRowsPerGroup + p]]);
+    }
+}
+
+// 32-bit words per stream (W): ceil(4 sum_p F[p] / 32).
 int stream_words(const uint8_t *bits)
 {
-    int key_of[kDK];
+    int key_of[kDK], F[stepq::kRowsPerGroup];
     storage_rows(bits, key_of);
-    int W = 0;
-    for (int g = 0; g < stepq::kRowGroups; g++) {
-        int bitsum = 0;
-        for (int rr = 0; rr < stepq::kRowsPerGroup; rr++) bitsum += bits[key_of[g * stepq::kRowsPerGroup + rr]];
-        W = std::max(W, (4 * bitsum + 31) / 32);
-    }
-    return W;
+    position_widths(bits, key_of, F);
+    int nbits = 0;
+    for (int p = 0; p < stepq::kRowsPerGroup; p++) nbits += 4 * F[p];
+    return (nbits + 31) / 32;
 }
 
 // The fit constants of head h in storage order (rec fields bits, s, rho, rq,
@@ -120,6 +129,14 @@ int fill_rows(const stepq_desc *d, int h, stepq::HeadRec &R)
         }
     }
     R.head_b = (same && bits[0] != STEPQ_PIVOT_BITS) ? bits[0] : 0;
+    int F[stepq::kRowsPerGroup];
+    position_widths(bits, key_of, F);
+    R.n16 = 0;
+    for (int p = 0; p < stepq::kRowsPerGroup; p++) {
+        R.pos_bits[p] = (uint8_t)F[p];
+        R.n16 += F[p] == STEPQ_PIVOT_BITS;
+    }
+    R.pad = 0;
     return npiv;
 }
 
@@ -242,6 +259,7 @@ stepq::StepArgs base_args(const stepq_pool *p)
     a.off_q = p->off_q; a.off_k = p->off_k; a.off_v = p->off_v;
     a.off_alpha = p->off_alpha; a.off_ab = p->off_ab; a.off_rec = p->off_rec;
     a.n_pivot_items = p->n_pivot_items;
+    a.max_n16 = p->max_n16;
     return a;
 }
 
@@ -341,6 +359,7 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
     int *order = reinterpret_cast<int *>(at(L.off_order));
     long long pre = 0;
     long long max_staged = 0;
+    int max_n16 = 0;
     std::vector<int> kind(H, stepq::kHeadQuant);
     for (int h = 0; h < H; h++) {
         stepq::HeadRec &R = rec[h];
@@ -353,7 +372,10 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
         kind[h] = npiv == 0 ? stepq::kHeadQuant : (npiv == kDK ? stepq::kHeadAllPivot : stepq::kHeadMixed);
         R.head_kind = kind[h];
         R.slab_words = L.slab_words[h];
-        if (kind[h] != stepq::kHeadAllPivot) max_staged = std::max(max_staged, L.item_bytes[h]);
+        if (kind[h] != stepq::kHeadAllPivot) {
+            max_staged = std::max(max_staged, L.item_bytes[h]);
+            max_n16 = std::max(max_n16, R.n16);
+        }
     }
     build_order_stage(H, nullptr, B, kind, L.item_bytes, head_off, L.req_bytes, order,
                       reinterpret_cast<int *>(at(L.off_stage)));
@@ -406,6 +428,7 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
     p->t.stage = reinterpret_cast<const int4 *>(dev + L.off_stage);
     p->t.status = reinterpret_cast<int *>(dev + L.off_status);
     p->n_pivot_items = n_pivot_items;
+    p->max_n16 = max_n16;
     p->nslots = nslots;
     p->slot_bytes = slot_bytes;
     p->off_q = off_q; p->off_k = off_k; p->off_v = off_v;
@@ -733,6 +756,7 @@ stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *states, siz
     int *t_head_bytes = reinterpret_cast<int *>(img + off_head_bytes);
     int *order = reinterpret_cast<int *>(img + off_order);
     int *stage = reinterpret_cast<int *>(img + off_stage);
+    int max_n16 = 0;
     for (int h = 0; h < H; h++) {
         stepq::HeadRec &R = rec[h];
         fill_rows(desc, h, R);
@@ -742,6 +766,7 @@ stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *states, siz
         R.slab_words = slab_words[h];
         t_head_off[h] = head_off[h];
         t_head_bytes[h] = (int)item_bytes[h];
+        if (kind[h] != stepq::kHeadAllPivot) max_n16 = std::max(max_n16, R.n16);
     }
     // item order: all-pivot heads' items first, then the others, heaviest
     // heads first; items of equal weight in item order
@@ -804,6 +829,7 @@ stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *states, siz
     a.off_q = off_q; a.off_k = off_k; a.off_v = off_v;
     a.off_alpha = off_alpha; a.off_ab = off_ab; a.off_rec = off_rec_slot;
     a.n_pivot_items = n_pivot_items;
+    a.max_n16 = max_n16;
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.out = out;
     e = stepq::launch_decode_step(a, s);
     return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "stepq_decode_step_noalloc launch");

@@ -83,72 +83,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 constexpr float kMagic = 8388608.0f;
 constexpr uint32_t kMagicBits = 0x4B000000u;
 
-// ---------------------------------------------------------------------------
-// packed stream codec for row-wise widths: a stream is a little-endian sequence
-// of fields (the fixed-width forms live with the kernels).
-// ---------------------------------------------------------------------------
-
-// Variable-width reader over stream words fetched on demand from shared memory
-// (word m of the stream at base[m * stride]).
-struct BitReader {
-    const uint32_t *base;
-    int stride;
-    int next;        // next word index
-    uint64_t buf;    // unread bits, LSB first
-    int nbits;       // number of unread bits in buf (0..63)
-    __device__ __forceinline__ void init(const uint32_t *b, int s)
-    {
-        base = b; stride = s; next = 0; buf = 0; nbits = 0;
-    }
-    // The next n (<= 32) bits.
-    __device__ __forceinline__ uint32_t take(int n)
-    {
-        if (nbits < n) {
-            buf |= (uint64_t)base[next * stride] << nbits;
-            nbits += 32;
-            next++;
-        }
-        const uint32_t v = (uint32_t)buf & (n == 32 ? 0xFFFFFFFFu : ((1u << n) - 1u));
-        buf >>= n;
-        nbits -= n;
-        return v;
-    }
-};
-
-// Variable-width writer emitting whole words to global memory (word m of the
-// stream at base[m * stride]); flush() writes the zero-padded last word.
-struct BitWriter {
-    uint32_t *base;
-    int stride;
-    int next;
-    uint64_t buf;
-    int nbits;
-    __device__ __forceinline__ void init(uint32_t *b, int s)
-    {
-        base = b; stride = s; next = 0; buf = 0; nbits = 0;
-    }
-    __device__ __forceinline__ void put(uint32_t v, int n)
-    {
-        buf |= (uint64_t)v << nbits;
-        nbits += n;
-        if (nbits >= 32) {
-            base[next * stride] = (uint32_t)buf;
-            next++;
-            buf >>= 32;
-            nbits -= 32;
-        }
-    }
-    __device__ __forceinline__ void flush()
-    {
-        if (nbits > 0) {
-            base[next * stride] = (uint32_t)buf;
-            next++;
-            buf = 0;
-            nbits = 0;
-        }
-    }
-};
-
 __device__ __forceinline__ int qmax_of(int b) { return (1 << (b - 1)) - 1; }
 
 }  // namespace dev

@@ -2,6 +2,7 @@
 // packed-state gated Delta-rule decode step.  Not part of the C ABI.
 #pragma once
 
+#include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -34,13 +35,20 @@ struct HeadRec {
     // sorted by width and dealt to the row groups in turn):
     uint8_t bits[kDK];           // row widths (16 = pivot)
     uint8_t key_row[kDK];        // the key row stored as this row
+    // field width of each row position p (storage rows 16 g + p): the widest
+    // row at that position over the row groups; every stream of the head
+    // lays out its fields alike.  Positions of 16-bit fields (pivot rows)
+    // come first: n16 of them.
+    uint8_t pos_bits[kRowsPerGroup];
     long long head_off;          // byte offset of the head's item inside a request
     int head_b;                  // common row width, 0 if the rows differ
     int head_kind;               // kHeadQuant / kHeadAllPivot / kHeadMixed
     int head_bytes;              // bytes of one item
     int slab_words;              // 32-bit words per stream (W)
-    int pad[2];
+    int n16;
+    int pad;
 };
+static_assert(offsetof(HeadRec, pos_bits) % 16 == 0, "pos_bits is read as one 16-byte vector");
 static_assert(sizeof(HeadRec) % 16 == 0, "head record must be a multiple of 16 bytes");
 
 // Per-head tables derived on the host at pool creation, resident in the tail
@@ -68,6 +76,7 @@ struct StepArgs {
     int slot_bytes;
     int off_q, off_k, off_v, off_alpha, off_ab, off_rec;  // offsets inside a slot
     int n_pivot_items;  // items of all-pivot heads, placed first in the order
+    int max_n16;        // the most leading 16-bit field positions of any other head
     const float *q, *k, *v, *alpha, *beta;
     float *out;
     const float *S_in;  // pack

@@ -105,9 +105,11 @@ struct alignas(16) RowFactors {
     float4 h2[64], w2[64];          // fit: h = a / r', w = rho r'^2
     float kqp[4];
     float ra[kDK];                  // a_i = alpha_i r_i (alpha_i on pivot rows), by row
-    int rb[kDK];                    // widths, by sslot
+    int rb[kDK];                    // widths, by sslot (row-wise widths only)
+    float qf[kDK];                  // Q_i as a float (0 on pivot rows), by sslot (row-wise widths only)
     float beta;
     int item, head_b;               // the item; its head's common width (0: row-wise)
+    int n16;                        // its head's leading positions of 16-bit fields
 };
 
 struct alignas(16) ItemSmem {
@@ -179,14 +181,14 @@ __device__ __forceinline__ float2 decode_pair(const uint32_t *wd, const uint32_t
 }
 
 // ---------------------------------------------------------------------------
-// Decode the thread's stream (word m at words[32 m]) into X: code values as
-// floats; pivot rows their binary16 values.  Fixed width B > 0 keeps the
-// stream in registers; B == 0 reads the row widths from rb_lane[8 rr].
+// Decode the thread's stream (word m at words[32 m]) of a head of one width B
+// into X (code values as floats), the stream kept in registers.
 // ---------------------------------------------------------------------------
 template <int B>
-__device__ __forceinline__ void decode_stream(const int *rb_lane, const uint32_t *words, X2 &X)
+__device__ __forceinline__ void decode_stream(const uint32_t *words, X2 &X)
 {
-    if constexpr (B > 0) {
+    static_assert(B > 0, "fixed widths only");
+    {
         uint32_t wd[2 * B + 1], hw[2 * B];
 #pragma unroll
         for (int m = 0; m < 2 * B; m++) wd[m] = words[m * kStreams];
@@ -197,30 +199,62 @@ __device__ __forceinline__ void decode_stream(const int *rb_lane, const uint32_t
         for (int rr = 0; rr < kRowsPerGroup; rr++)
 #pragma unroll
             for (int hh = 0; hh < 2; hh++) X[rr][hh] = decode_pair<B>(wd, hw, 4 * rr + 2 * hh);
-    } else {
-        BitReader br;
-        br.init(words, kStreams);
+    }
+}
+
+// The 16 position widths of a head, one byte each.
+__device__ __forceinline__ int pos_width(const uint4 &pb, int rr)
+{
+    const uint32_t w = (rr < 4) ? pb.x : (rr < 8) ? pb.y : (rr < 12) ? pb.z : pb.w;
+    return (int)((w >> (8 * (rr & 3))) & 0xFFu);
+}
+
+// ---------------------------------------------------------------------------
+// Decode for row-wise widths.  The 4 fields of row position rr lie at the same
+// bit offset O in every stream of the head, F = pos_bits[rr] bits each, so the
+// lanes of a warp decode in lockstep at warp-uniform offsets: the 32 bits from
+// O on (a funnel shift of two words), fields 0 and 1 in place and fields 2
+// and 3 from the bits shifted down by 2F, each as 2^(23 - e F) + u by the
+// exponent trick.  Positions of 16-bit fields (rows at a pivot row's
+// position) lead, word aligned; a pivot row's field is its binary16 value.
+// Only positions rr < NP are checked for them (NP = 1 when the head has at
+// most one such position).  rb_lane[8 rr] is the thread's row width at rr.
+// ---------------------------------------------------------------------------
+template <int NP>
+__device__ __forceinline__ void decode_rowwise(const int *rb_lane, const HeadRec *rec, const uint32_t *words, int W,
+                                               X2 &X)
+{
+    const uint4 pb = *reinterpret_cast<const uint4 *>(rec->pos_bits);
+    const int n16 = rec->n16;
+    int O = 0;
 #pragma unroll
-        for (int rr = 0; rr < kRowsPerGroup; rr++) {
-            const int b = rb_lane[8 * rr];
-            if (b == kPivotBits) {
-#pragma unroll
-                for (int hh = 0; hh < 2; hh++) {
-                    const uint32_t hv = br.take(32);
-                    X[rr][hh] = __half22float2(*reinterpret_cast<const __half2 *>(&hv));
-                }
+    for (int rr = 0; rr < kRowsPerGroup; rr++) {
+        const int F = pos_width(pb, rr);
+        const int m = O >> 5;
+        if (rr < NP && rr < n16) {
+            const uint32_t w0 = words[m * kStreams], w1 = words[(m + 1) * kStreams];
+            if (rb_lane[8 * rr] == kPivotBits) {
+                X[rr][0] = __half22float2(*reinterpret_cast<const __half2 *>(&w0));
+                X[rr][1] = __half22float2(*reinterpret_cast<const __half2 *>(&w1));
             } else {
-                const uint32_t f = br.take(4 * b);
-                const uint32_t mask = (1u << b) - 1u;
-                const float mz = -(kMagic + (float)(1 << (b - 1)));
-                const float2 mz2 = f2(mz, mz);
-#pragma unroll
-                for (int hh = 0; hh < 2; hh++) {
-                    const uint32_t u0 = ((f >> (2 * hh * b)) & mask) | kMagicBits;
-                    const uint32_t u1 = ((f >> ((2 * hh + 1) * b)) & mask) | kMagicBits;
-                    X[rr][hh] = __fadd2_rn(f2(__uint_as_float(u0), __uint_as_float(u1)), mz2);
-                }
+                const float2 sub = f2(-(kMagic + 32768.f), -(kMagic + 32768.f));
+                X[rr][0] = __fadd2_rn(
+                    f2(__uint_as_float((w0 & 0xFFFFu) | kMagicBits), __uint_as_float((w0 >> 16) | kMagicBits)), sub);
+                X[rr][1] = __fadd2_rn(
+                    f2(__uint_as_float((w1 & 0xFFFFu) | kMagicBits), __uint_as_float((w1 >> 16) | kMagicBits)), sub);
             }
+            O += 64;
+        } else {
+            const uint32_t w0 = words[m * kStreams], w1 = words[min(m + 1, W - 1) * kStreams];
+            const uint32_t f = __funnelshift_r(w0, w1, O & 31);
+            const uint32_t fh = f >> (2 * F);
+            const uint32_t m0 = (1u << F) - 1u, m1 = m0 << F;
+            const uint32_t e1 = (150u - (uint32_t)F) << 23;  // 2^(23 - F)
+            const float z = __uint_as_float((uint32_t)(126 + F) << 23);  // 2^(F - 1)
+            const float2 sub = f2(-(kMagic + z), -(__uint_as_float(e1) + z));
+            X[rr][0] = __fadd2_rn(f2(__uint_as_float((f & m0) | kMagicBits), __uint_as_float((f & m1) | e1)), sub);
+            X[rr][1] = __fadd2_rn(f2(__uint_as_float((fh & m0) | kMagicBits), __uint_as_float((fh & m1) | e1)), sub);
+            O += 4 * F;
         }
     }
 }
@@ -249,7 +283,7 @@ __device__ __forceinline__ float reduce_scatter_2x4(float2 A0, float2 A1, float2
 // warp's rows; then c_j = N_j / D_j (kept when D_j = 0), its reciprocal and
 // c0_j / c_j for the warp's 16 columns.
 // ---------------------------------------------------------------------------
-template <int B, bool ROWWISE, bool CLIP>
+template <int B, bool ROWWISE, bool CLIP, int NP>
 __device__ __forceinline__ void ls_round(ItemSmem &sm, const RowFactors &rf, const X2 &X)
 {
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31, rg = l & 7, cg = l >> 3;
@@ -265,13 +299,13 @@ __device__ __forceinline__ void ls_round(ItemSmem &sm, const RowFactors &rf, con
 #pragma unroll
         for (int u = 0; u < 2; u++) {
             const int rr = 2 * p + u;
-            if (ROWWISE && rf.rb[8 * rr + rg] == kPivotBits) continue;
+            if (ROWWISE && rr < NP && rr < rf.n16 && rf.rb[8 * rr + rg] == kPivotBits) continue;
             // round to the nearest integer, ties to even: x + 1.5 * 2^23 - 1.5 * 2^23;
             // clipping acts on the biased value
             float2 m0 = __ffma2_rn(X[rr][0], ic0, rm2);
             float2 m1 = __ffma2_rn(X[rr][1], ic1, rm2);
             if (CLIP) {
-                const float Q = (float)qmax_of(ROWWISE ? rf.rb[8 * rr + rg] : B);
+                const float Q = ROWWISE ? rf.qf[8 * rr + rg] : (float)qmax_of(B);
                 const float lo = kRoundMagic - Q, hi = kRoundMagic + Q;
                 m0 = f2(fminf(fmaxf(m0.x, lo), hi), fminf(fmaxf(m0.y, lo), hi));
                 m1 = f2(fminf(fmaxf(m1.x, lo), hi), fminf(fmaxf(m1.y, lo), hi));
@@ -355,6 +389,80 @@ __device__ __forceinline__ void pack_fixed(const X2 &X, float2 ic0, float2 ic1, 
         }
 }
 
+// Final codes and store for row-wise widths: the fields of row position rr go
+// to the head's common bit offset O in F = pos_bits[rr] bits (offset-binary
+// about 2^(F - 1)), the code clipped to the row's own range +-Q_i.  The four
+// fields of a position form one value f = sum_e y_e 2^(e F) minus the share of
+// the constant 0x4B000000 in it (y_e the float bits of 2^23 + u_e); f joins
+// the pending word at bit O % 32, and a word is stored as soon as it is
+// complete.  Clipping is decided per position with the widest range there,
+// which bounds every row's.  Leading positions of 16-bit fields store a pivot
+// row's binary16 values or the 16-bit codes of the rows beside it.
+template <int NP>
+__device__ __forceinline__ void pack_rowwise(const X2 &X, float2 ic0, float2 ic1, const RowFactors &rf,
+                                             const HeadRec *rec, float rat, int rg, uint32_t *words)
+{
+    const uint4 pb = *reinterpret_cast<const uint4 *>(rec->pos_bits);
+    const int n16 = rec->n16;
+    int O = 0;
+    uint32_t acc = 0u;  // the bits of word O / 32 below O % 32
+#pragma unroll
+    for (int rr = 0; rr < kRowsPerGroup; rr++) {
+        const int F = pos_width(pb, rr);
+        const int m = O >> 5;
+        if (rr < NP && rr < n16) {
+            uint32_t o0, o1;
+            if (rf.rb[8 * rr + rg] == kPivotBits) {
+                const __half2 h0 = __floats2half2_rn(X[rr][0].x, X[rr][0].y);
+                const __half2 h1 = __floats2half2_rn(X[rr][1].x, X[rr][1].y);
+                o0 = *reinterpret_cast<const uint32_t *>(&h0);
+                o1 = *reinterpret_cast<const uint32_t *>(&h1);
+            } else {
+                const float Q = rf.qf[8 * rr + rg];
+                const float2 mz2 = f2(kMagic + 32768.f, kMagic + 32768.f);
+                float2 t0 = __fmul2_rn(X[rr][0], ic0), t1 = __fmul2_rn(X[rr][1], ic1);
+                t0 = f2(fminf(fmaxf(t0.x, -Q), Q), fminf(fmaxf(t0.y, -Q), Q));
+                t1 = f2(fminf(fmaxf(t1.x, -Q), Q), fminf(fmaxf(t1.y, -Q), Q));
+                const float2 y0 = __fadd2_rn(t0, mz2), y1 = __fadd2_rn(t1, mz2);
+                o0 = (__float_as_uint(y0.x) & 0xFFFFu) | (__float_as_uint(y0.y) << 16);
+                o1 = (__float_as_uint(y1.x) & 0xFFFFu) | (__float_as_uint(y1.y) << 16);
+            }
+            words[m * kStreams] = o0;
+            words[(m + 1) * kStreams] = o1;
+            O += 64;
+        } else {
+            const float z = __uint_as_float((uint32_t)(126 + F) << 23);  // 2^(F - 1)
+            const float mz = kMagic + z;
+            const float2 mz2 = f2(mz, mz);
+            float2 y0, y1;
+            if ((z - 1.f) * (rat - 1.f) < 0.49f) {
+                y0 = __ffma2_rn(X[rr][0], ic0, mz2);
+                y1 = __ffma2_rn(X[rr][1], ic1, mz2);
+            } else {
+                const float Q = rf.qf[8 * rr + rg];
+                float2 t0 = __fmul2_rn(X[rr][0], ic0), t1 = __fmul2_rn(X[rr][1], ic1);
+                t0 = f2(fminf(fmaxf(t0.x, -Q), Q), fminf(fmaxf(t0.y, -Q), Q));
+                t1 = f2(fminf(fmaxf(t1.x, -Q), Q), fminf(fmaxf(t1.y, -Q), Q));
+                y0 = __fadd2_rn(t0, mz2);
+                y1 = __fadd2_rn(t1, mz2);
+            }
+            const uint32_t M1 = 1u << F, M2 = M1 << F, M3 = M2 << F;
+            uint32_t f = __float_as_uint(y0.x) - kMagicBits * (1u + M1 + M2 + M3);
+            f += __float_as_uint(y0.y) * M1;
+            f += __float_as_uint(y1.x) * M2;
+            f += __float_as_uint(y1.y) * M3;
+            const int sh = O & 31;
+            acc |= f << sh;
+            if (sh + 4 * F >= 32) {
+                words[m * kStreams] = acc;
+                acc = __funnelshift_l(f, 0u, sh);  // the bits of f beyond the word (none when sh = 0)
+            }
+            O += 4 * F;
+        }
+    }
+    if (O & 31) words[(O >> 5) * kStreams] = acc;
+}
+
 // Nothing to do between the two barriers of the fit (pack kernel).
 struct NoMid {
     __device__ __forceinline__ bool operator()() const { return true; }
@@ -377,7 +485,7 @@ enum FitResult { kFitDone = 0, kFitAbortNow = 1, kFitAbortAfter = 2 };
 // item is abandoned at barrier 1 with nothing stored (kFitAbortNow); if `mid`
 // fails on any thread the item is completed and kFitAbortAfter returned.
 // ---------------------------------------------------------------------------
-template <int B, bool ROWWISE, bool MULTI, class Mid>
+template <int B, bool ROWWISE, bool MULTI, int NP, class Mid>
 __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf, const HeadRec *rec, X2 &X,
                                                    uint8_t *item_g, int W, int ls_iters, bool store_c,
                                                    bool ok_in, const Mid &mid)
@@ -484,13 +592,13 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
     // the row's range.  More than one round is a separate instantiation (MULTI)
     // so that the one-round code holds a single round body.
     if (!MULTI) {
-        if (ls_iters > 0) ls_round<B, ROWWISE, false>(sm, rf, X);
+        if (ls_iters > 0) ls_round<B, ROWWISE, false, NP>(sm, rf, X);
     } else {
         for (int it = 0; it < ls_iters; it++) {
             if (it == 0)
-                ls_round<B, ROWWISE, false>(sm, rf, X);
+                ls_round<B, ROWWISE, false, NP>(sm, rf, X);
             else
-                ls_round<B, ROWWISE, true>(sm, rf, X);
+                ls_round<B, ROWWISE, true, NP>(sm, rf, X);
         }
     }
     // the column scales are final: store them before the codes
@@ -514,42 +622,7 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
         else
             pack_fixed<B, false>(X, ic0, ic1, words);
     } else {
-        BitWriter bw;
-        bw.init(words, kStreams);
-#pragma unroll
-        for (int rr = 0; rr < kRowsPerGroup; rr++) {
-            const int b = rf.rb[8 * rr + rg];
-            if (b == kPivotBits) {
-#pragma unroll
-                for (int hh = 0; hh < 2; hh++) {
-                    const __half2 hv = __floats2half2_rn(X[rr][hh].x, X[rr][hh].y);
-                    bw.put(*reinterpret_cast<const uint32_t *>(&hv), 32);
-                }
-            } else {
-                const int Qb = qmax_of(b);
-                const bool clip = (float)Qb * (rat - 1.f) >= 0.49f;
-                const float mz = kMagic + (float)(1 << (b - 1));
-                const float2 mz2 = f2(mz, mz);
-                const uint32_t mask = (1u << b) - 1u;
-                uint32_t f = 0;
-#pragma unroll
-                for (int hh = 0; hh < 2; hh++) {
-                    float2 mm;
-                    if (!clip) {
-                        mm = __ffma2_rn(X[rr][hh], hh ? ic1 : ic0, mz2);
-                    } else {
-                        float2 t = __fmul2_rn(X[rr][hh], hh ? ic1 : ic0);
-                        t = f2(fminf(fmaxf(t.x, -(float)Qb), (float)Qb), fminf(fmaxf(t.y, -(float)Qb), (float)Qb));
-                        mm = __fadd2_rn(t, mz2);
-                    }
-                    f |= (__float_as_uint(mm.x) & mask) << (2 * hh * b);
-                    f |= (__float_as_uint(mm.y) & mask) << ((2 * hh + 1) * b);
-                }
-                bw.put(f, 4 * b);
-            }
-        }
-        bw.flush();
-        for (int m = bw.next; m < W; m++) words[m * kStreams] = 0u;  // the stream's padding words
+        pack_rowwise<NP>(X, ic0, ic1, rf, rec, rat, rg, words);
     }
     return abort_after ? kFitAbortAfter : kFitDone;
 }
@@ -736,11 +809,15 @@ __device__ __forceinline__ void phase0(RowFactors &rf, const StepArgs &a, const 
         put_pair(rf.q2, i, rec->rq[i]);
     }
     rf.ra[i] = A;
-    if (KDA) rf.rb[sslot(i)] = b;
+    if (KDA) {
+        rf.rb[sslot(i)] = b;
+        rf.qf[sslot(i)] = (b == kPivotBits) ? 0.f : (float)qmax_of(b);
+    }
     if (i == 0) {
         rf.beta = beta;
         rf.item = item;
         rf.head_b = rec->head_b;
+        if (KDA) rf.n16 = rec->n16;
 
     }
 }
@@ -783,7 +860,7 @@ struct StageNext {
 // A staged item: reconstruct + project (phase A), read out, Delta update
 // (phase B), then the fit, during which the next item is prepared.  The slot
 // sb stays untouched until the fit's second barrier.
-template <int B, bool KDA, bool MULTI>
+template <int B, bool KDA, bool MULTI, int NP>
 __device__ __forceinline__ FitResult run_item(ItemSmem &sm, const StepArgs &a, RowFactors &rf, const uint8_t *sb,
                                               bool ok_slot, const StageNext<KDA> &next)
 {
@@ -795,7 +872,13 @@ __device__ __forceinline__ FitResult run_item(ItemSmem &sm, const StepArgs &a, R
     const int W = (B > 0) ? 2 * B : rec->slab_words;
     X2 X;
     // ---- phase A: codes -> floats, key and query projections, readout -------
-    decode_stream<B>(rf.rb + rg, reinterpret_cast<const uint32_t *>(sb + kHeaderBytes) + (kStreams * W) * w + l, X);
+    {
+        const uint32_t *words = reinterpret_cast<const uint32_t *>(sb + kHeaderBytes) + (kStreams * W) * w + l;
+        if constexpr (B > 0)
+            decode_stream<B>(words, X);
+        else
+            decode_rowwise<NP>(rf.rb + rg, rec, words, W, X);
+    }
     const float *s_c = reinterpret_cast<const float *>(sb) + kDK;
     const float4 c4 = ld4(s_c + col0);
     {
@@ -813,7 +896,7 @@ __device__ __forceinline__ FitResult run_item(ItemSmem &sm, const StepArgs &a, R
 #pragma unroll
             for (int u = 0; u < 2; u++) {
                 const int rr = 2 * p + u;
-                if (ROWWISE && rf.rb[8 * rr + rg] == kPivotBits) {
+                if (ROWWISE && rr < NP && rr < rf.n16 && rf.rb[8 * rr + rg] == kPivotBits) {
                     // a pivot value enters the projections in units of c_j; S' = alpha h
                     const float2 hs0 = __fmul2_rn(X[rr][0], ic0), hs1 = __fmul2_rn(X[rr][1], ic1);
                     V0 = __ffma2_rn(kp[u], hs0, V0);
@@ -867,7 +950,7 @@ __device__ __forceinline__ FitResult run_item(ItemSmem &sm, const StepArgs &a, R
 #pragma unroll
             for (int u = 0; u < 2; u++) {
                 const int rr = 2 * p + u;
-                if (ROWWISE && rf.rb[8 * rr + rg] == kPivotBits) {
+                if (ROWWISE && rr < NP && rr < rf.n16 && rf.rb[8 * rr + rg] == kPivotBits) {
                     X[rr][0] = __ffma2_rn(gp[u], dd0, X[rr][0]);
                     X[rr][1] = __ffma2_rn(gp[u], dd1, X[rr][1]);
                 } else {
@@ -879,7 +962,7 @@ __device__ __forceinline__ FitResult run_item(ItemSmem &sm, const StepArgs &a, R
     }
     const int rq = item / a.heads;
     uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + rec->head_off;
-    return fit_and_store<B, ROWWISE, MULTI>(sm, rf, rec, X, item_g, W, a.ls_iters, true, ok_slot, next);
+    return fit_and_store<B, ROWWISE, MULTI, NP>(sm, rf, rec, X, item_g, W, a.ls_iters, true, ok_slot, next);
 }
 
 // After a failed wait: record it, let every copy that may still be in flight
@@ -898,7 +981,9 @@ __device__ __forceinline__ void abort_drain(ItemSmem &sm, const StepArgs &a, uin
     __syncthreads();
 }
 
-template <bool KDA, bool MULTI>
+// NP (row-wise widths): the leading positions checked for 16-bit fields; 1
+// when no head of the pool has more than one, else all 16.
+template <bool KDA, bool MULTI, int NP>
 __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
 {
     extern __shared__ __align__(128) uint8_t ring[];
@@ -950,16 +1035,16 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
         const StageNext<KDA> next{sm, a, ring, n + G, slot_next, parity_next, sm.u.rf[par ^ 1]};
         FitResult res = kFitDone;
         if (KDA) {
-            res = run_item<0, KDA, MULTI>(sm, a, rf, sb, ok, next);
+            res = run_item<0, KDA, MULTI, NP>(sm, a, rf, sb, ok, next);
         } else {
             switch (rf.head_b) {
-                case 2: res = run_item<2, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
-                case 3: res = run_item<3, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
-                case 4: res = run_item<4, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
-                case 5: res = run_item<5, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
-                case 6: res = run_item<6, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
-                case 7: res = run_item<7, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
-                case 8: res = run_item<8, KDA, MULTI>(sm, a, rf, sb, ok, next); break;
+                case 2: res = run_item<2, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
+                case 3: res = run_item<3, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
+                case 4: res = run_item<4, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
+                case 5: res = run_item<5, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
+                case 6: res = run_item<6, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
+                case 7: res = run_item<7, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
+                case 8: res = run_item<8, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
                 default:  // unreachable: Gated-DeltaNet heads have one width, validated on the host
                     abort_drain(sm, a, n_cons, min(n_cons + nsl, n_stage), kStatusBadHead);
                     return;
@@ -995,7 +1080,9 @@ __device__ __forceinline__ void load_head(RowFactors &rf, const HeadRec *rec)
         const int i = tid;
         rf.ra[i] = 1.f;
         rf.rb[sslot(i)] = rec->bits[i];
+        rf.qf[sslot(i)] = (rec->bits[i] == kPivotBits) ? 0.f : (float)qmax_of(rec->bits[i]);
         put_pair(rf.q2, i, rec->rq[i]);
+        if (i == 0) rf.n16 = rec->n16;
     }
 }
 
@@ -1013,7 +1100,7 @@ __device__ __forceinline__ void pack_body(ItemSmem &sm, RowFactors &rf, const He
         X[rr][0] = f2(x.x, x.y);
         X[rr][1] = f2(x.z, x.w);
     }
-    fit_and_store<B, ROWWISE, true>(sm, rf, rec, X, item_g, (B > 0) ? 2 * B : rec->slab_words, a.ls_iters,
+    fit_and_store<B, ROWWISE, true, kRowsPerGroup>(sm, rf, rec, X, item_g, (B > 0) ? 2 * B : rec->slab_words, a.ls_iters,
                                     rec->head_kind != kHeadAllPivot, true, NoMid{});
 }
 
@@ -1047,7 +1134,13 @@ __device__ __forceinline__ void unpack_body(const RowFactors &rf, const HeadRec 
     const int col0 = 16 * w + 4 * cg;
     X2 X;
     const int W = (B > 0) ? 2 * B : rec->slab_words;
-    decode_stream<B>(rf.rb + rg, reinterpret_cast<const uint32_t *>(item_g + kHeaderBytes) + (kStreams * W) * w + l, X);
+    {
+        const uint32_t *words = reinterpret_cast<const uint32_t *>(item_g + kHeaderBytes) + (kStreams * W) * w + l;
+        if constexpr (B > 0)
+            decode_stream<B>(words, X);
+        else
+            decode_rowwise<kRowsPerGroup>(rf.rb + rg, rec, words, W, X);
+    }
     const float *r = reinterpret_cast<const float *>(item_g);
     const float4 c4 = ld4(r + kDK + col0);
     float *dst = a.S_out + (long long)item * kDK * kDV;
@@ -1104,7 +1197,13 @@ __device__ __forceinline__ void split_update_body(const RowFactors &rf, const He
     const int col0 = 16 * w + 4 * cg;
     const int W = (B > 0) ? 2 * B : rec->slab_words;
     X2 X;
-    decode_stream<B>(rf.rb + rg, reinterpret_cast<const uint32_t *>(item_g + kHeaderBytes) + (kStreams * W) * w + l, X);
+    {
+        const uint32_t *words = reinterpret_cast<const uint32_t *>(item_g + kHeaderBytes) + (kStreams * W) * w + l;
+        if constexpr (B > 0)
+            decode_stream<B>(words, X);
+        else
+            decode_rowwise<kRowsPerGroup>(rf.rb + rg, rec, words, W, X);
+    }
     const float *r = reinterpret_cast<const float *>(item_g);
     const float4 c4 = ld4(r + kDK + col0);
     const long long vec = (long long)item * kDK;
@@ -1269,20 +1368,27 @@ int sm_count()
     return g_sms;
 }
 
-template <bool KDA, bool MULTI>
+template <bool KDA, bool MULTI, int NP>
 cudaError_t launch_decode_t(const StepArgs &a, cudaStream_t s)
 {
     const int dyn = a.nslots * a.slot_bytes;
-    cudaError_t e = cudaFuncSetAttribute(k_decode<KDA, MULTI>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    cudaError_t e = cudaFuncSetAttribute(k_decode<KDA, MULTI, NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<KDA, MULTI>, kThreads, dyn);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<KDA, MULTI, NP>, kThreads, dyn);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const long long want = (long long)per_sm * sm_count();
     const int grid = (int)(a.n_items < want ? a.n_items : want);
-    k_decode<KDA, MULTI><<<grid, kThreads, dyn, s>>>(a);
+    k_decode<KDA, MULTI, NP><<<grid, kThreads, dyn, s>>>(a);
     return cudaGetLastError();
+}
+
+template <bool MULTI>
+cudaError_t launch_decode_m(const StepArgs &a, cudaStream_t s)
+{
+    if (!a.kda) return launch_decode_t<false, MULTI, 0>(a, s);
+    return (a.max_n16 <= 1) ? launch_decode_t<true, MULTI, 1>(a, s) : launch_decode_t<true, MULTI, kRowsPerGroup>(a, s);
 }
 
 }  // namespace
@@ -1290,16 +1396,15 @@ cudaError_t launch_decode_t(const StepArgs &a, cudaStream_t s)
 cudaError_t launch_decode_step(const StepArgs &a, cudaStream_t s)
 {
     if (a.n_items == 0) return cudaSuccess;
-    if (a.ls_iters <= 1) return a.kda ? launch_decode_t<true, false>(a, s) : launch_decode_t<false, false>(a, s);
-    return a.kda ? launch_decode_t<true, true>(a, s) : launch_decode_t<false, true>(a, s);
+    return (a.ls_iters <= 1) ? launch_decode_m<false>(a, s) : launch_decode_m<true>(a, s);
 }
 
 int decode_ctas_per_sm(int nslots, int slot_bytes)
 {
     const int dyn = nslots * slot_bytes;
     int per_sm = 0;
-    if (cudaFuncSetAttribute(k_decode<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<false, false>, kThreads, dyn) != cudaSuccess) {
+    if (cudaFuncSetAttribute(k_decode<false, false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<false, false, 0>, kThreads, dyn) != cudaSuccess) {
         cudaGetLastError();
         return 0;
     }

@@ -321,15 +321,21 @@ def storage_rows(bits_head: np.ndarray) -> np.ndarray:
     return key_of
 
 
+def position_widths(bits_head: np.ndarray) -> np.ndarray:
+    """F[p], p < 16: the field width of row position p (storage row 16 g + p of
+    every row group g), the widest row at that position over the groups."""
+    bits_head = np.asarray(bits_head)
+    dk = bits_head.shape[0]
+    sb = bits_head[storage_rows(bits_head)].astype(np.int64)
+    return sb.reshape(dk // GROUP_ROWS, GROUP_ROWS).max(axis=0)
+
+
 def stream_words(bits: np.ndarray) -> np.ndarray:
-    """32-bit words per stream of each head, [H]: the most any 16-row group of
-    storage rows needs for its 4 columns' fields."""
+    """32-bit words per stream of each head, [H]: ceil(4 sum_p F[p] / 32)."""
     H, dk = bits.shape
     out = np.zeros(H, dtype=np.int64)
     for h in range(H):
-        sb = bits[h][storage_rows(bits[h])].astype(np.int64)
-        per_group = sb.reshape(dk // GROUP_ROWS, GROUP_ROWS).sum(axis=1)
-        out[h] = ((GROUP_COLS * per_group + 31) // 32).max()
+        out[h] = (GROUP_COLS * int(position_widths(bits[h]).sum()) + 31) // 32
     return out
 
 

@@ -148,6 +148,24 @@ def test_every_width_and_pivot_rows_kda():
     lockstep(Setup(cfg, bits=bits), steps=4)
 
 
+def test_kda_position_layouts():
+    """Row-wise heads whose 16-bit field positions number at most one (the
+    kernel that checks only position 0 for pivots): mixed widths without
+    pivots, exactly 8 pivot rows (position 0 all pivots), one pivot row (a
+    16-bit position shared with 8-bit codes) and a single width."""
+    cfg = W.with_overrides(W.CONFIGS[2], batch=3, heads=4)
+    r = np.random.default_rng(1)
+    bits = np.empty((4, 128), np.uint8)
+    bits[0] = r.choice([3, 4, 5, 6, 7, 8], size=128)
+    bits[1] = r.choice([2, 5, 8], size=128)
+    bits[1, r.choice(128, 8, replace=False)] = 16
+    bits[2] = r.choice([4, 6], size=128)
+    bits[2, 77] = 16
+    bits[3] = 5
+    assert max(int(W.position_widths(b)[1]) for b in bits) < 16  # no head has a second 16-bit position
+    lockstep(Setup(cfg, bits=bits), steps=4)
+
+
 def perturbed_copy(ref, bits, heads, seed):
     """The oracle pool with one code of every item moved by one step: a rollout
     whose rounding noise is decorrelated from the original in every item."""

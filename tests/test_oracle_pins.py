@@ -347,8 +347,13 @@ def test_pack_format_slab_streams():
     key_of = [0] * dk
     for j, i in enumerate(ranked):
         key_of[16 * (j % 8) + j // 8] = i
-    # W: the most words any 16-row group needs for 4 columns' fields
-    Wh = max((4 * sum(int(bits[key_of[16 * g + t]]) for t in range(16)) + 31) // 32 for g in range(8))
+    # position p of every row group stores F_p-bit fields, F_p the widest row
+    # at that position; W = ceil(4 sum F_p / 32)
+    F = [max(int(bits[key_of[16 * g + t]]) for g in range(8)) for t in range(16)]
+    Wh = (4 * sum(F) + 31) // 32
+    # the deal puts the widest row of every position in group 0, so W is also
+    # the most words any group would need with fields of its rows' own widths
+    assert Wh == max((4 * sum(int(bits[key_of[16 * g + t]]) for t in range(16)) + 31) // 32 for g in range(8))
     assert item.size == 4 * dk + 4 * dv + 8 * 32 * 4 * Wh
     assert bytes(item[:4 * dk]) == rr[key_of].astype("<f4").tobytes()
     assert bytes(item[4 * dk: 4 * dk + 4 * dv]) == cc.astype("<f4").tobytes()
@@ -366,9 +371,9 @@ def test_pack_format_slab_streams():
                     if b == 16:
                         fields.append((int(np.array([piv[i, j]], "<f2").view("<u2")[0]), 16))
                     else:
-                        u = code[i, j] + (1 << (b - 1))
-                        assert 1 <= u <= (1 << b) - 1
-                        fields.append((u, b))
+                        u = code[i, j] + (1 << (F[rho_] - 1))
+                        assert 1 <= u <= (1 << F[rho_]) - 1
+                        fields.append((u, F[rho_]))
             assert list(slab[:, l]) == stream_words(fields, Wh), (s_, l)
     back = oracle.unpack_item(bits, item, dk, dv)
     np.testing.assert_array_equal(back["code"], code)
