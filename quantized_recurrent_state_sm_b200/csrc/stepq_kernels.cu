@@ -97,6 +97,18 @@ __device__ __forceinline__ float2 shfl2(float2 v, int m)
     return f2(__shfl_xor_sync(kFull, v.x, m), __shfl_xor_sync(kFull, v.y, m));
 }
 
+// Row position p of a row-wise head: where its fields sit in every stream and
+// the constants of their decode and pack, all derived from the field width F
+// and the bit offset O of the position (built once per item by 16 threads).
+struct alignas(16) PosRec {
+    int w0, w1, sh, f2;          // word offsets (x 32 streams) of words O/32 and O/32 + 1 (last word
+                                 // at most), O % 32, 2F
+    uint32_t m0, m1, e1, done;   // masks of fields 0 and 1, exponent bits of 2^(23 - F), whether
+                                 // the position ends a word
+    float s0, s1, mz, qf;        // -(2^23 + 2^(F-1)), -(2^(23-F) + 2^(F-1)), 2^23 + 2^(F-1), 2^(F-1) - 1
+    uint32_t M1, M2, M3, share;  // 2^F, 2^2F, 2^3F; the share of 0x4B000000 in sum_e y_e 2^(e F)
+};
+
 // Per-item factors, double-buffered by item parity: the factors of the next
 // item are written while the current item's fit still reads its own.
 struct alignas(16) RowFactors {
@@ -110,7 +122,40 @@ struct alignas(16) RowFactors {
     float beta;
     int item, head_b;               // the item; its head's common width (0: row-wise)
     int n16;                        // its head's leading positions of 16-bit fields
+    int tail_w;                     // row-wise: word offset of the last, partial word (-1: none)
+    PosRec pos[kRowsPerGroup];      // row-wise: the head's row positions
 };
+
+// Thread p < 16: position p of the head's table (row-wise widths).
+__device__ __forceinline__ void make_pos(RowFactors &rf, const HeadRec *rec, int p)
+{
+    int O = 0;
+    for (int q = 0; q < p; q++) O += 4 * rec->pos_bits[q];
+    const int F = rec->pos_bits[p], W = rec->slab_words, m = O >> 5, sh = O & 31;
+    PosRec r;
+    r.w0 = m * kStreams;
+    r.w1 = min(m + 1, W - 1) * kStreams;
+    r.sh = sh;
+    r.f2 = 2 * F;
+    r.m0 = (1u << F) - 1u;
+    r.m1 = r.m0 << F;
+    r.e1 = (150u - (uint32_t)F) << 23;
+    r.done = (sh + 4 * F >= 32) ? 1u : 0u;
+    const float z = (float)(1 << (F - 1));
+    r.s0 = -(kMagic + z);
+    r.s1 = -(__uint_as_float(r.e1) + z);
+    r.mz = kMagic + z;
+    r.qf = z - 1.f;
+    r.M1 = 1u << F;
+    r.M2 = r.M1 << F;
+    r.M3 = r.M2 << F;
+    r.share = kMagicBits * (1u + r.M1 + r.M2 + r.M3);
+    rf.pos[p] = r;
+    if (p == kRowsPerGroup - 1) {
+        const int end = O + 4 * F;
+        rf.tail_w = (end & 31) ? (end >> 5) * kStreams : -1;
+    }
+}
 
 struct alignas(16) ItemSmem {
     struct {
@@ -202,13 +247,6 @@ __device__ __forceinline__ void decode_stream(const uint32_t *words, X2 &X)
     }
 }
 
-// The 16 position widths of a head, one byte each.
-__device__ __forceinline__ int pos_width(const uint4 &pb, int rr)
-{
-    const uint32_t w = (rr < 4) ? pb.x : (rr < 8) ? pb.y : (rr < 12) ? pb.z : pb.w;
-    return (int)((w >> (8 * (rr & 3))) & 0xFFu);
-}
-
 // ---------------------------------------------------------------------------
 // Decode for row-wise widths.  The 4 fields of row position rr lie at the same
 // bit offset O in every stream of the head, F = pos_bits[rr] bits each, so the
@@ -218,22 +256,18 @@ __device__ __forceinline__ int pos_width(const uint4 &pb, int rr)
 // exponent trick.  Positions of 16-bit fields (rows at a pivot row's
 // position) lead, word aligned; a pivot row's field is its binary16 value.
 // Only positions rr < NP are checked for them (NP = 1 when the head has at
-// most one such position).  rb_lane[8 rr] is the thread's row width at rr.
+// most one such position).  rf.pos is the head's position table.
 // ---------------------------------------------------------------------------
 template <int NP>
-__device__ __forceinline__ void decode_rowwise(const int *rb_lane, const HeadRec *rec, const uint32_t *words, int W,
-                                               X2 &X)
+__device__ __forceinline__ void decode_rowwise(const RowFactors &rf, int rg, const uint32_t *words, X2 &X)
 {
-    const uint4 pb = *reinterpret_cast<const uint4 *>(rec->pos_bits);
-    const int n16 = rec->n16;
-    int O = 0;
+    const int n16 = rf.n16;
 #pragma unroll
     for (int rr = 0; rr < kRowsPerGroup; rr++) {
-        const int F = pos_width(pb, rr);
-        const int m = O >> 5;
+        const uint4 A = *reinterpret_cast<const uint4 *>(&rf.pos[rr].w0);
         if (rr < NP && rr < n16) {
-            const uint32_t w0 = words[m * kStreams], w1 = words[(m + 1) * kStreams];
-            if (rb_lane[8 * rr] == kPivotBits) {
+            const uint32_t w0 = words[A.x], w1 = words[A.y];
+            if (rf.rb[8 * rr + rg] == kPivotBits) {
                 X[rr][0] = __half22float2(*reinterpret_cast<const __half2 *>(&w0));
                 X[rr][1] = __half22float2(*reinterpret_cast<const __half2 *>(&w1));
             } else {
@@ -243,18 +277,13 @@ __device__ __forceinline__ void decode_rowwise(const int *rb_lane, const HeadRec
                 X[rr][1] = __fadd2_rn(
                     f2(__uint_as_float((w1 & 0xFFFFu) | kMagicBits), __uint_as_float((w1 >> 16) | kMagicBits)), sub);
             }
-            O += 64;
         } else {
-            const uint32_t w0 = words[m * kStreams], w1 = words[min(m + 1, W - 1) * kStreams];
-            const uint32_t f = __funnelshift_r(w0, w1, O & 31);
-            const uint32_t fh = f >> (2 * F);
-            const uint32_t m0 = (1u << F) - 1u, m1 = m0 << F;
-            const uint32_t e1 = (150u - (uint32_t)F) << 23;  // 2^(23 - F)
-            const float z = __uint_as_float((uint32_t)(126 + F) << 23);  // 2^(F - 1)
-            const float2 sub = f2(-(kMagic + z), -(__uint_as_float(e1) + z));
-            X[rr][0] = __fadd2_rn(f2(__uint_as_float((f & m0) | kMagicBits), __uint_as_float((f & m1) | e1)), sub);
-            X[rr][1] = __fadd2_rn(f2(__uint_as_float((fh & m0) | kMagicBits), __uint_as_float((fh & m1) | e1)), sub);
-            O += 4 * F;
+            const uint4 M = *reinterpret_cast<const uint4 *>(&rf.pos[rr].m0);
+            const float2 sub = *reinterpret_cast<const float2 *>(&rf.pos[rr].s0);
+            const uint32_t f = __funnelshift_r(words[A.x], words[A.y], A.z);
+            const uint32_t fh = f >> A.w;
+            X[rr][0] = __fadd2_rn(f2(__uint_as_float((f & M.x) | kMagicBits), __uint_as_float((f & M.y) | M.z)), sub);
+            X[rr][1] = __fadd2_rn(f2(__uint_as_float((fh & M.x) | kMagicBits), __uint_as_float((fh & M.y) | M.z)), sub);
         }
     }
 }
@@ -399,17 +428,14 @@ __device__ __forceinline__ void pack_fixed(const X2 &X, float2 ic0, float2 ic1, 
 // which bounds every row's.  Leading positions of 16-bit fields store a pivot
 // row's binary16 values or the 16-bit codes of the rows beside it.
 template <int NP>
-__device__ __forceinline__ void pack_rowwise(const X2 &X, float2 ic0, float2 ic1, const RowFactors &rf,
-                                             const HeadRec *rec, float rat, int rg, uint32_t *words)
+__device__ __forceinline__ void pack_rowwise(const X2 &X, float2 ic0, float2 ic1, const RowFactors &rf, float rat,
+                                             int rg, uint32_t *words)
 {
-    const uint4 pb = *reinterpret_cast<const uint4 *>(rec->pos_bits);
-    const int n16 = rec->n16;
-    int O = 0;
-    uint32_t acc = 0u;  // the bits of word O / 32 below O % 32
+    const int n16 = rf.n16;
+    uint32_t acc = 0u;  // the bits of the current word below the position's offset
 #pragma unroll
     for (int rr = 0; rr < kRowsPerGroup; rr++) {
-        const int F = pos_width(pb, rr);
-        const int m = O >> 5;
+        const uint4 A = *reinterpret_cast<const uint4 *>(&rf.pos[rr].w0);
         if (rr < NP && rr < n16) {
             uint32_t o0, o1;
             if (rf.rb[8 * rr + rg] == kPivotBits) {
@@ -427,15 +453,14 @@ __device__ __forceinline__ void pack_rowwise(const X2 &X, float2 ic0, float2 ic1
                 o0 = (__float_as_uint(y0.x) & 0xFFFFu) | (__float_as_uint(y0.y) << 16);
                 o1 = (__float_as_uint(y1.x) & 0xFFFFu) | (__float_as_uint(y1.y) << 16);
             }
-            words[m * kStreams] = o0;
-            words[(m + 1) * kStreams] = o1;
-            O += 64;
+            words[A.x] = o0;
+            words[A.y] = o1;
         } else {
-            const float z = __uint_as_float((uint32_t)(126 + F) << 23);  // 2^(F - 1)
-            const float mz = kMagic + z;
-            const float2 mz2 = f2(mz, mz);
+            const float2 zq = *reinterpret_cast<const float2 *>(&rf.pos[rr].mz);  // (2^23 + z, Q_F)
+            const uint4 M = *reinterpret_cast<const uint4 *>(&rf.pos[rr].M1);
+            const float2 mz2 = f2(zq.x, zq.x);
             float2 y0, y1;
-            if ((z - 1.f) * (rat - 1.f) < 0.49f) {
+            if (zq.y * (rat - 1.f) < 0.49f) {
                 y0 = __ffma2_rn(X[rr][0], ic0, mz2);
                 y1 = __ffma2_rn(X[rr][1], ic1, mz2);
             } else {
@@ -446,21 +471,18 @@ __device__ __forceinline__ void pack_rowwise(const X2 &X, float2 ic0, float2 ic1
                 y0 = __fadd2_rn(t0, mz2);
                 y1 = __fadd2_rn(t1, mz2);
             }
-            const uint32_t M1 = 1u << F, M2 = M1 << F, M3 = M2 << F;
-            uint32_t f = __float_as_uint(y0.x) - kMagicBits * (1u + M1 + M2 + M3);
-            f += __float_as_uint(y0.y) * M1;
-            f += __float_as_uint(y1.x) * M2;
-            f += __float_as_uint(y1.y) * M3;
-            const int sh = O & 31;
-            acc |= f << sh;
-            if (sh + 4 * F >= 32) {
-                words[m * kStreams] = acc;
-                acc = __funnelshift_l(f, 0u, sh);  // the bits of f beyond the word (none when sh = 0)
+            uint32_t f = __float_as_uint(y0.x) - M.w;
+            f += __float_as_uint(y0.y) * M.x;
+            f += __float_as_uint(y1.x) * M.y;
+            f += __float_as_uint(y1.y) * M.z;
+            acc |= f << A.z;
+            if (rf.pos[rr].done) {
+                words[A.x] = acc;
+                acc = __funnelshift_l(f, 0u, A.z);  // the bits of f beyond the word (none when O % 32 = 0)
             }
-            O += 4 * F;
         }
     }
-    if (O & 31) words[(O >> 5) * kStreams] = acc;
+    if (rf.tail_w >= 0) words[rf.tail_w] = acc;
 }
 
 // Nothing to do between the two barriers of the fit (pack kernel).
@@ -622,7 +644,7 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
         else
             pack_fixed<B, false>(X, ic0, ic1, words);
     } else {
-        pack_rowwise<NP>(X, ic0, ic1, rf, rec, rat, rg, words);
+        pack_rowwise<NP>(X, ic0, ic1, rf, rat, rg, words);
     }
     return abort_after ? kFitAbortAfter : kFitDone;
 }
@@ -812,6 +834,7 @@ __device__ __forceinline__ void phase0(RowFactors &rf, const StepArgs &a, const 
     if (KDA) {
         rf.rb[sslot(i)] = b;
         rf.qf[sslot(i)] = (b == kPivotBits) ? 0.f : (float)qmax_of(b);
+        if (i < kRowsPerGroup) make_pos(rf, rec, i);
     }
     if (i == 0) {
         rf.beta = beta;
@@ -877,7 +900,7 @@ __device__ __forceinline__ FitResult run_item(ItemSmem &sm, const StepArgs &a, R
         if constexpr (B > 0)
             decode_stream<B>(words, X);
         else
-            decode_rowwise<NP>(rf.rb + rg, rec, words, W, X);
+            decode_rowwise<NP>(rf, rg, words, X);
     }
     const float *s_c = reinterpret_cast<const float *>(sb) + kDK;
     const float4 c4 = ld4(s_c + col0);
@@ -1083,6 +1106,7 @@ __device__ __forceinline__ void load_head(RowFactors &rf, const HeadRec *rec)
         rf.qf[sslot(i)] = (rec->bits[i] == kPivotBits) ? 0.f : (float)qmax_of(rec->bits[i]);
         put_pair(rf.q2, i, rec->rq[i]);
         if (i == 0) rf.n16 = rec->n16;
+        if (i < kRowsPerGroup) make_pos(rf, rec, i);
     }
 }
 
@@ -1139,7 +1163,7 @@ __device__ __forceinline__ void unpack_body(const RowFactors &rf, const HeadRec 
         if constexpr (B > 0)
             decode_stream<B>(words, X);
         else
-            decode_rowwise<kRowsPerGroup>(rf.rb + rg, rec, words, W, X);
+            decode_rowwise<kRowsPerGroup>(rf, rg, words, X);
     }
     const float *r = reinterpret_cast<const float *>(item_g);
     const float4 c4 = ld4(r + kDK + col0);
@@ -1202,7 +1226,7 @@ __device__ __forceinline__ void split_update_body(const RowFactors &rf, const He
         if constexpr (B > 0)
             decode_stream<B>(words, X);
         else
-            decode_rowwise<kRowsPerGroup>(rf.rb + rg, rec, words, W, X);
+            decode_rowwise<kRowsPerGroup>(rf, rg, words, X);
     }
     const float *r = reinterpret_cast<const float *>(item_g);
     const float4 c4 = ld4(r + kDK + col0);
