@@ -50,6 +50,11 @@ def parse():
     p.add_argument("--config", type=int, default=CONFIG_INDEX)
     p.add_argument("--profile", action="store_true",
                    help="short run for ncu: no fp32-baseline, end-to-end or CPU legs")
+    p.add_argument("--calibrate", action="store_true",
+                   help="time the calibration that makes the config's tables instead of the decode step")
+    p.add_argument("--calib-batch", type=int, default=64)
+    p.add_argument("--calib-steps", type=int, default=32)
+    p.add_argument("--calib-every", type=int, default=8)
     return p.parse_args()
 
 
@@ -318,11 +323,89 @@ def run_split(args, cfg, pool, ring, out, stream, world):
     return {"ms_per_step": ms, "steps": n, "work_buffer_bytes": cfg.items * cfg.dk * cfg.dv * 4}
 
 
+def run_calibrate(args, cfg):
+    """The calibration of the config's tables on one GPU: stepq_calibrate over
+    a synthetic rollout of --calib-batch requests and --calib-steps steps
+    (states sampled every --calib-every steps), and its per-state kernel
+    (every candidate width fitted to every sampled state) timed alone.  The
+    oracle's per-state fit is timed on the host beside it."""
+    import torch
+    from quantized_recurrent_state_sm_b200 import stepq
+    import oracle
+    torch.cuda.set_device(0)
+    B, T, every, H = args.calib_batch, args.calib_steps, args.calib_every, cfg.heads
+    kda = cfg.variant == W.KDA
+    ch = sorted(cfg.bits_choices)
+    xs = [W.calibration_inputs(cfg, t, B) for t in range(T)]
+    dev = {k: torch.from_numpy(np.stack([x[k] for x in xs])).cuda() for k in xs[0]}
+    del xs
+    # initial state: the unquantised warm-up of the calibration requests on the GPU
+    S0 = torch.zeros((B, H, cfg.dk, cfg.dv), device="cuda")
+    req = W.calibration_requests(B)
+    for t in range(-cfg.warmup, 0):
+        x = {k: torch.from_numpy(v).cuda() for k, v in W.step_inputs(cfg, t, req).items()}
+        stepq.fp32_step(cfg.variant, S0, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    reps = max(1, min(args.steps, 5))
+    for i in range(max(1, min(args.warmup, 3))):
+        stepq.calibrate(cfg.variant, S0, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], ch,
+                        cfg.avg_bits, cfg.pivot_frac, every, cfg.ls_iters)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(reps):
+        rho, bits = stepq.calibrate(cfg.variant, S0, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], ch,
+                                    cfg.avg_bits, cfg.pivot_frac, every, cfg.ls_iters)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    calib_ms = ev[0].elapsed_time(ev[1]) / reps
+    # the per-state kernel alone on the initial states
+    rho_d = torch.from_numpy(rho).cuda()
+    n_rep = 20
+    stepq.calib_row_error(S0, rho_d, ch, cfg.ls_iters)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(n_rep):
+        stepq.calib_row_error(S0, rho_d, ch, cfg.ls_iters)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    k_ms = ev[0].elapsed_time(ev[1]) / n_rep
+    fits = B * H * len(ch)
+    # the oracle's fit of one state at every width, on the host
+    Sh = S0[0, 0].cpu().numpy()
+    t0 = time.perf_counter(); n_or = 0
+    while time.perf_counter() - t0 < min(args.cpu_seconds, 5.0):
+        for b in ch:
+            oracle.calib_row_error(Sh, b, rho[0], cfg.ls_iters)
+            n_or += 1
+    or_rate = n_or / (time.perf_counter() - t0)
+    line = {
+        "metric": "calibration: candidate-width fits of sampled fp32 states per second (k_calib_error)",
+        "value": fits / (k_ms * 1e-3), "unit": "state-width fits/s", "n_gpus": 1, "steps": reps,
+        "warmup": max(1, min(args.warmup, 3)), "ms_per_step": k_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"calibration of {workload_name(cfg)}", "calib_batch": B, "calib_steps": T,
+                   "sample_every": every, "widths": ch, "fits_per_launch": fits},
+        "calibrate_ms": calib_ms,
+        "calibrate_note": (f"stepq_calibrate end to end: {T} accumulate launches, {T} fp32 steps of {B * H} "
+                           f"states, {T // every} sampled error launches + reductions, host allocation"),
+        "cpu_baseline": {"value": or_rate, "unit": "state-width fits/s", "cores": 1, "kind": "oracle",
+                         "sample": f"one state, every width, for {min(args.cpu_seconds, 5.0):g} s"},
+        "bits_avg": float(bits.reshape(-1).astype(float).mean()),
+        "gpu_launches": n_rep,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     cfg = W.CONFIGS[args.config]
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.calibrate:
+        return run_calibrate(args, cfg)
 
     import torch
     import torch.distributed as dist

@@ -268,6 +268,96 @@ STEPQ_API stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *s
                                                  const float *alpha, const float *beta, float *out,
                                                  void *cuda_stream);
 
+/* ---- calibration: the offline step that makes a pool's tables ------------ *
+ * The pages fix a unit's width, once for all requests, from its quantisation
+ * distortion at candidate widths and its mean log retention under an average
+ * bit budget, keep the riskiest few units as FP16 pivots, and give every key
+ * row an impact score, the expected squared weight of its error in the
+ * readout (ai.info, "Methodology in Plain English" and "Key Contributions";
+ * ai-papers.net, "STEPQuantの仕組み"; ai-trend.me, "방법").  Units: heads
+ * (Gated-DeltaNet) or key rows (KDA).  This library's readings:
+ *   rho_i = mean over calibration requests and steps of q_i^2 (floored at
+ *   1e-30); lifetime weight w_u = 1 / (1 - abar_u^2) with abar_u =
+ *   exp(mean log alpha_u) (1 - abar^2 floored at 1e-12); distortion D_u(b) =
+ *   sum over sampled fp32 rollout states of sum_(rows i of u) rho_i
+ *   sum_j (S_ij - r_i c_j code_ij)^2, all rows of the head fitted at width b;
+ *   allocation: all units at the narrowest width, the ceil(pivot_frac * units)
+ *   units of largest w_u D_u(narrowest) made pivots (16 bits, in the budget),
+ *   then repeatedly the upgrade to the next candidate width with the largest
+ *   w_u (D_u(b) - D_u(b')) / (b' - b) > 0 that fits the remaining budget
+ *   round(avg_bits * units); ties go to the lower unit index.
+ * dk = dv = 128.  The piecewise calls below are what stepq_calibrate runs;
+ * they are exported for inspection and tests. */
+typedef struct {
+    int variant;        /* STEPQ_GDN or STEPQ_KDA */
+    int batch, heads, dk, dv;  /* calibration requests; dk = dv = 128 */
+    int steps;          /* rollout length T >= 1 */
+    int sample_every;   /* states sampled after steps t with (t + 1) % sample_every == 0 */
+    int ls_iters;       /* least-squares rounds of the fits (as the pool's) */
+    int n_widths;       /* 1 .. 8 candidate widths */
+    const int *widths;  /* host, strictly ascending, each in 2..8 */
+    double avg_bits;    /* average width budget per unit, pivots counted at 16 */
+    double pivot_frac;  /* share of units kept as FP16 pivots (ceil) */
+} stepq_calib_desc;
+
+/* Device scratch bytes stepq_calibrate needs for cd (0 if cd is invalid). */
+STEPQ_API size_t stepq_calib_scratch_bytes(const stepq_calib_desc *cd);
+
+/* The whole calibration, synchronous on cuda_stream (cudaStream_t or NULL):
+ * the impact scores from every step's q and the retention sums from every
+ * step's alpha; then the unquantised fp32 rollout from S0 (device,
+ * [batch][heads][dk][dv], not modified) over the same inputs, the per-row
+ * errors of every candidate width measured on the states after each sampled
+ * step; then the widths.  q, k: device [steps][batch][heads][dk]; v: device
+ * [steps][batch][heads][dv]; alpha: device [steps][batch][heads] (GDN) or
+ * [steps][batch][heads][dk] (KDA); beta: device [steps][batch][heads]; all
+ * fp32, 16-byte aligned (alpha and beta 4-byte for GDN).  scratch: device,
+ * at least stepq_calib_scratch_bytes, 256-byte aligned, caller-owned.
+ * Outputs (host): rho_out [heads*dk] and bits_out [heads*dk] (16 = pivot;
+ * every row of a Gated-DeltaNet head alike), ready for stepq_desc.
+ * STEPQ_ERR_INVALID_ARG when the pivots and the narrowest width alone exceed
+ * the budget. */
+STEPQ_API stepq_status stepq_calibrate(const stepq_calib_desc *cd, const float *S0, const float *q,
+                                       const float *k, const float *v, const float *alpha, const float *beta,
+                                       void *scratch, size_t scratch_bytes, void *cuda_stream, float *rho_out,
+                                       uint8_t *bits_out);
+
+/* One step's inputs into the running sums (asynchronous): acc_q2[h*dk+i] +=
+ * sum_b q[b][h][i]^2 and acc_loga[u] += sum_b log alpha[b][u] (u = h, or
+ * h*dk+i for KDA), in fp64, requests in order.  q: device [batch][heads][dk];
+ * alpha: device [batch][heads] (GDN) or [batch][heads][dk]; acc_q2: device
+ * fp64 [heads*dk]; acc_loga: device fp64 [heads] or [heads*dk]. */
+STEPQ_API stepq_status stepq_calib_accumulate(int variant, int batch, int heads, const float *q,
+                                              const float *alpha, double *acc_q2, double *acc_loga,
+                                              void *cuda_stream);
+
+/* Per-row squared errors of batch*heads fp32 states (asynchronous): state s
+ * = (request, head s % heads) fitted and quantised with every row at
+ * widths[x] (as stepq_pack would, rho = rho[head]) gives err[(s*n_widths +
+ * x)*dk + i] = r'_i^2 sum_j (p_ij - c_j code_ij)^2 (fp32) and its r' and c in
+ * rc[(s*n_widths + x)*(dk + dv) ..].  S: device [batch*heads][dk][dv]; rho:
+ * device [heads*dk]; widths: host, as in stepq_calib_desc; err, rc: device. */
+STEPQ_API stepq_status stepq_calib_row_error(int batch, int heads, const float *S, const float *rho,
+                                             int n_widths, const int *widths, int ls_iters, float *err,
+                                             float *rc, void *cuda_stream);
+
+/* err_sum[(h*n_widths + x)*dk + i] += err of request b, for b = 0, 1, ... in
+ * turn (fp64, asynchronous).  err: device, as written by
+ * stepq_calib_row_error; err_sum: device fp64 [heads][n_widths][dk]. */
+STEPQ_API stepq_status stepq_calib_reduce(int batch, int heads, int n_widths, const float *err,
+                                          double *err_sum, void *cuda_stream);
+
+/* Host: rho[u] = fp32(max(acc_q2[u] / n_samples, 1e-30)), u < heads*dk. */
+STEPQ_API stepq_status stepq_calib_rho(int heads, double n_samples, const double *acc_q2, float *rho);
+
+/* Host: the widths bits [heads*dk] from the sums (n_samples terms per unit in
+ * acc_loga; err_sum [heads][n_widths][dk]) and rho [heads*dk], by the
+ * allocation above.  STEPQ_ERR_INVALID_ARG when the budget is infeasible. */
+STEPQ_API stepq_status stepq_calib_bits(int variant, int heads, double n_samples, const double *acc_loga,
+                                        const float *rho, const double *err_sum, int n_widths,
+                                        const int *widths, double avg_bits, double pivot_frac,
+                                        uint8_t *bits);
+
 /* Human-readable name of a status; never NULL. */
 STEPQ_API const char *stepq_status_string(stepq_status s);
 

@@ -48,6 +48,15 @@ def lib():
         L.oracle_decode_step.argtypes = [i, P, i, i, P, P, i, i, P, P, P, P, P, P, P, P, P, P]
         L.oracle_fp32_step.argtypes = [i, i, i, i, P, P, P, P, P, P, P]
         L.oracle_fp64_step.argtypes = [i, i, i, i, P, P, P, P, P, P, P]
+        L.oracle_calib_accumulate.argtypes = [i, i, i, i, P, P, P, P]
+        L.oracle_calib_rho.argtypes = [i, i, C.c_double, P, P]
+        L.oracle_calib_row_error.argtypes = [i, i, P, i, P, i, P, P, P]
+        L.oracle_calib_weight.argtypes = [C.c_double]
+        L.oracle_calib_weight.restype = C.c_double
+        L.oracle_calib_allocate.argtypes = [i, P, P, i, P, C.c_double, i, P]
+        L.oracle_calib_allocate.restype = C.c_int
+        L.oracle_calib_bits.argtypes = [i, i, i, C.c_double, P, P, P, i, P, C.c_double, C.c_double, P]
+        L.oracle_calib_bits.restype = C.c_int
         _lib = L
     return _lib
 
@@ -240,3 +249,91 @@ def initial_state(cfg, requests=None, workload=None):
                   x["alpha"].reshape(R * H, -1) if cfg.variant == 1 else x["alpha"].reshape(-1),
                   x["beta"].reshape(-1), kda=cfg.variant == 1)
     return S.astype(np.float32).reshape(R, H, cfg.dk, cfg.dv)
+
+
+# ---- calibration (oracle/stepq_oracle_calib.c) -------------------------------
+
+def calib_accumulate(kda, q, alpha, acc_q2, acc_loga):
+    """Add one step's sums into acc_q2 [H, dk] and acc_loga ([H] or [H, dk]),
+    float64 arrays updated in place.  q [B, H, dk]; alpha [B, H] or [B, H, dk]."""
+    q = _c(q, np.float32); alpha = _c(alpha, np.float32)
+    B, H, dk = q.shape
+    assert acc_q2.dtype == np.float64 and acc_loga.dtype == np.float64
+    assert acc_q2.flags.c_contiguous and acc_loga.flags.c_contiguous
+    lib().oracle_calib_accumulate(int(kda), B, H, dk, _ptr(q), _ptr(alpha), _ptr(acc_q2), _ptr(acc_loga))
+
+
+def calib_rho(acc_q2, n_samples):
+    acc_q2 = _c(acc_q2, np.float64)
+    H, dk = acc_q2.shape
+    rho = np.zeros((H, dk), np.float32)
+    lib().oracle_calib_rho(H, dk, float(n_samples), _ptr(acc_q2), _ptr(rho))
+    return rho
+
+
+def calib_row_error(S, b, rho, ls_iters=1):
+    """(r, c, err) of S [dk, dv] stored with every row at width b."""
+    S = _c(S, np.float32); rho = _c(rho, np.float32)
+    dk, dv = S.shape
+    r = np.zeros(dk, np.float32); c = np.zeros(dv, np.float32); err = np.zeros(dk, np.float64)
+    lib().oracle_calib_row_error(dk, dv, _ptr(S), int(b), _ptr(rho), int(ls_iters), _ptr(r), _ptr(c), _ptr(err))
+    return r, c, err
+
+
+def calib_weight(mean_log_alpha):
+    return float(lib().oracle_calib_weight(float(mean_log_alpha)))
+
+
+def calib_allocate(weight, D, choices, avg_bits, n_piv):
+    weight = _c(weight, np.float64); D = _c(D, np.float64); ch = _c(choices, np.int32)
+    n, nc = D.shape
+    bits = np.zeros(n, np.uint8)
+    if lib().oracle_calib_allocate(n, _ptr(weight), _ptr(D), nc, _ptr(ch), float(avg_bits), int(n_piv), _ptr(bits)):
+        raise ValueError("bit budget below the pivots and the narrowest width")
+    return bits
+
+
+def calib_bits(kda, acc_loga, rho, err, choices, avg_bits, pivot_frac, n_samples):
+    """Row widths [H, dk] from the calibration sums; err [H, nc, dk]."""
+    rho = _c(rho, np.float32); err = _c(err, np.float64); acc_loga = _c(acc_loga, np.float64)
+    ch = _c(choices, np.int32)
+    H, nc, dk = err.shape
+    bits = np.zeros((H, dk), np.uint8)
+    if lib().oracle_calib_bits(int(kda), H, dk, float(n_samples), _ptr(acc_loga), _ptr(rho), _ptr(err), nc,
+                               _ptr(ch), float(avg_bits), float(pivot_frac), _ptr(bits)):
+        raise ValueError("bit budget below the pivots and the narrowest width")
+    return bits
+
+
+def calibrate(cfg, batch, steps, sample_every, workload=None):
+    """The whole calibration on the CPU: impact scores from the calibration
+    inputs, then per-row errors at every candidate width of the fp32 rollout's
+    states at steps t with (t + 1) % sample_every == 0 (after the step's
+    update), then the widths.  Returns dict rho [H, dk], bits [H, dk],
+    acc_q2, acc_loga, err [H, nc, dk]."""
+    if workload is None:
+        from quantized_recurrent_state_sm_b200 import workload
+    W = workload
+    kda = cfg.variant == 1
+    H, dk, dv = cfg.heads, cfg.dk, cfg.dv
+    choices = sorted(cfg.bits_choices)
+    acc_q2 = np.zeros((H, dk)); acc_loga = np.zeros((H, dk) if kda else (H,))
+    for t in range(steps):
+        x = W.calibration_inputs(cfg, t, batch)
+        calib_accumulate(kda, x["q"], x["alpha"], acc_q2, acc_loga)
+    n_samples = batch * steps
+    rho = calib_rho(acc_q2, n_samples)
+    S = initial_state(cfg, W.calibration_requests(batch), W).reshape(batch * H, dk, dv).copy()
+    err = np.zeros((H, len(choices), dk))
+    for t in range(steps):
+        x = W.calibration_inputs(cfg, t, batch)
+        n = batch * H
+        fp32_step(S, x["q"].reshape(n, dk), x["k"].reshape(n, dk), x["v"].reshape(n, dv),
+                  x["alpha"].reshape(n, dk) if kda else x["alpha"].reshape(n), x["beta"].reshape(n), kda=kda)
+        if (t + 1) % sample_every == 0:
+            for s in range(n):
+                h = s % H
+                for xw, b in enumerate(choices):
+                    err[h, xw] += calib_row_error(S[s], b, rho[h], cfg.ls_iters)[2]
+    bits = calib_bits(kda, acc_loga, rho, err, choices, cfg.avg_bits, cfg.pivot_frac, n_samples)
+    return {"rho": rho, "bits": bits, "acc_q2": acc_q2, "acc_loga": acc_loga, "err": err}

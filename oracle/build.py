@@ -5,7 +5,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB = os.path.join(HERE, "liboracle.so")
-SOURCES = ["stepq_oracle.c"]
+SOURCES = ["stepq_oracle.c", "stepq_oracle_calib.c"]
 DEPS = SOURCES + ["stepq_oracle.h", "stepq_oracle_core.inc"]
 
 

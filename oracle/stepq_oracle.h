@@ -147,6 +147,41 @@ void oracle_fp64_step(int n, int dk, int dv, int kda, double *S, const double *q
                       const double *k, const double *v, const double *alpha,
                       const double *beta, double *out);
 
+/* ---- calibration of the tables (stepq_oracle_calib.c) --------------------- *
+ * The offline step before the decode path: impact scores rho and row widths
+ * from a synthetic calibration rollout.  Units: heads (Gated-DeltaNet) or key
+ * rows (KDA). */
+#define ORACLE_CALIB_RHO_FLOOR 1e-30  /* rho of a row whose query weight is always 0 */
+#define ORACLE_CALIB_GAP_FLOOR 1e-12  /* 1 - abar^2 floor: a unit that never decays */
+
+/* One step's inputs into the running sums: acc_q2[h*dk+i] += sum_b q[b,h,i]^2
+ * (fp64, batch order); acc_loga[u] += sum_b log alpha[b,u], u = h for
+ * Gated-DeltaNet (alpha [batch*heads]) or h*dk+i for KDA (alpha
+ * [batch*heads*dk]).  q is [batch*heads*dk]. */
+void oracle_calib_accumulate(int kda, int batch, int heads, int dk, const float *q, const float *alpha,
+                             double *acc_q2, double *acc_loga);
+/* rho[u] = fp32(max(acc_q2[u] / n_samples, ORACLE_CALIB_RHO_FLOOR)), u < heads*dk. */
+void oracle_calib_rho(int heads, int dk, double n_samples, const double *acc_q2, float *rho);
+/* S [dk*dv] fitted and quantised with every row at width b (fp32 parity
+ * mode): r [dk], c [dv] and err[i] = sum_j (S_ij - r_i c_j code_ij)^2 in fp64. */
+void oracle_calib_row_error(int dk, int dv, const float *S, int b, const float *rho, int ls_iters, float *r,
+                            float *c, double *err);
+/* Lifetime weight 1 / (1 - exp(m)^2) of a unit with mean log retention m. */
+double oracle_calib_weight(double mean_log_alpha);
+/* Greedy lifetime-weighted allocation: D [n*nc] distortion of unit u at
+ * choices[x] (ascending); writes bits [n] (16 = pivot).  Returns -1 (bits
+ * still written, with no upgrade) when the pivots and the narrowest width
+ * alone exceed the budget round(avg_bits * n), else 0. */
+int oracle_calib_allocate(int n, const double *weight, const double *D, int nc, const int *choices,
+                          double avg_bits, int n_piv, uint8_t *bits);
+/* Widths of every row, bits [heads*dk], from the sums: weights from acc_loga
+ * (n_samples terms per unit), distortions from err [heads][nc][dk] (the
+ * per-row errors summed over the sampled states) weighted by rho [heads*dk];
+ * n_piv = ceil(pivot_frac * units).  Returns as oracle_calib_allocate. */
+int oracle_calib_bits(int kda, int heads, int dk, double n_samples, const double *acc_loga, const float *rho,
+                      const double *err, int nc, const int *choices, double avg_bits, double pivot_frac,
+                      uint8_t *bits);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,6 +8,7 @@
 #include <cstring>
 #include <mutex>
 #include <numeric>
+#include <queue>
 #include <set>
 #include <string>
 #include <vector>
@@ -653,6 +654,296 @@ stepq_status stepq_pool_check(stepq_pool *pool)
                                     "the affected items were not updated", code);
     }
     return STEPQ_OK;
+}
+
+// ---- calibration ----------------------------------------------------------
+
+namespace {
+
+constexpr double kRhoFloor = 1e-30;  // rho of a row whose query weight is always 0
+constexpr double kGapFloor = 1e-12;  // floor of 1 - abar^2 (a unit that never decays)
+
+stepq_status check_widths(int n_widths, const int *widths)
+{
+    if (n_widths < 1 || n_widths > stepq::kCalibMaxWidths)
+        return fail(STEPQ_ERR_INVALID_ARG, "n_widths %d outside 1..%d", n_widths, stepq::kCalibMaxWidths);
+    if (!widths) return fail(STEPQ_ERR_INVALID_ARG, "widths is NULL");
+    for (int x = 0; x < n_widths; x++) {
+        if (widths[x] < 2 || widths[x] > 8) return fail(STEPQ_ERR_INVALID_ARG, "width %d outside 2..8", widths[x]);
+        if (x > 0 && widths[x] <= widths[x - 1]) return fail(STEPQ_ERR_INVALID_ARG, "widths not ascending");
+    }
+    return STEPQ_OK;
+}
+
+stepq_status check_calib_desc(const stepq_calib_desc *cd)
+{
+    if (!cd) return fail(STEPQ_ERR_INVALID_ARG, "calibration descriptor is NULL");
+    if (cd->variant != STEPQ_GDN && cd->variant != STEPQ_KDA)
+        return fail(STEPQ_ERR_INVALID_ARG, "variant %d", cd->variant);
+    if (cd->dk != kDK || cd->dv != kDV) return fail(STEPQ_ERR_UNSUPPORTED, "dk = dv = 128 only");
+    if (cd->batch < 1 || cd->heads < 1 || (long long)cd->batch * cd->heads > (1LL << 24))
+        return fail(STEPQ_ERR_INVALID_ARG, "batch %d x heads %d", cd->batch, cd->heads);
+    if (cd->steps < 1 || cd->sample_every < 1 || cd->sample_every > cd->steps)
+        return fail(STEPQ_ERR_INVALID_ARG, "steps %d, sample_every %d: no state would be sampled", cd->steps,
+                    cd->sample_every);
+    if (cd->ls_iters < 0 || cd->ls_iters > 16) return fail(STEPQ_ERR_INVALID_ARG, "ls_iters %d", cd->ls_iters);
+    if (!(cd->avg_bits > 0.0 && cd->avg_bits <= 16.0)) return fail(STEPQ_ERR_INVALID_ARG, "avg_bits");
+    if (!(cd->pivot_frac >= 0.0 && cd->pivot_frac <= 1.0)) return fail(STEPQ_ERR_INVALID_ARG, "pivot_frac");
+    return check_widths(cd->n_widths, cd->widths);
+}
+
+struct CalibLayout {
+    size_t S, out, err, rc, acc_q2, acc_loga, err_sum, rho, total;
+};
+
+CalibLayout calib_layout(const stepq_calib_desc *cd)
+{
+    const size_t n = (size_t)cd->batch * cd->heads, H = (size_t)cd->heads, nW = (size_t)cd->n_widths;
+    CalibLayout L;
+    size_t o = 0;
+    L.S = o;        o = align_up(o + n * kDK * kDV * 4, 256);
+    L.out = o;      o = align_up(o + n * kDV * 4, 256);
+    L.err = o;      o = align_up(o + n * nW * kDK * 4, 256);
+    L.rc = o;       o = align_up(o + n * nW * (kDK + kDV) * 4, 256);
+    L.acc_q2 = o;   o = align_up(o + H * kDK * 8, 256);
+    L.acc_loga = o; o = align_up(o + H * kDK * 8, 256);
+    L.err_sum = o;  o = align_up(o + H * nW * kDK * 8, 256);
+    L.rho = o;      o = align_up(o + H * kDK * 4, 256);
+    L.total = o;
+    return L;
+}
+
+// Lifetime weight of a unit with mean log retention m.
+double lifetime_weight(double m)
+{
+    const double a = std::exp(m);
+    return 1.0 / std::max(1.0 - a * a, kGapFloor);
+}
+
+// The greedy allocation over n units (D: n x nc, by unit); false if the
+// pivots and the narrowest width alone exceed the budget.
+bool allocate_units(int n, const std::vector<double> &w, const std::vector<double> &D, int nc, const int *widths,
+                    double avg_bits, int n_piv, std::vector<uint8_t> &out)
+{
+    std::vector<int> level(n, 0);  // index into widths; -1: pivot
+    for (int p = 0; p < std::min(n_piv, n); p++) {
+        int pick = -1;
+        double top = 0.0;
+        for (int u = 0; u < n; u++) {
+            if (level[u] < 0) continue;
+            const double risk = w[u] * D[(size_t)u * nc];
+            if (pick < 0 || risk > top) {
+                pick = u;
+                top = risk;
+            }
+        }
+        level[pick] = -1;
+    }
+    long long spent = 0;
+    for (int u = 0; u < n; u++) spent += level[u] < 0 ? STEPQ_PIVOT_BITS : widths[0];
+    long long left = std::llround(avg_bits * n) - spent;
+    const bool feasible = left >= 0;
+    // upgrades by gain, largest first, ties to the lower unit: a unit's gain
+    // changes only when it is upgraded, and an upgrade that does not fit never
+    // fits later (the budget only shrinks), so a heap gives the picks of a
+    // scan over all units at every step
+    struct Up {
+        double gain;
+        int u;
+    };
+    auto below = [](const Up &a, const Up &b) { return a.gain < b.gain || (a.gain == b.gain && a.u > b.u); };
+    std::priority_queue<Up, std::vector<Up>, decltype(below)> heap(below);
+    auto offer = [&](int u) {
+        const int x = level[u];
+        if (x < 0 || x + 1 >= nc) return;
+        const int cost = widths[x + 1] - widths[x];
+        const double gain = w[u] * (D[(size_t)u * nc + x] - D[(size_t)u * nc + x + 1]) / cost;
+        if (gain > 0.0) heap.push({gain, u});
+    };
+    for (int u = 0; u < n; u++) offer(u);
+    while (!heap.empty() && left > 0) {
+        const int u = heap.top().u;
+        heap.pop();
+        const int cost = widths[level[u] + 1] - widths[level[u]];
+        if (cost > left) continue;
+        left -= cost;
+        level[u]++;
+        offer(u);
+    }
+    out.resize(n);
+    for (int u = 0; u < n; u++) out[u] = (uint8_t)(level[u] < 0 ? STEPQ_PIVOT_BITS : widths[level[u]]);
+    return feasible;
+}
+
+}  // namespace
+
+stepq_status stepq_calib_rho(int heads, double n_samples, const double *acc_q2, float *rho)
+{
+    if (heads < 1 || !acc_q2 || !rho || !(n_samples > 0.0))
+        return fail(STEPQ_ERR_INVALID_ARG, "stepq_calib_rho arguments");
+    for (long long u = 0; u < (long long)heads * kDK; u++)
+        rho[u] = (float)std::max(acc_q2[u] / n_samples, kRhoFloor);
+    return STEPQ_OK;
+}
+
+stepq_status stepq_calib_bits(int variant, int heads, double n_samples, const double *acc_loga, const float *rho,
+                              const double *err_sum, int n_widths, const int *widths, double avg_bits,
+                              double pivot_frac, uint8_t *bits)
+{
+    if ((variant != STEPQ_GDN && variant != STEPQ_KDA) || heads < 1 || !acc_loga || !rho || !err_sum || !bits ||
+        !(n_samples > 0.0) || !(avg_bits > 0.0) || !(pivot_frac >= 0.0 && pivot_frac <= 1.0))
+        return fail(STEPQ_ERR_INVALID_ARG, "stepq_calib_bits arguments");
+    stepq_status st = check_widths(n_widths, widths);
+    if (st != STEPQ_OK) return st;
+    const bool kda = variant == STEPQ_KDA;
+    const int n = kda ? heads * kDK : heads;
+    std::vector<double> w(n), D((size_t)n * n_widths);
+    for (int u = 0; u < n; u++) w[u] = lifetime_weight(acc_loga[u] / n_samples);
+    for (int h = 0; h < heads; h++)
+        for (int x = 0; x < n_widths; x++) {
+            const double *e = err_sum + ((size_t)h * n_widths + x) * kDK;
+            if (kda) {
+                for (int i = 0; i < kDK; i++) D[((size_t)h * kDK + i) * n_widths + x] = (double)rho[h * kDK + i] * e[i];
+            } else {
+                double acc = 0.0;
+                for (int i = 0; i < kDK; i++) acc += (double)rho[h * kDK + i] * e[i];
+                D[(size_t)h * n_widths + x] = acc;
+            }
+        }
+    const int n_piv = pivot_frac > 0.0 ? (int)std::ceil(pivot_frac * n - 1e-9) : 0;
+    std::vector<uint8_t> units;
+    const bool ok = allocate_units(n, w, D, n_widths, widths, avg_bits, n_piv, units);
+    for (int h = 0; h < heads; h++)
+        for (int i = 0; i < kDK; i++) bits[h * kDK + i] = kda ? units[h * kDK + i] : units[h];
+    if (!ok)
+        return fail(STEPQ_ERR_INVALID_ARG, "bit budget %.4f x %d below the pivots and the narrowest width",
+                    avg_bits, n);
+    return STEPQ_OK;
+}
+
+stepq_status stepq_calib_accumulate(int variant, int batch, int heads, const float *q, const float *alpha,
+                                    double *acc_q2, double *acc_loga, void *cuda_stream)
+{
+    if ((variant != STEPQ_GDN && variant != STEPQ_KDA) || batch < 0 || heads < 0)
+        return fail(STEPQ_ERR_INVALID_ARG, "stepq_calib_accumulate shape");
+    if (batch == 0 || heads == 0) return STEPQ_OK;
+    stepq_status st;
+    if ((st = check_dev(q, "q", 16)) != STEPQ_OK || (st = check_dev(alpha, "alpha", 4)) != STEPQ_OK ||
+        (st = check_dev(acc_q2, "acc_q2", 8)) != STEPQ_OK || (st = check_dev(acc_loga, "acc_loga", 8)) != STEPQ_OK)
+        return st;
+    stepq::CalibArgs c{};
+    c.batch = batch; c.heads = heads; c.kda = variant == STEPQ_KDA;
+    c.q = q; c.alpha = alpha; c.acc_q2 = acc_q2; c.acc_loga = acc_loga;
+    cudaError_t e = stepq::launch_calib_accumulate(c, reinterpret_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "stepq_calib_accumulate launch");
+}
+
+stepq_status stepq_calib_row_error(int batch, int heads, const float *S, const float *rho, int n_widths,
+                                   const int *widths, int ls_iters, float *err, float *rc, void *cuda_stream)
+{
+    if (batch < 0 || heads < 0 || (long long)batch * heads > (1LL << 24) || ls_iters < 0 || ls_iters > 16)
+        return fail(STEPQ_ERR_INVALID_ARG, "stepq_calib_row_error shape");
+    stepq_status st = check_widths(n_widths, widths);
+    if (st != STEPQ_OK) return st;
+    if (batch == 0 || heads == 0) return STEPQ_OK;
+    if ((st = check_dev(S, "S", 16)) != STEPQ_OK || (st = check_dev(rho, "rho", 4)) != STEPQ_OK ||
+        (st = check_dev(err, "err", 4)) != STEPQ_OK || (st = check_dev(rc, "rc", 4)) != STEPQ_OK)
+        return st;
+    stepq::CalibArgs c{};
+    c.batch = batch; c.heads = heads; c.n_widths = n_widths; c.ls_iters = ls_iters;
+    for (int x = 0; x < n_widths; x++) c.widths[x] = widths[x];
+    c.S = S; c.rho = rho; c.err = err; c.rc = rc;
+    cudaError_t e = stepq::launch_calib_error(c, reinterpret_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "stepq_calib_row_error launch");
+}
+
+stepq_status stepq_calib_reduce(int batch, int heads, int n_widths, const float *err, double *err_sum,
+                                void *cuda_stream)
+{
+    if (batch < 0 || heads < 0 || n_widths < 1 || n_widths > stepq::kCalibMaxWidths)
+        return fail(STEPQ_ERR_INVALID_ARG, "stepq_calib_reduce shape");
+    if (heads == 0) return STEPQ_OK;
+    stepq_status st;
+    if ((st = check_dev(err, "err", 4)) != STEPQ_OK || (st = check_dev(err_sum, "err_sum", 8)) != STEPQ_OK)
+        return st;
+    stepq::CalibArgs c{};
+    c.batch = batch; c.heads = heads; c.n_widths = n_widths; c.err = const_cast<float *>(err); c.err_sum = err_sum;
+    cudaError_t e = stepq::launch_calib_reduce(c, reinterpret_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "stepq_calib_reduce launch");
+}
+
+size_t stepq_calib_scratch_bytes(const stepq_calib_desc *cd)
+{
+    if (check_calib_desc(cd) != STEPQ_OK) return 0;
+    return calib_layout(cd).total;
+}
+
+stepq_status stepq_calibrate(const stepq_calib_desc *cd, const float *S0, const float *q, const float *k,
+                             const float *v, const float *alpha, const float *beta, void *scratch,
+                             size_t scratch_bytes, void *cuda_stream, float *rho_out, uint8_t *bits_out)
+{
+    stepq_status st = check_calib_desc(cd);
+    if (st != STEPQ_OK) return st;
+    if (!rho_out || !bits_out) return fail(STEPQ_ERR_INVALID_ARG, "rho_out / bits_out is NULL");
+    const CalibLayout L = calib_layout(cd);
+    if (scratch_bytes < L.total)
+        return fail(STEPQ_ERR_INVALID_ARG, "scratch of %zu bytes < %zu required", scratch_bytes, L.total);
+    const bool kda = cd->variant == STEPQ_KDA;
+    if ((st = check_dev(scratch, "scratch", 256)) != STEPQ_OK || (st = check_dev(S0, "S0", 16)) != STEPQ_OK ||
+        (st = check_dev(q, "q", 16)) != STEPQ_OK || (st = check_dev(k, "k", 16)) != STEPQ_OK ||
+        (st = check_dev(v, "v", 16)) != STEPQ_OK || (st = check_dev(alpha, "alpha", kda ? 16 : 4)) != STEPQ_OK ||
+        (st = check_dev(beta, "beta", 4)) != STEPQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(cuda_stream);
+    uint8_t *base = static_cast<uint8_t *>(scratch);
+    const int B = cd->batch, H = cd->heads, nW = cd->n_widths;
+    const size_t n = (size_t)B * H;
+    const size_t qstep = n * kDK, vstep = n * kDV, astep = kda ? n * kDK : n;
+    float *S = reinterpret_cast<float *>(base + L.S);
+    float *out = reinterpret_cast<float *>(base + L.out);
+    double *acc_q2 = reinterpret_cast<double *>(base + L.acc_q2);
+    double *acc_loga = reinterpret_cast<double *>(base + L.acc_loga);
+    double *err_sum = reinterpret_cast<double *>(base + L.err_sum);
+    float *rho_dev = reinterpret_cast<float *>(base + L.rho);
+    cudaError_t e = cudaSuccess;
+    auto cuda_ok = [&](cudaError_t r) { e = r; return r == cudaSuccess; };
+    // impact and retention sums over every step's inputs
+    if (!cuda_ok(cudaMemsetAsync(acc_q2, 0, (size_t)H * kDK * 8, s)) ||
+        !cuda_ok(cudaMemsetAsync(acc_loga, 0, (size_t)H * kDK * 8, s)))
+        return cuda_fail(e, "stepq_calibrate clear");
+    for (int t = 0; t < cd->steps; t++) {
+        st = stepq_calib_accumulate(cd->variant, B, H, q + t * qstep, alpha + t * astep, acc_q2, acc_loga, s);
+        if (st != STEPQ_OK) return st;
+    }
+    std::vector<double> h_q2((size_t)H * kDK), h_loga((size_t)H * kDK);
+    if (!cuda_ok(cudaMemcpyAsync(h_q2.data(), acc_q2, h_q2.size() * 8, cudaMemcpyDeviceToHost, s)) ||
+        !cuda_ok(cudaMemcpyAsync(h_loga.data(), acc_loga, h_loga.size() * 8, cudaMemcpyDeviceToHost, s)) ||
+        !cuda_ok(cudaStreamSynchronize(s)))
+        return cuda_fail(e, "stepq_calibrate read sums");
+    const double n_samples = (double)B * cd->steps;
+    if ((st = stepq_calib_rho(H, n_samples, h_q2.data(), rho_out)) != STEPQ_OK) return st;
+    // the rollout, its sampled states' errors at every candidate width
+    if (!cuda_ok(cudaMemcpyAsync(rho_dev, rho_out, (size_t)H * kDK * 4, cudaMemcpyHostToDevice, s)) ||
+        !cuda_ok(cudaMemcpyAsync(S, S0, n * kDK * kDV * 4, cudaMemcpyDeviceToDevice, s)) ||
+        !cuda_ok(cudaMemsetAsync(err_sum, 0, (size_t)H * nW * kDK * 8, s)))
+        return cuda_fail(e, "stepq_calibrate setup");
+    float *err = reinterpret_cast<float *>(base + L.err);
+    float *rc = reinterpret_cast<float *>(base + L.rc);
+    for (int t = 0; t < cd->steps; t++) {
+        if (!cuda_ok(stepq::launch_fp32_step(S, q + t * qstep, k + t * qstep, v + t * vstep, alpha + t * astep,
+                                             beta + t * n, out, (int)n, kda, s)))
+            return cuda_fail(e, "stepq_calibrate rollout");
+        if ((t + 1) % cd->sample_every != 0) continue;
+        if ((st = stepq_calib_row_error(B, H, S, rho_dev, nW, cd->widths, cd->ls_iters, err, rc, s)) != STEPQ_OK ||
+            (st = stepq_calib_reduce(B, H, nW, err, err_sum, s)) != STEPQ_OK)
+            return st;
+    }
+    std::vector<double> h_err((size_t)H * nW * kDK);
+    if (!cuda_ok(cudaMemcpyAsync(h_err.data(), err_sum, h_err.size() * 8, cudaMemcpyDeviceToHost, s)) ||
+        !cuda_ok(cudaStreamSynchronize(s)))
+        return cuda_fail(e, "stepq_calibrate read errors");
+    return stepq_calib_bits(cd->variant, H, n_samples, h_loga.data(), rho_out, h_err.data(), nW, cd->widths,
+                            cd->avg_bits, cd->pivot_frac, bits_out);
 }
 
 const char *stepq_status_string(stepq_status s)

@@ -93,6 +93,25 @@ cudaError_t launch_unpack(const StepArgs &a, cudaStream_t s);
 // The pages' split pipeline, first half: reconstruct, update, read out; the
 // updated unquantised state goes to a.S_in (a work buffer), for launch_pack.
 cudaError_t launch_split_update(const StepArgs &a, cudaStream_t s);
+// Calibration kernels (the offline step that makes a pool's tables).
+constexpr int kCalibMaxWidths = 8;
+struct CalibArgs {
+    int batch, heads, kda;
+    int n_widths;
+    int widths[kCalibMaxWidths];   // candidate widths, 2..8
+    int ls_iters;
+    const float *S;                // [batch*heads][dk][dv] fp32 states
+    const float *rho;              // [heads*dk] impact scores
+    float *err;                    // [batch*heads][n_widths][dk] per-row squared errors
+    float *rc;                     // [batch*heads][n_widths][dk + dv] fitted r', c
+    double *err_sum;               // [heads][n_widths][dk]
+    const float *q, *alpha;        // one step's inputs
+    double *acc_q2, *acc_loga;     // [heads*dk], [heads] or [heads*dk]
+};
+cudaError_t launch_calib_accumulate(const CalibArgs &c, cudaStream_t s);
+cudaError_t launch_calib_error(const CalibArgs &c, cudaStream_t s);
+cudaError_t launch_calib_reduce(const CalibArgs &c, cudaStream_t s);
+
 cudaError_t launch_fp32_step(float *S, const float *q, const float *k, const float *v,
                              const float *alpha, const float *beta, float *out, int n_items,
                              int kda, cudaStream_t s);

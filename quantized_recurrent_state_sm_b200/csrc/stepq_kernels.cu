@@ -485,6 +485,64 @@ __device__ __forceinline__ void pack_rowwise(const X2 &X, float2 ic0, float2 ic1
     if (rf.tail_w >= 0) words[rf.tail_w] = acc;
 }
 
+// The calibration's per-row error of a fixed width B: the codes the pack would
+// store (same clip decision), e = p - c code per element, the thread's row
+// partials of e^2 through the row-partial buffer, then row i (thread i):
+// r'_i^2 times the sum of its 32 partials.  r' is read back from the r[]
+// the fit wrote (by the same thread).
+template <int B>
+__device__ __forceinline__ void row_errors(ItemSmem &sm, const X2 &X, float2 ic0, float2 ic1, float rat,
+                                           const float *r_out, float *err_out)
+{
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31, rg = l & 7, cg = l >> 3;
+    const int col0 = 16 * w + 4 * cg;
+    constexpr int Qb = (1 << (B - 1)) - 1;
+    const bool clip = (float)Qb * (rat - 1.f) >= 0.49f;
+    const float4 c4 = ld4(&sm.cnew[col0]);
+    const float2 nc0 = f2(-c4.x, -c4.y), nc1 = f2(-c4.z, -c4.w);
+    const float2 rm2 = f2(kRoundMagic, kRoundMagic), nrm2 = f2(-kRoundMagic, -kRoundMagic);
+    float *T = &sm.rowp[(4 * w + cg) * kDK];
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+        float s[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const int rr = 4 * q + e;
+            float2 n0, n1;
+            if (!clip) {
+                n0 = __fadd2_rn(__ffma2_rn(X[rr][0], ic0, rm2), nrm2);
+                n1 = __fadd2_rn(__ffma2_rn(X[rr][1], ic1, rm2), nrm2);
+            } else {
+                float2 t0 = __fmul2_rn(X[rr][0], ic0), t1 = __fmul2_rn(X[rr][1], ic1);
+                t0 = f2(fminf(fmaxf(t0.x, -(float)Qb), (float)Qb), fminf(fmaxf(t0.y, -(float)Qb), (float)Qb));
+                t1 = f2(fminf(fmaxf(t1.x, -(float)Qb), (float)Qb), fminf(fmaxf(t1.y, -(float)Qb), (float)Qb));
+                n0 = __fadd2_rn(__fadd2_rn(t0, rm2), nrm2);
+                n1 = __fadd2_rn(__fadd2_rn(t1, rm2), nrm2);
+            }
+            const float2 e0 = __ffma2_rn(nc0, n0, X[rr][0]), e1 = __ffma2_rn(nc1, n1, X[rr][1]);
+            float2 s2 = __fmul2_rn(e0, e0);
+            s2 = __ffma2_rn(e1, e1, s2);
+            s[e] = s2.x + s2.y;
+        }
+        *reinterpret_cast<float4 *>(T + rowp_chunk(rg, q)) = make_float4(s[0], s[1], s[2], s[3]);
+    }
+    __syncthreads();
+    if (tid < kDK) {
+        const int i = tid, irg = i >> 4, irr = i & 15;
+        const float *src = &sm.rowp[rowp_chunk(irg, irr >> 2) + (irr & 3)];
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+        for (int bk = 0; bk < 32; bk += 4) {
+            s0 += src[(bk + 0) * kDK];
+            s1 += src[(bk + 1) * kDK];
+            s2 += src[(bk + 2) * kDK];
+            s3 += src[(bk + 3) * kDK];
+        }
+        const float rp = r_out[i];
+        err_out[i] = (rp * rp) * ((s0 + s1) + (s2 + s3));
+    }
+}
+
 // Nothing to do between the two barriers of the fit (pack kernel).
 struct NoMid {
     __device__ __forceinline__ bool operator()() const { return true; }
@@ -507,10 +565,13 @@ enum FitResult { kFitDone = 0, kFitAbortNow = 1, kFitAbortAfter = 2 };
 // item is abandoned at barrier 1 with nothing stored (kFitAbortNow); if `mid`
 // fails on any thread the item is completed and kFitAbortAfter returned.
 // ---------------------------------------------------------------------------
-template <int B, bool ROWWISE, bool MULTI, int NP, class Mid>
+// ERR (fixed widths; calibration): instead of packing, the squared
+// reconstruction error of every row, r'^2 sum_j (p_ij - c_j code_ij)^2 with the
+// codes the pack would store, goes to err_out[row] (item_g receives r' and c).
+template <int B, bool ROWWISE, bool MULTI, int NP, class Mid, bool ERR = false>
 __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf, const HeadRec *rec, X2 &X,
                                                    uint8_t *item_g, int W, int ls_iters, bool store_c,
-                                                   bool ok_in, const Mid &mid)
+                                                   bool ok_in, const Mid &mid, float *err_out = nullptr)
 {
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31, rg = l & 7, cg = l >> 3;
     const int col0 = 16 * w + 4 * cg;
@@ -636,6 +697,11 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
     // the largest |p / c| of a column is at most Q c0 / c: clip only where that
     // can reach Q + 1/2 (decided per warp)
     rat = __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(rat)));
+    if constexpr (ERR) {
+        static_assert(B > 0 && !ROWWISE, "the error mode fits one width");
+        row_errors<B>(sm, X, ic0, ic1, rat, reinterpret_cast<const float *>(item_g), err_out);
+        return kFitDone;
+    }
     uint32_t *words = reinterpret_cast<uint32_t *>(item_g + kHeaderBytes) + (kStreams * W) * w + l;
     if constexpr (B > 0) {
         constexpr int Qb = (1 << (B - 1)) - 1;
@@ -1415,7 +1481,132 @@ cudaError_t launch_decode_m(const StepArgs &a, cudaStream_t s)
     return (a.max_n16 <= 1) ? launch_decode_t<true, MULTI, 1>(a, s) : launch_decode_t<true, MULTI, kRowsPerGroup>(a, s);
 }
 
+// ---------------------------------------------------------------------------
+// Calibration.  k_calib_accumulate: one step's sums of q^2 per (head, key row)
+// and of log alpha per unit, over the batch in request order (fp64; one CTA
+// per head, thread i = key row).  k_calib_error: one CTA per (request, head)
+// state; for every candidate width the state is fitted and quantised with all
+// rows at that width, as the pack kernel would, and each row's squared
+// reconstruction error is written.  k_calib_reduce: the errors of a sampled
+// state added into the running fp64 sums, request by request.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kDK) k_calib_accumulate(CalibArgs c)
+{
+    const int h = blockIdx.x, i = threadIdx.x, H = c.heads;
+    double s = 0.0;
+    for (int b = 0; b < c.batch; b++) {
+        const double x = (double)c.q[((long long)b * H + h) * kDK + i];
+        s += x * x;
+    }
+    c.acc_q2[h * kDK + i] += s;
+    if (c.kda) {
+        double t = 0.0;
+        for (int b = 0; b < c.batch; b++) t += log((double)c.alpha[((long long)b * H + h) * kDK + i]);
+        c.acc_loga[h * kDK + i] += t;
+    } else if (i == 0) {
+        double t = 0.0;
+        for (int b = 0; b < c.batch; b++) t += log((double)c.alpha[(long long)b * H + h]);
+        c.acc_loga[h] += t;
+    }
+}
+
+template <int B, bool MULTI>
+__device__ __forceinline__ void calib_width(ItemSmem &sm, RowFactors &rf, const HeadRec *rec, const CalibArgs &c,
+                                            int item, int x)
+{
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31, rg = l & 7, cg = l >> 3;
+    const int col0 = 16 * w + 4 * cg;
+    X2 X;
+    const float *src = c.S + (long long)item * kDK * kDV;
+#pragma unroll
+    for (int rr = 0; rr < kRowsPerGroup; rr++) {
+        const float4 v = ld4(src + (kRowsPerGroup * rg + rr) * kDV + col0);
+        X[rr][0] = f2(v.x, v.y);
+        X[rr][1] = f2(v.z, v.w);
+    }
+    const long long o = (long long)item * c.n_widths + x;
+    fit_and_store<B, false, MULTI, 0, NoMid, true>(sm, rf, rec, X,
+                                                  reinterpret_cast<uint8_t *>(c.rc + o * (kDK + kDV)), 2 * B,
+                                                  c.ls_iters, true, true, NoMid{}, c.err + o * kDK);
+}
+
+template <bool MULTI>
+__global__ void __launch_bounds__(kThreads) k_calib_error(CalibArgs c)
+{
+    __shared__ ItemSmem sm;
+    __shared__ HeadRec rec;
+    RowFactors &rf = sm.u.rf[0];
+    const int item = blockIdx.x, h = item % c.heads, tid = threadIdx.x;
+    float s_i = 0.f, rho_i = 0.f;
+    if (tid < kDK) {
+        rho_i = c.rho[h * kDK + tid];
+        s_i = (float)(1.0 / sqrt((double)rho_i));  // fp32(rho^-1/2) from fp64, as the host tables
+    }
+    for (int x = 0; x < c.n_widths; x++) {
+        const int b = c.widths[x];
+        __syncthreads();  // the previous width's readers of rec, rf and the row partials are done
+        if (tid < kDK) {
+            const int i = tid;
+            rec.s[i] = s_i;
+            rec.rho[i] = rho_i;
+            rec.rq[i] = (float)(1.0 / (double)qmax_of(b));
+            rec.bits[i] = (uint8_t)b;
+            rec.key_row[i] = (uint8_t)i;
+            rf.ra[i] = 1.f;
+        }
+        if (tid == 0) {
+            rec.head_b = b;
+            rec.head_kind = kHeadQuant;
+            rec.n16 = 0;
+        }
+        __syncthreads();
+        switch (b) {
+            case 2: calib_width<2, MULTI>(sm, rf, &rec, c, item, x); break;
+            case 3: calib_width<3, MULTI>(sm, rf, &rec, c, item, x); break;
+            case 4: calib_width<4, MULTI>(sm, rf, &rec, c, item, x); break;
+            case 5: calib_width<5, MULTI>(sm, rf, &rec, c, item, x); break;
+            case 6: calib_width<6, MULTI>(sm, rf, &rec, c, item, x); break;
+            case 7: calib_width<7, MULTI>(sm, rf, &rec, c, item, x); break;
+            default: calib_width<8, MULTI>(sm, rf, &rec, c, item, x); break;  // widths are validated on the host
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kDK) k_calib_reduce(CalibArgs c)
+{
+    const int h = blockIdx.x / c.n_widths, x = blockIdx.x % c.n_widths, i = threadIdx.x;
+    double acc = c.err_sum[((long long)h * c.n_widths + x) * kDK + i];
+    for (int b = 0; b < c.batch; b++)
+        acc += (double)c.err[(((long long)b * c.heads + h) * c.n_widths + x) * kDK + i];
+    c.err_sum[((long long)h * c.n_widths + x) * kDK + i] = acc;
+}
+
 }  // namespace
+
+cudaError_t launch_calib_accumulate(const CalibArgs &c, cudaStream_t s)
+{
+    if (c.heads == 0 || c.batch == 0) return cudaSuccess;
+    k_calib_accumulate<<<c.heads, kDK, 0, s>>>(c);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_calib_error(const CalibArgs &c, cudaStream_t s)
+{
+    const long long n = (long long)c.batch * c.heads;
+    if (n == 0 || c.n_widths == 0) return cudaSuccess;
+    if (c.ls_iters <= 1)
+        k_calib_error<false><<<(unsigned)n, kThreads, 0, s>>>(c);
+    else
+        k_calib_error<true><<<(unsigned)n, kThreads, 0, s>>>(c);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_calib_reduce(const CalibArgs &c, cudaStream_t s)
+{
+    if (c.heads == 0 || c.n_widths == 0) return cudaSuccess;
+    k_calib_reduce<<<c.heads * c.n_widths, kDK, 0, s>>>(c);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_decode_step(const StepArgs &a, cudaStream_t s)
 {

@@ -35,10 +35,19 @@ class Desc(C.Structure):
                 ("dv", C.c_int), ("ls_iters", C.c_int), ("bits", C.c_void_p), ("rho", C.c_void_p)]
 
 
+class CalibDesc(C.Structure):
+    _fields_ = [("variant", C.c_int), ("batch", C.c_int), ("heads", C.c_int), ("dk", C.c_int),
+                ("dv", C.c_int), ("steps", C.c_int), ("sample_every", C.c_int), ("ls_iters", C.c_int),
+                ("n_widths", C.c_int), ("widths", C.c_void_p), ("avg_bits", C.c_double),
+                ("pivot_frac", C.c_double)]
+
+
 EXPORTS = ("stepq_pool_bytes", "stepq_state_bytes", "stepq_pool_create", "stepq_pool_destroy",
            "stepq_pool_set_stream", "stepq_pack", "stepq_unpack", "stepq_decode_step",
            "stepq_fp32_step", "stepq_pool_check", "stepq_status_string", "stepq_last_error",
-           "stepq_decode_step_noalloc", "stepq_decode_step_split", "stepq_pool_set_active")
+           "stepq_decode_step_noalloc", "stepq_decode_step_split", "stepq_pool_set_active",
+           "stepq_calib_scratch_bytes", "stepq_calibrate", "stepq_calib_accumulate", "stepq_calib_row_error",
+           "stepq_calib_reduce", "stepq_calib_rho", "stepq_calib_bits")
 
 
 def _load():
@@ -60,9 +69,18 @@ def _load():
     L.stepq_decode_step_noalloc.argtypes = [D, P, C.c_size_t, P, P, P, P, P, P, P]
     L.stepq_decode_step_split.argtypes = [P, P, P, P, P, P, P, P, P]
     L.stepq_pool_set_active.argtypes = [P, P, C.c_int]
+    CD, i, dbl = C.POINTER(CalibDesc), C.c_int, C.c_double
+    L.stepq_calib_scratch_bytes.argtypes = [CD]; L.stepq_calib_scratch_bytes.restype = C.c_size_t
+    L.stepq_calibrate.argtypes = [CD, P, P, P, P, P, P, P, C.c_size_t, P, P, P]
+    L.stepq_calib_accumulate.argtypes = [i, i, i, P, P, P, P, P]
+    L.stepq_calib_row_error.argtypes = [i, i, P, P, i, P, i, P, P, P]
+    L.stepq_calib_reduce.argtypes = [i, i, i, P, P, P]
+    L.stepq_calib_rho.argtypes = [i, dbl, P, P]
+    L.stepq_calib_bits.argtypes = [i, i, dbl, P, P, P, i, P, dbl, dbl, P]
     for fn in ("stepq_pool_create", "stepq_pool_destroy", "stepq_pool_set_stream", "stepq_pool_check", "stepq_pack",
                "stepq_unpack", "stepq_decode_step", "stepq_fp32_step", "stepq_decode_step_noalloc",
-               "stepq_decode_step_split", "stepq_pool_set_active"):
+               "stepq_decode_step_split", "stepq_pool_set_active", "stepq_calibrate", "stepq_calib_accumulate",
+               "stepq_calib_row_error", "stepq_calib_reduce", "stepq_calib_rho", "stepq_calib_bits"):
         getattr(L, fn).restype = C.c_int
     L.stepq_status_string.argtypes = [C.c_int]; L.stepq_status_string.restype = C.c_char_p
     L.stepq_last_error.argtypes = []; L.stepq_last_error.restype = C.c_char_p
@@ -260,3 +278,97 @@ def decode_step_noalloc(variant: int, bits, rho, states: torch.Tensor, q, k, v, 
                                          _dev(beta, "beta", (B, H)), _dev(out, "out", (B, H, DV)),
                                          _stream_ptr()))
     return out
+
+
+# ---- calibration -------------------------------------------------------------
+
+def _dev_any(t: torch.Tensor, name: str, dtype, shape) -> C.c_void_p:
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_cuda:
+        raise TypeError(f"{name} must be a {dtype} CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return C.c_void_p(t.data_ptr())
+
+
+def _host(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data_as(C.c_void_p)
+
+
+def calibrate(variant: int, S0: torch.Tensor, q, k, v, alpha, beta, widths, avg_bits: float,
+              pivot_frac: float, sample_every: int, ls_iters: int = 1):
+    """The library's calibration (stepq_calibrate): S0 [B, H, 128, 128] and the
+    rollout's inputs q, k [T, B, H, 128], v [T, B, H, 128], alpha [T, B, H] or
+    [T, B, H, 128], beta [T, B, H], all float32 CUDA tensors.  Returns
+    (rho [H, 128] float32, bits [H, 128] uint8) as numpy arrays."""
+    T, B, H = q.shape[0], q.shape[1], q.shape[2]
+    w, wp = _host(widths, np.int32)
+    cd = CalibDesc(variant, B, H, DK, DV, T, int(sample_every), int(ls_iters), int(w.size), wp,
+                   float(avg_bits), float(pivot_frac))
+    nbytes = lib.stepq_calib_scratch_bytes(C.byref(cd))
+    if nbytes == 0:
+        _check(ERR_INVALID_ARG)
+    scratch = torch.empty(nbytes, dtype=torch.uint8, device=S0.device)
+    rho = np.zeros((H, DK), np.float32); bits = np.zeros((H, DK), np.uint8)
+    ash = (T, B, H, DK) if variant == KDA else (T, B, H)
+    _check(lib.stepq_calibrate(C.byref(cd), _dev(S0, "S0", (B, H, DK, DV)), _dev(q, "q", (T, B, H, DK)),
+                               _dev(k, "k", (T, B, H, DK)), _dev(v, "v", (T, B, H, DV)), _dev(alpha, "alpha", ash),
+                               _dev(beta, "beta", (T, B, H)), C.c_void_p(scratch.data_ptr()), nbytes,
+                               _stream_ptr(), rho.ctypes.data_as(C.c_void_p), bits.ctypes.data_as(C.c_void_p)))
+    return rho, bits
+
+
+def calib_accumulate(variant: int, q: torch.Tensor, alpha: torch.Tensor, acc_q2: torch.Tensor,
+                     acc_loga: torch.Tensor):
+    """One step's q [B, H, 128] and alpha into the float64 CUDA sums acc_q2
+    [H, 128] and acc_loga ([H] or [H, 128])."""
+    B, H = q.shape[0], q.shape[1]
+    ash = (B, H, DK) if variant == KDA else (B, H)
+    _check(lib.stepq_calib_accumulate(variant, B, H, _dev(q, "q", (B, H, DK)), _dev(alpha, "alpha", ash),
+                                      _dev_any(acc_q2, "acc_q2", torch.float64, (H, DK)),
+                                      _dev_any(acc_loga, "acc_loga", torch.float64, (H, DK) if variant == KDA else (H,)),
+                                      _stream_ptr()))
+
+
+def calib_row_error(S: torch.Tensor, rho: torch.Tensor, widths, ls_iters: int = 1):
+    """Per-row squared errors of the states S [B, H, 128, 128] stored at each of
+    `widths`: returns (err [B, H, nW, 128], rc [B, H, nW, 256]) float32 CUDA tensors."""
+    B, H = S.shape[0], S.shape[1]
+    w, wp = _host(widths, np.int32)
+    err = torch.empty((B, H, w.size, DK), dtype=torch.float32, device=S.device)
+    rc = torch.empty((B, H, w.size, DK + DV), dtype=torch.float32, device=S.device)
+    _check(lib.stepq_calib_row_error(B, H, _dev(S, "S", (B, H, DK, DV)), _dev(rho, "rho", (H, DK)), int(w.size), wp,
+                                     int(ls_iters), C.c_void_p(err.data_ptr()), C.c_void_p(rc.data_ptr()),
+                                     _stream_ptr()))
+    return err, rc
+
+
+def calib_reduce(err: torch.Tensor, err_sum: torch.Tensor):
+    """err_sum [H, nW, 128] (float64 CUDA) += err [B, H, nW, 128], request by request."""
+    B, H, nW = err.shape[0], err.shape[1], err.shape[2]
+    _check(lib.stepq_calib_reduce(B, H, nW, _dev(err, "err", (B, H, nW, DK)),
+                                  _dev_any(err_sum, "err_sum", torch.float64, (H, nW, DK)), _stream_ptr()))
+
+
+def calib_rho(acc_q2: np.ndarray, n_samples: float) -> np.ndarray:
+    """Host: impact scores [H, 128] from the sums of q^2."""
+    a, ap = _host(acc_q2, np.float64)
+    H = a.shape[0]
+    rho = np.zeros((H, DK), np.float32)
+    _check(lib.stepq_calib_rho(H, float(n_samples), ap, rho.ctypes.data_as(C.c_void_p)))
+    return rho
+
+
+def calib_bits(variant: int, acc_loga, rho, err_sum, widths, avg_bits, pivot_frac, n_samples) -> np.ndarray:
+    """Host: the row widths [H, 128] from the calibration sums (err_sum [H, nW, 128])."""
+    la, lap = _host(acc_loga, np.float64)
+    r, rp = _host(rho, np.float32)
+    e, ep = _host(err_sum, np.float64)
+    w, wp = _host(widths, np.int32)
+    H = e.shape[0]
+    bits = np.zeros((H, DK), np.uint8)
+    _check(lib.stepq_calib_bits(variant, H, float(n_samples), lap, rp, ep, int(w.size), wp, float(avg_bits),
+                                float(pivot_frac), bits.ctypes.data_as(C.c_void_p)))
+    return bits

@@ -47,6 +47,7 @@ PIVOT_BITS = 16  # a pivot unit stores every value as an IEEE binary16 number
 # stream identifiers for the counter-based generator
 S_Q, S_K, S_V, S_BETA = 1, 2, 3, 4
 S_GATE, S_RHO, S_OUT_K, S_OUT_V = 5, 6, 7, 8
+S_Q_GAIN = 9
 
 GDN, KDA = 0, 1
 
@@ -108,6 +109,7 @@ class Config:
     outlier_frac: float = 0.0
     outlier_gain: float = 1.0
     ls_iters: int = 1
+    q_gain_sigma: float = 0.0  # per (head, key row) query gains ~ LogNormal(0, sigma) (0: none)
 
     @property
     def input_seed(self) -> int:
@@ -240,6 +242,17 @@ def bit_table(cfg: Config) -> np.ndarray:
     return out.astype(np.uint8)
 
 
+def query_gains(cfg: Config) -> np.ndarray:
+    """Per (head, key row) query gains, float64 [H, dk], applied before the
+    normalisation of q: ones when cfg.q_gain_sigma is 0, else LogNormal(0, sigma),
+    so that key rows weigh differently in the readout."""
+    if cfg.q_gain_sigma <= 0:
+        return np.ones((cfg.heads, cfg.dk))
+    key = derive_key(cfg.table_seed, S_Q_GAIN)
+    z = normal(key, np.arange(cfg.heads * cfg.dk))
+    return np.exp(cfg.q_gain_sigma * z).reshape(cfg.heads, cfg.dk)
+
+
 def outlier_gains(cfg: Config):
     """(k_gain [H, dk], v_gain [H, dv]) float64; ones when the config has no outliers."""
     kg = np.ones((cfg.heads, cfg.dk))
@@ -279,6 +292,8 @@ def step_inputs(cfg: Config, t: int, requests=None):
     k = field(S_K, cfg.dk) * kg[None]
     k = k / np.linalg.norm(k, axis=-1, keepdims=True)
     q = field(S_Q, cfg.dk)
+    if cfg.q_gain_sigma > 0:
+        q = q * query_gains(cfg)[None]
     q = q / np.linalg.norm(q, axis=-1, keepdims=True)
     v = field(S_V, cfg.dv) * vg[None]
     zb = normal(derive_key(cfg.input_seed, S_BETA, bb, hh, t), np.zeros_like(bb))
@@ -289,6 +304,21 @@ def step_inputs(cfg: Config, t: int, requests=None):
         "q": q.astype(np.float32), "k": k.astype(np.float32), "v": v.astype(np.float32),
         "beta": beta.astype(np.float32), "alpha": np.ascontiguousarray(alpha, dtype=np.float32),
     }
+
+
+# Calibration rollouts: requests and steps of their own (counter ranges no
+# serving step or request uses), the same generators otherwise.
+CALIB_REQUEST0 = 1 << 20
+CALIB_STEP0 = 1 << 20
+
+
+def calibration_requests(batch: int) -> np.ndarray:
+    return CALIB_REQUEST0 + np.arange(batch)
+
+
+def calibration_inputs(cfg: Config, tau: int, batch: int):
+    """Inputs of calibration step tau (0, 1, ...) for `batch` calibration requests."""
+    return step_inputs(cfg, CALIB_STEP0 + tau, calibration_requests(batch))
 
 
 def parity_requests(cfg: Config):
