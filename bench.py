@@ -52,6 +52,9 @@ def parse():
                    help="short run for ncu: no fp32-baseline, end-to-end or CPU legs")
     p.add_argument("--calibrate", action="store_true",
                    help="time the calibration that makes the config's tables instead of the decode step")
+    p.add_argument("--ablations", action="store_true",
+                   help="error structure of the method and its ablation variants over synthetic rollouts")
+    p.add_argument("--ablation-steps", type=int, default=256)
     p.add_argument("--calib-batch", type=int, default=64)
     p.add_argument("--calib-steps", type=int, default=32)
     p.add_argument("--calib-every", type=int, default=8)
@@ -399,6 +402,118 @@ def run_calibrate(args, cfg):
     return 0
 
 
+def _ranks(x):
+    r = np.empty(len(x)); r[np.argsort(x, kind="stable")] = np.arange(len(x))
+    return r
+
+
+def spearman(a, b):
+    return float(np.corrcoef(_ranks(np.asarray(a)), _ranks(np.asarray(b)))[0, 1])
+
+
+def run_ablations(args, cfg):
+    """Rollouts of --ablation-steps decode steps from the same initial state,
+    for the method and its ablation variants, beside the unquantised fp32
+    recursion on the same inputs: readout and state errors per variant, and
+    the pages' error-structure measures (accumulated state error against
+    half-life under a uniform width with one scale per state; the error share
+    of the longest-lived quarter of units; row and column RMS contrasts of
+    the fp32 states).  The method's tables come from stepq_calibrate on a
+    calibration rollout (its own requests and steps); the stand-in tables
+    (LogNormal impact weights) are run as a row of their own.  Synthetic
+    inputs throughout."""
+    import torch
+    from quantized_recurrent_state_sm_b200 import stepq
+    torch.cuda.set_device(0)
+    B, H, T = cfg.batch, cfg.heads, args.ablation_steps
+    kda = cfg.variant == W.KDA
+    u_bits = int(round(cfg.avg_bits))
+    cfg_u = W.with_overrides(cfg, bits_choices=(u_bits,), pivot_frac=0.0)
+    # the calibrated tables
+    Bc, Tc, every = 16, 32, 8
+    xs = [W.calibration_inputs(cfg, t, Bc) for t in range(Tc)]
+    cdev = {k: torch.from_numpy(np.stack([x[k] for x in xs])).cuda() for k in xs[0]}
+    Sc = torch.zeros((Bc, H, cfg.dk, cfg.dv), device="cuda")
+    for t in range(-cfg.warmup, 0):
+        x = {k: torch.from_numpy(v).cuda() for k, v in W.step_inputs(cfg, t, W.calibration_requests(Bc)).items()}
+        stepq.fp32_step(cfg.variant, Sc, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+    rho_c, bits_c = stepq.calibrate(cfg.variant, Sc, cdev["q"], cdev["k"], cdev["v"], cdev["alpha"], cdev["beta"],
+                                    sorted(cfg.bits_choices), cfg.avg_bits, cfg.pivot_frac, every, cfg.ls_iters)
+    rho_u, _ = stepq.calibrate(cfg.variant, Sc, cdev["q"], cdev["k"], cdev["v"], cdev["alpha"], cdev["beta"],
+                               [u_bits], float(u_bits), 0.0, every, cfg.ls_iters)
+    del cdev, Sc
+    bits_u = W.bit_table(cfg_u)
+    ones = np.ones_like(rho_c)
+    variants = [
+        ("method, calibrated tables (lifetime widths, dual-axis fit, impact weights)", bits_c, rho_c, stepq.SCALE_DUAL),
+        ("method, stand-in tables (lifetime widths, LogNormal impact weights)", W.bit_table(cfg), W.rho(cfg),
+         stepq.SCALE_DUAL),
+        (f"spatial only (uniform {u_bits}-bit, dual-axis fit, calibrated impact weights)", bits_u, rho_u,
+         stepq.SCALE_DUAL),
+        ("temporal only (calibrated widths, one scale per state)", bits_c, rho_c, stepq.SCALE_HEAD),
+        (f"uniform {u_bits}-bit, one scale per state", bits_u, rho_u, stepq.SCALE_HEAD),
+        ("row scales only (calibrated widths)", bits_c, rho_c, stepq.SCALE_ROW),
+        ("column scales only (calibrated widths)", bits_c, rho_c, stepq.SCALE_COL),
+        ("no impact weights (calibrated widths, rho = 1)", bits_c, ones, stepq.SCALE_DUAL),
+    ]
+    ring = [{k: torch.from_numpy(v).cuda() for k, v in W.step_inputs(cfg, t).items()} for t in range(-cfg.warmup, T)]
+    S0 = torch.zeros((B, H, cfg.dk, cfg.dv), device="cuda")
+    for t in range(cfg.warmup):
+        d = ring[t]
+        stepq.fp32_step(cfg.variant, S0, d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+    Sf = S0.clone()
+    of = []
+    for t in range(T):
+        d = ring[cfg.warmup + t]
+        of.append(stepq.fp32_step(cfg.variant, Sf, d["q"], d["k"], d["v"], d["alpha"], d["beta"]).clone())
+    torch.cuda.synchronize()
+    hl = W.half_lives(cfg)  # [H] (GDN) or [H, dk] (KDA)
+    rows = []
+    structure = {}
+    for name, bits, rh, mode in variants:
+        pool = stepq.PackedStatePool(cfg.variant, B, H, bits, rh, cfg.ls_iters)
+        pool.set_scale_mode(mode)
+        pool.pack(S0)
+        o_err = []
+        for t in range(T):
+            d = ring[cfg.warmup + t]
+            o = pool.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+            if t >= T - 64:
+                o_err.append(float(torch.linalg.vector_norm(o - of[t]) / torch.linalg.vector_norm(of[t])))
+        Sq = pool.unpack()
+        pool.check()
+        diff2 = (Sq - Sf).double() ** 2
+        ref2 = Sf.double() ** 2
+        state_rel = float(torch.sqrt(diff2.sum() / ref2.sum()))
+        rows.append({"variant": name, "readout_rel_l2_last64": float(np.mean(o_err)), "state_rel_l2": state_rel,
+                     "avg_bits": float(bits.astype(float).mean())})
+        if name.startswith(f"uniform {u_bits}-bit"):
+            # accumulated squared state error per unit, summed over requests and value columns
+            dims = (0, 3) if kda else (0, 2, 3)
+            e_unit = diff2.sum(dim=dims).cpu().numpy().reshape(-1)
+            h = hl.reshape(-1)
+            top = np.argsort(-h, kind="stable")[: max(1, h.size // 4)]
+            structure["uniform_width"] = u_bits
+            structure["spearman_accumulated_error_vs_half_life"] = spearman(np.sqrt(e_unit), h)
+            structure["error_share_longest_quarter"] = float(e_unit[top].sum() / e_unit.sum())
+        del pool
+        torch.cuda.empty_cache()
+    # row / column RMS contrasts of the final fp32 states
+    S2 = Sf.double() ** 2
+    row_rms = torch.sqrt(S2.mean(dim=3)); col_rms = torch.sqrt(S2.mean(dim=2))   # [B, H, 128]
+    rc = (row_rms.max(dim=2).values / row_rms.median(dim=2).values).cpu().numpy().reshape(-1)
+    cc = (col_rms.max(dim=2).values / col_rms.median(dim=2).values).cpu().numpy().reshape(-1)
+    structure.update({"row_rms_contrast_median": float(np.median(rc)), "col_rms_contrast_median": float(np.median(cc)),
+                      "share_both_contrasts_above_3": float(np.mean((rc > 3) & (cc > 3))),
+                      "calibrated_rho_max_over_min_median_head": float(np.median(rho_c.max(axis=1) / rho_c.min(axis=1)))})
+    line = {"metric": "ablations: readout and state error vs the unquantised fp32 recursion",
+            "config": {"workload": workload_name(cfg), "steps": T, "unit": "head" if not kda else "key row",
+                       "calibration": {"batch": Bc, "steps": Tc, "sample_every": every}},
+            "variants": rows, "structure": structure, "data": "synthetic"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     cfg = W.CONFIGS[args.config]
@@ -406,6 +521,8 @@ def main():
         return run_reference(args, cfg)
     if args.calibrate:
         return run_calibrate(args, cfg)
+    if args.ablations:
+        return run_ablations(args, cfg)
 
     import torch
     import torch.distributed as dist

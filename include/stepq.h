@@ -65,6 +65,13 @@ typedef enum {
  * takes no part in the scale fit (ai.info summary, "Key Contributions"). */
 #define STEPQ_PIVOT_BITS 16
 
+/* Scale fits (stepq_pool_set_scale_mode).  STEPQ_SCALE_DUAL is the method;
+ * the others are the ablation variants the pages compare it with. */
+#define STEPQ_SCALE_DUAL 0
+#define STEPQ_SCALE_ROW 1
+#define STEPQ_SCALE_COL 2
+#define STEPQ_SCALE_HEAD 3
+
 /* Largest batch * heads a pool may hold. */
 #define STEPQ_MAX_ITEMS (1 << 24)
 
@@ -137,6 +144,21 @@ STEPQ_API stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, 
 /* Release the handle (host memory only; the device buffer stays the caller's).
  * Passing NULL returns STEPQ_ERR_INVALID_ARG. */
 STEPQ_API stepq_status stepq_pool_destroy(stepq_pool *pool);
+
+/* The scale fit of the pool's later stepq_pack, stepq_decode_step and
+ * stepq_decode_step_split calls (default STEPQ_SCALE_DUAL, the method: row
+ * scales from magnitude and impact, least-squares column scales).  The
+ * ablation variants (ai.info, "Main Findings": the method against
+ * spatial-only, temporal-only and uniform settings; state outliers lie along
+ * key rows and value columns at once) keep the stored form r_i c_j code_ij
+ * with plain absolute-maximum scales, no impact weights and no least squares:
+ *   STEPQ_SCALE_ROW : c_j = 1, r_i = max_j |S_ij| / Q_i (a zero row: 1 / Q_i);
+ *   STEPQ_SCALE_COL : r_i = 1 / Q_i, c_j = max_i |S_ij| (a zero column: 1);
+ *   STEPQ_SCALE_HEAD: r_i = 1 / Q_i, every c_j the largest |S_ij| of the
+ *                     state (one scale per (request, head)).
+ * Pivot rows are kept in binary16 in every mode.  Host-only; takes effect on
+ * the next call.  STEPQ_ERR_INVALID_ARG for another mode. */
+STEPQ_API stepq_status stepq_pool_set_scale_mode(stepq_pool *pool, int mode);
 
 /* Stream on which the pool's later calls enqueue their kernels. */
 STEPQ_API stepq_status stepq_pool_set_stream(stepq_pool *pool, void *cuda_stream);

@@ -48,6 +48,9 @@ def lib():
         L.oracle_decode_step.argtypes = [i, P, i, i, P, P, i, i, P, P, P, P, P, P, P, P, P, P]
         L.oracle_fp32_step.argtypes = [i, i, i, i, P, P, P, P, P, P, P]
         L.oracle_fp64_step.argtypes = [i, i, i, i, P, P, P, P, P, P, P]
+        L.oracle_fit_quantise_mode_f32.argtypes = [i, i, i, P, P, P, i, i, P, P, P, P, P]
+        L.oracle_pack_pool_mode.argtypes = [i, i, P, i, i, P, P, i, P, P]
+        L.oracle_decode_step_mode.argtypes = [i, i, P, i, i, P, P, i, i, P, P, P, P, P, P, P, P, P]
         L.oracle_calib_accumulate.argtypes = [i, i, i, i, P, P, P, P]
         L.oracle_calib_rho.argtypes = [i, i, C.c_double, P, P]
         L.oracle_calib_row_error.argtypes = [i, i, P, i, P, i, P, P, P]
@@ -70,6 +73,7 @@ def _c(a, dtype):
 
 
 PIVOT_FP16, PIVOT_EXACT = 0, 1
+SCALE_DUAL, SCALE_ROW, SCALE_COL, SCALE_HEAD = 0, 1, 2, 3
 
 
 def fit_quantise(S, bits, rho, ls_iters=1, pivot_mode=PIVOT_FP16, dtype=np.float32, diag=False):
@@ -88,6 +92,20 @@ def fit_quantise(S, bits, rho, ls_iters=1, pivot_mode=PIVOT_FP16, dtype=np.float
     if diag:
         out["tpre"] = tpre; out["lsgap"] = gap
     return out
+
+
+def fit_quantise_mode(mode, S, bits, rho, ls_iters=1):
+    """Fit variant `mode` (SCALE_*) + quantise one state S [dk, dv] (fp32).
+    Returns dict r, c, code, piv, tpre (the pre-rounding values p / c)."""
+    S = _c(S, np.float32)
+    dk, dv = S.shape
+    bits = _c(bits, np.uint8); rho = _c(rho, np.float32)
+    r = np.zeros(dk, np.float32); c = np.zeros(dv, np.float32)
+    code = np.zeros((dk, dv), np.int32); piv = np.zeros((dk, dv), np.float32)
+    tpre = np.zeros((dk, dv), np.float32)
+    lib().oracle_fit_quantise_mode_f32(int(mode), dk, dv, _ptr(S), _ptr(bits), _ptr(rho), ls_iters, PIVOT_FP16,
+                                       _ptr(r), _ptr(c), _ptr(code), _ptr(piv), _ptr(tpre))
+    return {"r": r, "c": c, "code": code, "piv": piv, "tpre": tpre}
 
 
 def quantise(S, bits, r, c, dtype=np.float32):
@@ -165,7 +183,8 @@ class SlotPool:
     slot_head[s] is the head of slot s; bits and rho are per-head tables [H, dk].
     """
 
-    def __init__(self, slot_head, bits, rho, dk=128, dv=128, ls_iters=1, kda=False):
+    def __init__(self, slot_head, bits, rho, dk=128, dv=128, ls_iters=1, kda=False, mode=SCALE_DUAL):
+        self.mode = int(mode)
         self.slot_head = _c(slot_head, np.int32)
         self.n = int(self.slot_head.shape[0])
         self.bits = _c(bits, np.uint8); self.rho = _c(rho, np.float32)
@@ -178,6 +197,10 @@ class SlotPool:
 
     def pack(self, S):
         S = _c(S, np.float32).reshape(self.n, self.dk, self.dv)
+        if self.mode != SCALE_DUAL:
+            lib().oracle_pack_pool_mode(self.mode, self.n, _ptr(self.slot_head), self.dk, self.dv, _ptr(self.bits),
+                                        _ptr(self.rho), self.ls_iters, _ptr(S), _ptr(self.pool))
+            return
         lib().oracle_pack_pool(self.n, _ptr(self.slot_head), self.dk, self.dv, _ptr(self.bits),
                                _ptr(self.rho), self.ls_iters, _ptr(S), _ptr(self.pool))
 
@@ -201,6 +224,16 @@ class SlotPool:
         alpha = _c(alpha, np.float32); beta = _c(beta, np.float32)
         assert alpha.size == (n * dk if self.kda else n)
         out = np.zeros((n, dv), np.float32)
+        if self.mode != SCALE_DUAL:  # no least squares: no least-squares gaps
+            S_new = np.zeros((n, dk, dv), np.float32) if diag else None
+            tpre = np.zeros((n, dk, dv), np.float32) if diag else None
+            lib().oracle_decode_step_mode(self.mode, n, _ptr(self.slot_head), dk, dv, _ptr(self.bits),
+                                          _ptr(self.rho), self.ls_iters, int(self.kda), _ptr(self.pool), _ptr(q),
+                                          _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(out), _ptr(S_new),
+                                          _ptr(tpre))
+            if diag:
+                return out, {"S_new": S_new, "tpre": tpre, "lsgap": np.full((n, dv), np.inf, np.float32)}
+            return out
         S_new = np.zeros((n, dk, dv), np.float32) if diag else None
         tpre = np.zeros((n, dk, dv), np.float32) if diag else None
         gap = np.zeros((n, dv), np.float32) if diag else None

@@ -311,6 +311,46 @@ void oracle_decode_step(int n, const int32_t *slot_head, int dk, int dv, const u
     scratch_free(&w);
 }
 
+void oracle_pack_pool_mode(int mode, int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits,
+                           const float *rho, int ls_iters, const float *S, uint8_t *pool)
+{
+    scratch_t w = scratch_new(dk, dv);
+    size_t off = 0;
+    for (int s = 0; s < n; s++) {
+        const uint8_t *bh = bits + (size_t)slot_head[s] * dk;
+        const float *rh = rho + (size_t)slot_head[s] * dk;
+        oracle_fit_quantise_mode_f32(mode, dk, dv, S + (size_t)s * dk * dv, bh, rh, ls_iters, ORACLE_PIVOT_FP16,
+                                     w.r, w.c, w.code, w.piv, NULL);
+        oracle_pack_item(dk, dv, bh, w.r, w.c, w.code, w.piv, pool + off);
+        off += oracle_item_bytes(dk, dv, bh);
+    }
+    scratch_free(&w);
+}
+
+void oracle_decode_step_mode(int mode, int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits,
+                             const float *rho, int ls_iters, int kda, uint8_t *pool, const float *q,
+                             const float *k, const float *v, const float *alpha, const float *beta,
+                             float *out, float *S_new, float *tpre)
+{
+    scratch_t w = scratch_new(dk, dv);
+    size_t off = 0;
+    for (int s = 0; s < n; s++) {
+        const uint8_t *bh = bits + (size_t)slot_head[s] * dk;
+        const float *rh = rho + (size_t)slot_head[s] * dk;
+        oracle_unpack_item(dk, dv, bh, pool + off, w.r, w.c, w.code, w.piv);
+        oracle_dequant_f32(dk, dv, bh, w.r, w.c, w.code, w.piv, w.S);
+        for (int i = 0; i < dk; i++) w.arow[i] = kda ? alpha[(size_t)s * dk + i] : alpha[s];
+        oracle_update_f32(dk, dv, w.S, w.arow, q + (size_t)s * dk, k + (size_t)s * dk,
+                          v + (size_t)s * dv, beta[s], out + (size_t)s * dv);
+        if (S_new) memcpy(S_new + (size_t)s * dk * dv, w.S, sizeof(float) * (size_t)dk * dv);
+        oracle_fit_quantise_mode_f32(mode, dk, dv, w.S, bh, rh, ls_iters, ORACLE_PIVOT_FP16, w.r, w.c,
+                                     w.code, w.piv, tpre ? tpre + (size_t)s * dk * dv : NULL);
+        oracle_pack_item(dk, dv, bh, w.r, w.c, w.code, w.piv, pool + off);
+        off += oracle_item_bytes(dk, dv, bh);
+    }
+    scratch_free(&w);
+}
+
 void oracle_fp32_step(int n, int dk, int dv, int kda, float *S, const float *q, const float *k,
                       const float *v, const float *alpha, const float *beta, float *out)
 {

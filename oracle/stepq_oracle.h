@@ -70,6 +70,19 @@ void oracle_fit_quantise_f64(int dk, int dv, const double *S, const uint8_t *bit
                              const float *rho, int ls_iters, int pivot_mode,
                              double *r, double *c, int32_t *code, double *piv,
                              double *tpre, double *lsgap);
+/* Fit variants for the ablations (stepq_oracle_core.inc states each):
+ * ORACLE_SCALE_DUAL (the method), _ROW (row scales only), _COL (column scales
+ * only), _HEAD (one scale per state).  Outputs as oracle_fit_quantise_f32. */
+#define ORACLE_SCALE_DUAL 0
+#define ORACLE_SCALE_ROW 1
+#define ORACLE_SCALE_COL 2
+#define ORACLE_SCALE_HEAD 3
+void oracle_fit_quantise_mode_f32(int mode, int dk, int dv, const float *S, const uint8_t *bits,
+                                  const float *rho, int ls_iters, int pivot_mode, float *r, float *c,
+                                  int32_t *code, float *piv, float *tpre);
+void oracle_fit_quantise_mode_f64(int mode, int dk, int dv, const double *S, const uint8_t *bits,
+                                  const float *rho, int ls_iters, int pivot_mode, double *r, double *c,
+                                  int32_t *code, double *piv, double *tpre);
 
 /* Quantise S with given scales (final step of the fit, exposed for checks). */
 void oracle_quantise_f32(int dk, int dv, const float *S, const uint8_t *bits, const float *r,
@@ -139,6 +152,14 @@ void oracle_decode_step(int n, const int32_t *slot_head, int dk, int dv, const u
                         const float *rho, int ls_iters, int kda, uint8_t *pool,
                         const float *q, const float *k, const float *v, const float *alpha,
                         const float *beta, float *out, float *S_new, float *tpre, float *lsgap);
+/* oracle_pack_pool and oracle_decode_step with a fit variant (ORACLE_SCALE_*);
+ * mode ORACLE_SCALE_DUAL is the two functions above. */
+void oracle_pack_pool_mode(int mode, int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits,
+                           const float *rho, int ls_iters, const float *S, uint8_t *pool);
+void oracle_decode_step_mode(int mode, int n, const int32_t *slot_head, int dk, int dv, const uint8_t *bits,
+                             const float *rho, int ls_iters, int kda, uint8_t *pool, const float *q,
+                             const float *k, const float *v, const float *alpha, const float *beta,
+                             float *out, float *S_new, float *tpre);
 /* Unquantised fp32 recursion over slots (the fp32-state baseline). */
 void oracle_fp32_step(int n, int dk, int dv, int kda, float *S, const float *q, const float *k,
                       const float *v, const float *alpha, const float *beta, float *out);

@@ -30,6 +30,7 @@ struct stepq_pool {
     stepq::Tables t{};
     int n_pivot_items = 0;
     int max_n16 = 0;  // the most leading 16-bit field positions of a staged head
+    int scale_mode = STEPQ_SCALE_DUAL;
     int nslots = 0, slot_bytes = 0;
     int off_q = 0, off_k = 0, off_v = 0, off_alpha = 0, off_ab = 0, off_rec = 0;
     // the active request set: decode steps update requests active[0..n_active)
@@ -261,6 +262,7 @@ stepq::StepArgs base_args(const stepq_pool *p)
     a.off_alpha = p->off_alpha; a.off_ab = p->off_ab; a.off_rec = p->off_rec;
     a.n_pivot_items = p->n_pivot_items;
     a.max_n16 = p->max_n16;
+    a.scale_mode = p->scale_mode;
     return a;
 }
 
@@ -464,6 +466,15 @@ stepq_status stepq_pool_set_stream(stepq_pool *pool, void *cuda_stream)
     stepq_status st = check_pool(pool);
     if (st != STEPQ_OK) return st;
     pool->stream = reinterpret_cast<cudaStream_t>(cuda_stream);
+    return STEPQ_OK;
+}
+
+stepq_status stepq_pool_set_scale_mode(stepq_pool *pool, int mode)
+{
+    stepq_status st = check_pool(pool);
+    if (st != STEPQ_OK) return st;
+    if (mode < STEPQ_SCALE_DUAL || mode > STEPQ_SCALE_HEAD) return fail(STEPQ_ERR_INVALID_ARG, "scale mode %d", mode);
+    pool->scale_mode = mode;
     return STEPQ_OK;
 }
 

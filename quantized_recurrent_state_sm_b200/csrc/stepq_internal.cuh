@@ -17,6 +17,9 @@ constexpr int kSlabCols = 16;     // value columns of a slab = columns a warp ow
 constexpr int kSlabs = kDV / kSlabCols;
 constexpr int kStreams = 32;      // streams per slab: 8 row groups x 4 column groups of 4
 constexpr int kPivotBits = 16;
+// scale fits: the method, and the ablation variants (row scales only, column
+// scales only, one scale per state); the values of STEPQ_SCALE_*
+constexpr int kScaleDual = 0, kScaleRow = 1, kScaleCol = 2, kScaleHead = 3;
 constexpr int kHeaderBytes = 4 * kDK + 4 * kDV;  // r[dk] | c[dv]
 constexpr int kMaxSlots = 8;
 
@@ -77,6 +80,7 @@ struct StepArgs {
     int off_q, off_k, off_v, off_alpha, off_ab, off_rec;  // offsets inside a slot
     int n_pivot_items;  // items of all-pivot heads, placed first in the order
     int max_n16;        // the most leading 16-bit field positions of any other head
+    int scale_mode;     // kScaleDual (the method) or an ablation variant
     const float *q, *k, *v, *alpha, *beta;
     float *out;
     const float *S_in;  // pack

@@ -568,7 +568,11 @@ enum FitResult { kFitDone = 0, kFitAbortNow = 1, kFitAbortAfter = 2 };
 // ERR (fixed widths; calibration): instead of packing, the squared
 // reconstruction error of every row, r'^2 sum_j (p_ij - c_j code_ij)^2 with the
 // codes the pack would store, goes to err_out[row] (item_g receives r' and c).
-template <int B, bool ROWWISE, bool MULTI, int NP, class Mid, bool ERR = false>
+// MODE (ablations): kScaleDual is the method; kScaleRow keeps c = 1 and sets
+// r_i = max_j |S_ij| / Q_i (0 -> 1 / Q_i); kScaleCol sets r_i = 1 / Q_i and
+// c_j = max_i |S_ij| (0 -> 1); kScaleHead as kScaleCol with every c_j the
+// largest of them.  The variants use no impact weights and no least squares.
+template <int B, bool ROWWISE, bool MULTI, int NP, class Mid, bool ERR = false, int MODE = kScaleDual>
 __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf, const HeadRec *rec, X2 &X,
                                                    uint8_t *item_g, int W, int ls_iters, bool store_c,
                                                    bool ok_in, const Mid &mid, float *err_out = nullptr)
@@ -584,9 +588,14 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
 #pragma unroll
             for (int e = 0; e < 4; e++) {
                 const int rr = 4 * q + e;
-                float2 s2 = __fmul2_rn(X[rr][0], X[rr][0]);
-                s2 = __ffma2_rn(X[rr][1], X[rr][1], s2);
-                s[e] = s2.x + s2.y;
+                if constexpr (MODE == kScaleRow) {  // row maxima of |P|
+                    s[e] = max_abs3(fabsf(X[rr][0].x), X[rr][0].y, X[rr][1].x);
+                    s[e] = max_abs3(s[e], X[rr][1].y, 0.f);
+                } else {
+                    float2 s2 = __fmul2_rn(X[rr][0], X[rr][0]);
+                    s2 = __ffma2_rn(X[rr][1], X[rr][1], s2);
+                    s[e] = s2.x + s2.y;
+                }
             }
             *reinterpret_cast<float4 *>(T + rowp_chunk(rg, q)) = make_float4(s[0], s[1], s[2], s[3]);
         }
@@ -600,21 +609,36 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
         float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
         for (int bk = 0; bk < 32; bk += 4) {
-            s0 += src[(bk + 0) * kDK];
-            s1 += src[(bk + 1) * kDK];
-            s2 += src[(bk + 2) * kDK];
-            s3 += src[(bk + 3) * kDK];
+            if constexpr (MODE == kScaleRow) {
+                s0 = fmaxf(s0, src[(bk + 0) * kDK]);
+                s1 = fmaxf(s1, src[(bk + 1) * kDK]);
+                s2 = fmaxf(s2, src[(bk + 2) * kDK]);
+                s3 = fmaxf(s3, src[(bk + 3) * kDK]);
+            } else {
+                s0 += src[(bk + 0) * kDK];
+                s1 += src[(bk + 1) * kDK];
+                s2 += src[(bk + 2) * kDK];
+                s3 += src[(bk + 3) * kDK];
+            }
         }
-        const float ss = (s0 + s1) + (s2 + s3);
         const int b = ROWWISE ? rec->bits[i] : B;
         float rnew = 0.f, h = 1.f, wt = 0.f;  // pivot rows: p = S, not part of any fit
         if (!ROWWISE || b != kPivotBits) {
             const float a = rf.ra[i];
-            float m = a * sqrt_approx(ss * (1.0f / kDV));
-            if (m == 0.f) m = 1.f;
-            rnew = (m * rec->s[i]) * rec->rq[i];
+            if constexpr (MODE == kScaleDual) {
+                const float ss = (s0 + s1) + (s2 + s3);
+                float m = a * sqrt_approx(ss * (1.0f / kDV));
+                if (m == 0.f) m = 1.f;
+                rnew = (m * rec->s[i]) * rec->rq[i];
+                wt = (rec->rho[i] * rnew) * rnew;
+            } else if constexpr (MODE == kScaleRow) {
+                float m = a * fmaxf(fmaxf(s0, s1), fmaxf(s2, s3));
+                if (m == 0.f) m = 1.f;
+                rnew = m * rec->rq[i];
+            } else {
+                rnew = rec->rq[i];
+            }
             h = div_approx(a, rnew);
-            wt = (rec->rho[i] * rnew) * rnew;
         }
         put_pair(rf.h2, i, h);
         put_pair(rf.w2, i, wt);
@@ -660,6 +684,15 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
         m = fmaxf(m, __shfl_xor_sync(kFull, hiB ? k0 : k1, 2));
         m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
         if constexpr (!ROWWISE) m = m * (1.0f / (float)((1 << (B - 1)) - 1));  // every row has width B
+        if constexpr (MODE == kScaleRow) m = 1.f;
+        if constexpr (MODE == kScaleHead) {  // the largest over all 128 columns
+            if ((rg & 1) == 0) sm.cnew[col0 + 2 * hiA + hiB] = m;
+            __syncthreads();
+            float top = fmaxf(fmaxf(sm.cnew[l], sm.cnew[l + 32]), fmaxf(sm.cnew[l + 64], sm.cnew[l + 96]));
+            top = __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(top)));  // non-negative floats
+            __syncthreads();
+            m = top;
+        }
         if ((rg & 1) == 0) {
             const int j = col0 + 2 * hiA + hiB;
             const float c0 = (m > 0.f) ? m : 1.f;
@@ -674,7 +707,9 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
     // |p / c0| <= Q, so the first round needs no clipping; later rounds clip to
     // the row's range.  More than one round is a separate instantiation (MULTI)
     // so that the one-round code holds a single round body.
-    if (!MULTI) {
+    if constexpr (MODE != kScaleDual) {
+        // the variants keep the maxima
+    } else if (!MULTI) {
         if (ls_iters > 0) ls_round<B, ROWWISE, false, NP>(sm, rf, X);
     } else {
         for (int it = 0; it < ls_iters; it++) {
@@ -949,7 +984,7 @@ struct StageNext {
 // A staged item: reconstruct + project (phase A), read out, Delta update
 // (phase B), then the fit, during which the next item is prepared.  The slot
 // sb stays untouched until the fit's second barrier.
-template <int B, bool KDA, bool MULTI, int NP>
+template <int B, bool KDA, bool MULTI, int NP, int MODE>
 __device__ __forceinline__ FitResult run_item(ItemSmem &sm, const StepArgs &a, RowFactors &rf, const uint8_t *sb,
                                               bool ok_slot, const StageNext<KDA> &next)
 {
@@ -1051,7 +1086,8 @@ __device__ __forceinline__ FitResult run_item(ItemSmem &sm, const StepArgs &a, R
     }
     const int rq = item / a.heads;
     uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + rec->head_off;
-    return fit_and_store<B, ROWWISE, MULTI, NP>(sm, rf, rec, X, item_g, W, a.ls_iters, true, ok_slot, next);
+    return fit_and_store<B, ROWWISE, MULTI, NP, StageNext<KDA>, false, MODE>(sm, rf, rec, X, item_g, W, a.ls_iters,
+                                                                           true, ok_slot, next);
 }
 
 // After a failed wait: record it, let every copy that may still be in flight
@@ -1072,7 +1108,7 @@ __device__ __forceinline__ void abort_drain(ItemSmem &sm, const StepArgs &a, uin
 
 // NP (row-wise widths): the leading positions checked for 16-bit fields; 1
 // when no head of the pool has more than one, else all 16.
-template <bool KDA, bool MULTI, int NP>
+template <bool KDA, bool MULTI, int NP, int MODE>
 __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
 {
     extern __shared__ __align__(128) uint8_t ring[];
@@ -1124,16 +1160,16 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
         const StageNext<KDA> next{sm, a, ring, n + G, slot_next, parity_next, sm.u.rf[par ^ 1]};
         FitResult res = kFitDone;
         if (KDA) {
-            res = run_item<0, KDA, MULTI, NP>(sm, a, rf, sb, ok, next);
+            res = run_item<0, KDA, MULTI, NP, MODE>(sm, a, rf, sb, ok, next);
         } else {
             switch (rf.head_b) {
-                case 2: res = run_item<2, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
-                case 3: res = run_item<3, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
-                case 4: res = run_item<4, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
-                case 5: res = run_item<5, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
-                case 6: res = run_item<6, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
-                case 7: res = run_item<7, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
-                case 8: res = run_item<8, KDA, MULTI, 0>(sm, a, rf, sb, ok, next); break;
+                case 2: res = run_item<2, KDA, MULTI, 0, MODE>(sm, a, rf, sb, ok, next); break;
+                case 3: res = run_item<3, KDA, MULTI, 0, MODE>(sm, a, rf, sb, ok, next); break;
+                case 4: res = run_item<4, KDA, MULTI, 0, MODE>(sm, a, rf, sb, ok, next); break;
+                case 5: res = run_item<5, KDA, MULTI, 0, MODE>(sm, a, rf, sb, ok, next); break;
+                case 6: res = run_item<6, KDA, MULTI, 0, MODE>(sm, a, rf, sb, ok, next); break;
+                case 7: res = run_item<7, KDA, MULTI, 0, MODE>(sm, a, rf, sb, ok, next); break;
+                case 8: res = run_item<8, KDA, MULTI, 0, MODE>(sm, a, rf, sb, ok, next); break;
                 default:  // unreachable: Gated-DeltaNet heads have one width, validated on the host
                     abort_drain(sm, a, n_cons, min(n_cons + nsl, n_stage), kStatusBadHead);
                     return;
@@ -1176,7 +1212,7 @@ __device__ __forceinline__ void load_head(RowFactors &rf, const HeadRec *rec)
     }
 }
 
-template <int B, bool ROWWISE>
+template <int B, bool ROWWISE, int MODE>
 __device__ __forceinline__ void pack_body(ItemSmem &sm, RowFactors &rf, const HeadRec *rec, const StepArgs &a,
                                           int item, uint8_t *item_g)
 {
@@ -1190,10 +1226,12 @@ __device__ __forceinline__ void pack_body(ItemSmem &sm, RowFactors &rf, const He
         X[rr][0] = f2(x.x, x.y);
         X[rr][1] = f2(x.z, x.w);
     }
-    fit_and_store<B, ROWWISE, true, kRowsPerGroup>(sm, rf, rec, X, item_g, (B > 0) ? 2 * B : rec->slab_words, a.ls_iters,
-                                    rec->head_kind != kHeadAllPivot, true, NoMid{});
+    fit_and_store<B, ROWWISE, true, kRowsPerGroup, NoMid, false, MODE>(sm, rf, rec, X, item_g,
+                                                                       (B > 0) ? 2 * B : rec->slab_words, a.ls_iters,
+                                                                       rec->head_kind != kHeadAllPivot, true, NoMid{});
 }
 
+template <int MODE>
 __global__ void __launch_bounds__(kThreads) k_pack(StepArgs a)
 {
     __shared__ ItemSmem sm;
@@ -1205,14 +1243,14 @@ __global__ void __launch_bounds__(kThreads) k_pack(StepArgs a)
     __syncthreads();
     uint8_t *item_g = a.pool + (long long)rq * a.req_bytes + rec->head_off;
     switch (rec->head_kind == kHeadQuant ? rec->head_b : 0) {
-        case 2: pack_body<2, false>(sm, rf, rec, a, item, item_g); break;
-        case 3: pack_body<3, false>(sm, rf, rec, a, item, item_g); break;
-        case 4: pack_body<4, false>(sm, rf, rec, a, item, item_g); break;
-        case 5: pack_body<5, false>(sm, rf, rec, a, item, item_g); break;
-        case 6: pack_body<6, false>(sm, rf, rec, a, item, item_g); break;
-        case 7: pack_body<7, false>(sm, rf, rec, a, item, item_g); break;
-        case 8: pack_body<8, false>(sm, rf, rec, a, item, item_g); break;
-        default: pack_body<0, true>(sm, rf, rec, a, item, item_g); break;
+        case 2: pack_body<2, false, MODE>(sm, rf, rec, a, item, item_g); break;
+        case 3: pack_body<3, false, MODE>(sm, rf, rec, a, item, item_g); break;
+        case 4: pack_body<4, false, MODE>(sm, rf, rec, a, item, item_g); break;
+        case 5: pack_body<5, false, MODE>(sm, rf, rec, a, item, item_g); break;
+        case 6: pack_body<6, false, MODE>(sm, rf, rec, a, item, item_g); break;
+        case 7: pack_body<7, false, MODE>(sm, rf, rec, a, item, item_g); break;
+        case 8: pack_body<8, false, MODE>(sm, rf, rec, a, item, item_g); break;
+        default: pack_body<0, true, MODE>(sm, rf, rec, a, item, item_g); break;
     }
 }
 
@@ -1458,27 +1496,29 @@ int sm_count()
     return g_sms;
 }
 
-template <bool KDA, bool MULTI, int NP>
+template <bool KDA, bool MULTI, int NP, int MODE>
 cudaError_t launch_decode_t(const StepArgs &a, cudaStream_t s)
 {
     const int dyn = a.nslots * a.slot_bytes;
-    cudaError_t e = cudaFuncSetAttribute(k_decode<KDA, MULTI, NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_decode<KDA, MULTI, NP, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<KDA, MULTI, NP>, kThreads, dyn);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<KDA, MULTI, NP, MODE>, kThreads, dyn);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const long long want = (long long)per_sm * sm_count();
     const int grid = (int)(a.n_items < want ? a.n_items : want);
-    k_decode<KDA, MULTI, NP><<<grid, kThreads, dyn, s>>>(a);
+    k_decode<KDA, MULTI, NP, MODE><<<grid, kThreads, dyn, s>>>(a);
     return cudaGetLastError();
 }
 
-template <bool MULTI>
+template <bool MULTI, int MODE>
 cudaError_t launch_decode_m(const StepArgs &a, cudaStream_t s)
 {
-    if (!a.kda) return launch_decode_t<false, MULTI, 0>(a, s);
-    return (a.max_n16 <= 1) ? launch_decode_t<true, MULTI, 1>(a, s) : launch_decode_t<true, MULTI, kRowsPerGroup>(a, s);
+    if (!a.kda) return launch_decode_t<false, MULTI, 0, MODE>(a, s);
+    return (a.max_n16 <= 1) ? launch_decode_t<true, MULTI, 1, MODE>(a, s)
+                            : launch_decode_t<true, MULTI, kRowsPerGroup, MODE>(a, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -1611,15 +1651,21 @@ cudaError_t launch_calib_reduce(const CalibArgs &c, cudaStream_t s)
 cudaError_t launch_decode_step(const StepArgs &a, cudaStream_t s)
 {
     if (a.n_items == 0) return cudaSuccess;
-    return (a.ls_iters <= 1) ? launch_decode_m<false>(a, s) : launch_decode_m<true>(a, s);
+    switch (a.scale_mode) {  // the variants fit without least squares: one instantiation each
+        case kScaleRow: return launch_decode_m<false, kScaleRow>(a, s);
+        case kScaleCol: return launch_decode_m<false, kScaleCol>(a, s);
+        case kScaleHead: return launch_decode_m<false, kScaleHead>(a, s);
+        default: break;
+    }
+    return (a.ls_iters <= 1) ? launch_decode_m<false, kScaleDual>(a, s) : launch_decode_m<true, kScaleDual>(a, s);
 }
 
 int decode_ctas_per_sm(int nslots, int slot_bytes)
 {
     const int dyn = nslots * slot_bytes;
     int per_sm = 0;
-    if (cudaFuncSetAttribute(k_decode<false, false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<false, false, 0>, kThreads, dyn) != cudaSuccess) {
+    if (cudaFuncSetAttribute(k_decode<false, false, 0, kScaleDual>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<false, false, 0, kScaleDual>, kThreads, dyn) != cudaSuccess) {
         cudaGetLastError();
         return 0;
     }
@@ -1629,7 +1675,12 @@ int decode_ctas_per_sm(int nslots, int slot_bytes)
 cudaError_t launch_pack(const StepArgs &a, cudaStream_t s)
 {
     if (a.n_items == 0) return cudaSuccess;
-    k_pack<<<a.n_items, kThreads, 0, s>>>(a);
+    switch (a.scale_mode) {
+        case kScaleRow: k_pack<kScaleRow><<<a.n_items, kThreads, 0, s>>>(a); break;
+        case kScaleCol: k_pack<kScaleCol><<<a.n_items, kThreads, 0, s>>>(a); break;
+        case kScaleHead: k_pack<kScaleHead><<<a.n_items, kThreads, 0, s>>>(a); break;
+        default: k_pack<kScaleDual><<<a.n_items, kThreads, 0, s>>>(a); break;
+    }
     return cudaGetLastError();
 }
 

@@ -18,6 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libstepq.so")
 
 GDN, KDA = 0, 1
+SCALE_DUAL, SCALE_ROW, SCALE_COL, SCALE_HEAD = 0, 1, 2, 3
 PIVOT_BITS = 16
 DK = DV = 128
 
@@ -46,7 +47,7 @@ EXPORTS = ("stepq_pool_bytes", "stepq_state_bytes", "stepq_pool_create", "stepq_
            "stepq_pool_set_stream", "stepq_pack", "stepq_unpack", "stepq_decode_step",
            "stepq_fp32_step", "stepq_pool_check", "stepq_status_string", "stepq_last_error",
            "stepq_decode_step_noalloc", "stepq_decode_step_split", "stepq_pool_set_active",
-           "stepq_calib_scratch_bytes", "stepq_calibrate", "stepq_calib_accumulate", "stepq_calib_row_error",
+           "stepq_pool_set_scale_mode", "stepq_calib_scratch_bytes", "stepq_calibrate", "stepq_calib_accumulate", "stepq_calib_row_error",
            "stepq_calib_reduce", "stepq_calib_rho", "stepq_calib_bits")
 
 
@@ -69,6 +70,7 @@ def _load():
     L.stepq_decode_step_noalloc.argtypes = [D, P, C.c_size_t, P, P, P, P, P, P, P]
     L.stepq_decode_step_split.argtypes = [P, P, P, P, P, P, P, P, P]
     L.stepq_pool_set_active.argtypes = [P, P, C.c_int]
+    L.stepq_pool_set_scale_mode.argtypes = [P, C.c_int]
     CD, i, dbl = C.POINTER(CalibDesc), C.c_int, C.c_double
     L.stepq_calib_scratch_bytes.argtypes = [CD]; L.stepq_calib_scratch_bytes.restype = C.c_size_t
     L.stepq_calibrate.argtypes = [CD, P, P, P, P, P, P, P, C.c_size_t, P, P, P]
@@ -79,7 +81,7 @@ def _load():
     L.stepq_calib_bits.argtypes = [i, i, dbl, P, P, P, i, P, dbl, dbl, P]
     for fn in ("stepq_pool_create", "stepq_pool_destroy", "stepq_pool_set_stream", "stepq_pool_check", "stepq_pack",
                "stepq_unpack", "stepq_decode_step", "stepq_fp32_step", "stepq_decode_step_noalloc",
-               "stepq_decode_step_split", "stepq_pool_set_active", "stepq_calibrate", "stepq_calib_accumulate",
+               "stepq_decode_step_split", "stepq_pool_set_active", "stepq_pool_set_scale_mode", "stepq_calibrate", "stepq_calib_accumulate",
                "stepq_calib_row_error", "stepq_calib_reduce", "stepq_calib_rho", "stepq_calib_bits"):
         getattr(L, fn).restype = C.c_int
     L.stepq_status_string.argtypes = [C.c_int]; L.stepq_status_string.restype = C.c_char_p
@@ -157,6 +159,11 @@ class PackedStatePool:
     @property
     def n_items(self) -> int:
         return self.batch * self.heads
+
+    def set_scale_mode(self, mode: int):
+        """The scale fit of later pack / decode calls: SCALE_DUAL (the method)
+        or an ablation variant SCALE_ROW, SCALE_COL, SCALE_HEAD."""
+        _check(lib.stepq_pool_set_scale_mode(self._h, int(mode)))
 
     def set_active(self, requests=None):
         """Restrict later decode steps to the listed requests (distinct slot

@@ -29,7 +29,7 @@ def to_dev(x):
 class Setup:
     """A GPU pool and the oracle's pool over the compared slots."""
 
-    def __init__(self, cfg, requests=None, bits=None, rho=None):
+    def __init__(self, cfg, requests=None, bits=None, rho=None, mode=0):
         self.cfg = cfg
         self.bits = W.bit_table(cfg) if bits is None else bits
         self.rho = W.rho(cfg) if rho is None else rho
@@ -38,7 +38,10 @@ class Setup:
         self.slots = (self.req[:, None] * H + np.arange(H)[None, :]).reshape(-1)
         self.kda = cfg.variant == W.KDA
         self.gpu = stepq.PackedStatePool(cfg.variant, cfg.batch, H, self.bits, self.rho, cfg.ls_iters)
-        self.ref = oracle.SlotPool(self.slots % H, self.bits, self.rho, ls_iters=cfg.ls_iters, kda=self.kda)
+        if mode:
+            self.gpu.set_scale_mode(mode)
+        self.ref = oracle.SlotPool(self.slots % H, self.bits, self.rho, ls_iters=cfg.ls_iters, kda=self.kda,
+                                   mode=mode)
         offs, total = W.item_offsets(self.bits, 128, cfg.batch)
         assert total == self.gpu.state_nbytes
         self.gpu_off = offs.reshape(-1)[self.slots]
