@@ -514,6 +514,73 @@ def run_ablations(args, cfg):
     return 0
 
 
+def rollout_drift(cfg, pool, S, ring, steps=256):
+    """Readout relative L2 error against the unquantised fp32 recursion after
+    `steps` steps from S (pool packed from S first; not timed)."""
+    import torch
+    from quantized_recurrent_state_sm_b200 import stepq
+    pool.pack(S)
+    Sf = S.clone()
+    o = of = None
+    for i in range(steps):
+        d = ring[i % RING]
+        o = pool.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+        of = stepq.fp32_step(cfg.variant, Sf, d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+    err = float(torch.linalg.vector_norm(o - of) / torch.linalg.vector_norm(of))
+    del Sf
+    return err if np.isfinite(err) else None
+
+
+def run_calibrated_tables(args, cfg, S, ring, out, stream, world):
+    """The same step on tables made by stepq_calibrate (16 calibration requests
+    x 32 steps) instead of the workload's stand-in tables: the stand-in
+    LogNormal impact weights make the requantised state diverge (a property
+    of the method as read, identical in the oracle), the calibrated ones keep
+    it finite.  Same pool size, average width and pivot share."""
+    import torch
+    from quantized_recurrent_state_sm_b200 import stepq
+    H = cfg.heads
+    Bc, Tc = 16, 32
+    xs = [W.calibration_inputs(cfg, t, Bc) for t in range(Tc)]
+    cdev = {k: torch.from_numpy(np.stack([x[k] for x in xs])).cuda() for k in xs[0]}
+    Sc = torch.zeros((Bc, H, cfg.dk, cfg.dv), device="cuda")
+    for t in range(-cfg.warmup, 0):
+        x = {k: torch.from_numpy(v).cuda() for k, v in W.step_inputs(cfg, t, W.calibration_requests(Bc)).items()}
+        stepq.fp32_step(cfg.variant, Sc, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+    rho_c, bits_c = stepq.calibrate(cfg.variant, Sc, cdev["q"], cdev["k"], cdev["v"], cdev["alpha"], cdev["beta"],
+                                    sorted(cfg.bits_choices), cfg.avg_bits, cfg.pivot_frac, 8, cfg.ls_iters)
+    del cdev, Sc
+    pool = stepq.PackedStatePool(cfg.variant, cfg.batch, H, bits_c, rho_c, cfg.ls_iters)
+    pool.pack(S)
+    n = max(10, args.steps // 5)
+
+    def step(i):
+        d = ring[i % RING]
+        pool.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"], out)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda") / n
+    finite = bool(torch.isfinite(out).all())
+    drift = rollout_drift(cfg, pool, S, ring)
+    pool.close()
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "value": whole_job_rate(world, cfg.items, n, ms * n), "steps": n,
+            "state_finite": finite, "avg_bits": float(bits_c.astype(float).mean()),
+            "readout_drift_256_steps": drift,
+            "tables": f"stepq_calibrate on {Bc} calibration requests x {Tc} steps"}
+
+
 def main():
     args = parse()
     cfg = W.CONFIGS[args.config]
@@ -571,8 +638,6 @@ def main():
         del S_tmp
     pool.pack(S)
     torch.cuda.synchronize()
-    del S
-    torch.cuda.empty_cache()
 
     def step(i):
         d = ring[i % RING]
@@ -596,6 +661,11 @@ def main():
     ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
     ms_per_step = ms / args.steps
     value = whole_job_rate(world, cfg.items, args.steps, ms)
+    state_finite = bool(torch.isfinite(out).all())
+    calibrated = None if args.profile else run_calibrated_tables(args, cfg, S, ring, out, stream, world)
+    drift = None if args.profile else rollout_drift(cfg, pool, S, ring)
+    del S
+    torch.cuda.empty_cache()
 
     # end to end through the public API with host buffers: pinned H2D of the
     # step's inputs, the decode step, D2H of the readout, every step
@@ -632,7 +702,11 @@ def main():
                 "ms_per_step": fp32_ms, "packed_speedup": fp32_ms / ms_per_step,
                 "state_bytes": cfg.items * cfg.dk * cfg.dv * 4},
             "clocks": clocks.summary(),
+            "state_finite": state_finite,
+            "readout_drift_256_steps": drift,
         }
+        if calibrated is not None:
+            line["calibrated_tables"] = calibrated
         if split is not None:
             split["fused_speedup"] = split["ms_per_step"] / ms_per_step
             line["split_pipeline"] = split
