@@ -513,11 +513,21 @@ def run_ablations(args, cfg):
                 o_err.append(float(torch.linalg.vector_norm(o - of[t]) / torch.linalg.vector_norm(of[t])))
         Sq = pool.unpack()
         pool.check()
+        # the variant's step time on the same pool (after the rollout; CUDA events)
+        n_t = 50
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for t in range(n_t):
+            d = ring[cfg.warmup + t]
+            pool.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+        t1.record()
+        torch.cuda.synchronize()
+        step_ms = t0.elapsed_time(t1) / n_t
         diff2 = (Sq - Sf).double() ** 2
         ref2 = Sf.double() ** 2
         state_rel = float(torch.sqrt(diff2.sum() / ref2.sum()))
         rows.append({"variant": name, "readout_rel_l2_last64": float(np.mean(o_err)), "state_rel_l2": state_rel,
-                     "avg_bits": float(bits.astype(float).mean())})
+                     "avg_bits": float(bits.astype(float).mean()), "ms_per_step": step_ms})
         if name.startswith(f"uniform {u_bits}-bit"):
             # accumulated squared state error per unit, summed over requests and value columns
             dims = (0, 3) if kda else (0, 2, 3)
