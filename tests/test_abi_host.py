@@ -92,3 +92,50 @@ def test_null_and_dead_handles(S):
     assert S.lib.stepq_pool_create(C.byref(d), C.c_void_p(16), 16, None, C.byref(out)) == S.ERR_INVALID_ARG
     assert S.lib.stepq_pool_create(C.byref(d), None, 0, None, None) == S.ERR_INVALID_ARG
     assert S.lib.stepq_status_string(3) == b"STEPQ_ERR_CUDA"
+
+
+def test_calibration_descriptor_validation(S):
+    """stepq_calib_scratch_bytes is 0 and stepq_calibrate returns
+    STEPQ_ERR_INVALID_ARG / UNSUPPORTED for invalid calibration descriptors,
+    on the host, before any device call."""
+    widths = np.array([3, 4, 6], np.int32)
+    wp = widths.ctypes.data_as(C.c_void_p)
+
+    def desc(**kw):
+        d = S.CalibDesc(S.GDN, 4, 8, 128, 128, 16, 8, 1, 3, wp, 4.0, 0.01)
+        for k, v in kw.items():
+            setattr(d, k, v)
+        return d
+
+    assert S.lib.stepq_calib_scratch_bytes(C.byref(desc())) > 0
+    bad = [dict(variant=7), dict(dk=64), dict(batch=0), dict(steps=0), dict(sample_every=0),
+           dict(sample_every=32), dict(ls_iters=-1), dict(n_widths=0), dict(n_widths=9),
+           dict(widths=None), dict(avg_bits=0.0), dict(pivot_frac=1.5)]
+    for kw in bad:
+        assert S.lib.stepq_calib_scratch_bytes(C.byref(desc(**kw))) == 0, kw
+    for ws in ([4, 3], [1, 4], [3, 9], [4, 4]):
+        w2 = np.array(ws, np.int32)
+        d = desc(n_widths=len(ws), widths=w2.ctypes.data_as(C.c_void_p))
+        assert S.lib.stepq_calib_scratch_bytes(C.byref(d)) == 0, ws
+    rho = np.zeros(8 * 128, np.float32); bits = np.zeros(8 * 128, np.uint8)
+    st = S.lib.stepq_calibrate(C.byref(desc(dk=64)), None, None, None, None, None, None, None, 0, None,
+                               rho.ctypes.data_as(C.c_void_p), bits.ctypes.data_as(C.c_void_p))
+    assert st == S.ERR_UNSUPPORTED
+    st = S.lib.stepq_calibrate(C.byref(desc()), None, None, None, None, None, None, None, 0, None,
+                               rho.ctypes.data_as(C.c_void_p), bits.ctypes.data_as(C.c_void_p))
+    assert st == S.ERR_INVALID_ARG  # scratch too small, before any pointer is touched
+
+
+def test_calibration_host_steps_validate(S):
+    acc = np.ones((2, 128)); rho = np.ones((2, 128), np.float32)
+    with pytest.raises(S.StepqError):
+        S.calib_rho(acc, 0.0)
+    err = np.ones((2, 3, 128))
+    with pytest.raises(S.StepqError):
+        S.calib_bits(S.GDN, np.zeros(2), rho, err, [3, 4, 3], 4.0, 0.0, 10.0)  # widths not ascending
+    with pytest.raises(S.StepqError):
+        S.calib_bits(S.GDN, np.zeros(2), rho, err, [3, 4, 6], 2.0, 0.0, 10.0)  # budget below the narrowest
+
+
+def test_scale_mode_rejects_unknown(S):
+    assert S.lib.stepq_pool_set_scale_mode(None, 0) == S.ERR_INVALID_ARG
