@@ -119,6 +119,7 @@ struct alignas(16) RowFactors {
     float ra[kDK];                  // a_i = alpha_i r_i (alpha_i on pivot rows), by row
     int rb[kDK];                    // widths, by sslot (row-wise widths only)
     float qf[kDK];                  // Q_i as a float (0 on pivot rows), by sslot (row-wise widths only)
+    int2 qlh[kDK];                  // bit patterns of 2^23 + 2^(F-1) -+ Q_i (F: the row's position width), by sslot
     float beta;
     int item, head_b;               // the item; its head's common width (0: row-wise)
     int n16;                        // its head's leading positions of 16-bit fields
@@ -392,18 +393,16 @@ __device__ __forceinline__ void pack_fixed(const X2 &X, float2 ic0, float2 ic1, 
     for (int rr = 0; rr < kRowsPerGroup; rr++)
 #pragma unroll
         for (int hh = 0; hh < 2; hh++) {
-            float2 mm;
-            if (!CLIP) {
-                mm = __ffma2_rn(X[rr][hh], hh ? ic1 : ic0, mz2);
-            } else {
-                float2 t = __fmul2_rn(X[rr][hh], hh ? ic1 : ic0);
-                t = f2(fminf(fmaxf(t.x, -(float)Qb), (float)Qb), fminf(fmaxf(t.y, -(float)Qb), (float)Qb));
-                mm = __fadd2_rn(t, mz2);
-            }
+            // p / c + 2^23 + z rounded once; clipping clamps its bit pattern to those
+            // of 2^23 + z -+ Q (the float order is the integer order of the bits,
+            // negative values included as signed integers)
+            const float2 mm = __ffma2_rn(X[rr][hh], hh ? ic1 : ic0, mz2);
+            constexpr int kLo = (int)kMagicBits + (1 << (B - 1)) - Qb, kHi = (int)kMagicBits + (1 << (B - 1)) + Qb;
 #pragma unroll
             for (int e = 0; e < 2; e++) {
                 const int c = 4 * rr + 2 * hh + e;
-                const uint32_t y = __float_as_uint(e ? mm.y : mm.x);
+                uint32_t y = __float_as_uint(e ? mm.y : mm.x);
+                if (CLIP) y = (uint32_t)min(max((int)y, kLo), kHi);
                 const int pos = c * B, lo = pos >> 5, sh = pos & 31;
                 if (sh + B <= 32) {
                     ow[lo] += y << sh;
@@ -459,22 +458,20 @@ __device__ __forceinline__ void pack_rowwise(const X2 &X, float2 ic0, float2 ic1
             const float2 zq = *reinterpret_cast<const float2 *>(&rf.pos[rr].mz);  // (2^23 + z, Q_F)
             const uint4 M = *reinterpret_cast<const uint4 *>(&rf.pos[rr].M1);
             const float2 mz2 = f2(zq.x, zq.x);
-            float2 y0, y1;
-            if (zq.y * (rat - 1.f) < 0.49f) {
-                y0 = __ffma2_rn(X[rr][0], ic0, mz2);
-                y1 = __ffma2_rn(X[rr][1], ic1, mz2);
-            } else {
-                const float Q = rf.qf[8 * rr + rg];
-                float2 t0 = __fmul2_rn(X[rr][0], ic0), t1 = __fmul2_rn(X[rr][1], ic1);
-                t0 = f2(fminf(fmaxf(t0.x, -Q), Q), fminf(fmaxf(t0.y, -Q), Q));
-                t1 = f2(fminf(fmaxf(t1.x, -Q), Q), fminf(fmaxf(t1.y, -Q), Q));
-                y0 = __fadd2_rn(t0, mz2);
-                y1 = __fadd2_rn(t1, mz2);
+            const float2 y0 = __ffma2_rn(X[rr][0], ic0, mz2), y1 = __ffma2_rn(X[rr][1], ic1, mz2);
+            uint32_t u0 = __float_as_uint(y0.x), u1 = __float_as_uint(y0.y);
+            uint32_t u2 = __float_as_uint(y1.x), u3 = __float_as_uint(y1.y);
+            if (zq.y * (rat - 1.f) >= 0.49f) {  // clip to the row's own range, on the bit patterns
+                const int2 b = rf.qlh[8 * rr + rg];
+                u0 = (uint32_t)min(max((int)u0, b.x), b.y);
+                u1 = (uint32_t)min(max((int)u1, b.x), b.y);
+                u2 = (uint32_t)min(max((int)u2, b.x), b.y);
+                u3 = (uint32_t)min(max((int)u3, b.x), b.y);
             }
-            uint32_t f = __float_as_uint(y0.x) - M.w;
-            f += __float_as_uint(y0.y) * M.x;
-            f += __float_as_uint(y1.x) * M.y;
-            f += __float_as_uint(y1.y) * M.z;
+            uint32_t f = u0 - M.w;
+            f += u1 * M.x;
+            f += u2 * M.y;
+            f += u3 * M.z;
             acc |= f << A.z;
             if (rf.pos[rr].done) {
                 words[A.x] = acc;
@@ -934,7 +931,10 @@ __device__ __forceinline__ void phase0(RowFactors &rf, const StepArgs &a, const 
     rf.ra[i] = A;
     if (KDA) {
         rf.rb[sslot(i)] = b;
-        rf.qf[sslot(i)] = (b == kPivotBits) ? 0.f : (float)qmax_of(b);
+        const int Q = (b == kPivotBits) ? 0 : qmax_of(b);
+        rf.qf[sslot(i)] = (float)Q;
+        const int zb = (int)kMagicBits + (1 << (rec->pos_bits[i & 15] - 1));
+        rf.qlh[sslot(i)] = make_int2(zb - Q, zb + Q);
         if (i < kRowsPerGroup) make_pos(rf, rec, i);
     }
     if (i == 0) {
@@ -1205,7 +1205,10 @@ __device__ __forceinline__ void load_head(RowFactors &rf, const HeadRec *rec)
         const int i = tid;
         rf.ra[i] = 1.f;
         rf.rb[sslot(i)] = rec->bits[i];
-        rf.qf[sslot(i)] = (rec->bits[i] == kPivotBits) ? 0.f : (float)qmax_of(rec->bits[i]);
+        const int Q = (rec->bits[i] == kPivotBits) ? 0 : qmax_of(rec->bits[i]);
+        rf.qf[sslot(i)] = (float)Q;
+        const int zb = (int)kMagicBits + (1 << (rec->pos_bits[i & 15] - 1));
+        rf.qlh[sslot(i)] = make_int2(zb - Q, zb + Q);
         put_pair(rf.q2, i, rec->rq[i]);
         if (i == 0) rf.n16 = rec->n16;
         if (i < kRowsPerGroup) make_pos(rf, rec, i);
