@@ -53,6 +53,19 @@ __device__ __forceinline__ int pslot(int i) { return ((i & 15) >> 1) * 8 + (i >>
 // Row i's place in per-row scalar arrays read by row group.
 __device__ __forceinline__ int sslot(int i) { return (i & 15) * 8 + (i >> 4); }
 
+// Row-wise widths (KDA): the row handled by thread t (0..127) where one thread
+// per row writes the duplicated-pair factors.  A half-warp covers the 8 row
+// groups x 2 rows of one pair position, so its 16 float2 writes fill 16
+// consecutive slots (no bank conflict, where consecutive rows per thread give
+// an 8-way conflict), and the row-partial reads stay conflict-free under
+// rowp_chunk's swizzle.  (The fixed-width kernels keep row = thread: there
+// the remap's extra registers cost more than the conflicts.)
+__device__ __forceinline__ int frow(int t)
+{
+    const int l = t & 31, m = 2 * (t >> 5) + (l >> 4);
+    return 16 * (l & 7) + 2 * m + ((l >> 3) & 1);
+}
+
 __device__ __forceinline__ void put_pair(float4 *arr, int i, float v)
 {
     reinterpret_cast<float2 *>(arr + pslot(i))[i & 1] = make_float2(v, v);
@@ -116,7 +129,7 @@ struct alignas(16) RowFactors {
     float4 a2[64], q2[64];          // alpha, 1/Q (0 on pivot rows); row-wise widths only
     float4 h2[64], w2[64];          // fit: h = a / r', w = rho r'^2
     float kqp[4];
-    float ra[kDK];                  // a_i = alpha_i r_i (alpha_i on pivot rows), by row
+    float ra[kDK];                  // a_i = alpha_i r_i (alpha_i on pivot rows), by row-factor thread
     int rb[kDK];                    // widths, by sslot (row-wise widths only)
     float qf[kDK];                  // Q_i as a float (0 on pivot rows), by sslot (row-wise widths only)
     int2 qlh[kDK];                  // bit patterns of 2^23 + 2^(F-1) -+ Q_i (F: the row's position width), by sslot
@@ -601,7 +614,7 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
     bool ok_mid = true;
     if (tid < kDK) {
         // ---- row i: RMS over the 128 columns, new row scale, fit factors -----
-        const int i = tid, irg = i >> 4, irr = i & 15;
+        const int i = ROWWISE ? frow(tid) : tid, irg = i >> 4, irr = i & 15;
         const float *src = &sm.rowp[rowp_chunk(irg, irr >> 2) + (irr & 3)];
         float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
@@ -621,7 +634,7 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
         const int b = ROWWISE ? rec->bits[i] : B;
         float rnew = 0.f, h = 1.f, wt = 0.f;  // pivot rows: p = S, not part of any fit
         if (!ROWWISE || b != kPivotBits) {
-            const float a = rf.ra[i];
+            const float a = rf.ra[tid];
             if constexpr (MODE == kScaleDual) {
                 const float ss = (s0 + s1) + (s2 + s3);
                 float m = a * sqrt_approx(ss * (1.0f / kDV));
@@ -904,7 +917,7 @@ __device__ __forceinline__ void produce(ItemSmem &sm, const StepArgs &a, int n_f
 template <bool KDA>
 __device__ __forceinline__ void phase0(RowFactors &rf, const StepArgs &a, const uint8_t *sb, int item)
 {
-    const int i = threadIdx.x - kDK;  // storage row
+    const int t = threadIdx.x - kDK, i = KDA ? frow(t) : t;  // storage row
     const HeadRec *rec = reinterpret_cast<const HeadRec *>(sb + a.off_rec);
     const float beta = *reinterpret_cast<const float *>(sb + a.off_ab + 4);
     const int b = rec->bits[i], key = rec->key_row[i];
@@ -928,7 +941,7 @@ __device__ __forceinline__ void phase0(RowFactors &rf, const StepArgs &a, const 
         put_pair(rf.a2, i, al);
         put_pair(rf.q2, i, rec->rq[i]);
     }
-    rf.ra[i] = A;
+    rf.ra[t] = A;  // by thread: read back by row-factor thread t, which handles the same row
     if (KDA) {
         rf.rb[sslot(i)] = b;
         const int Q = (b == kPivotBits) ? 0 : qmax_of(b);
@@ -976,7 +989,7 @@ struct StageNext {
         float kq = reinterpret_cast<const float *>(sb + a.off_k)[i] * reinterpret_cast<const float *>(sb + a.off_q)[i];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(kFull, kq, o);
-        if ((i & 31) == 0) rf_next.kqp[i >> 5] = kq;
+        if ((threadIdx.x & 31) == 0) rf_next.kqp[threadIdx.x >> 5] = kq;  // any split of the rows
         return true;
     }
 };
