@@ -9,7 +9,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libstepq.so")
 SOURCES = ["stepq_abi.cu", "stepq_kernels.cu"]
-HEADERS = ["stepq_internal.cuh"]
+HEADERS = ["stepq_internal.cuh", "stepq_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
