@@ -157,3 +157,19 @@ def test_low_impact_row_is_amplified_by_rounding():
             ratios.append(np.linalg.norm(Sh[0]) / np.linalg.norm(S[0]))
             assert np.abs(f["code"][0]).max() <= maxcode
         assert lo < np.mean(ratios) < hi, (rho0, np.mean(ratios))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode", [ROW, HEAD])
+def test_gpu_decode_variants_many_pivot_rows(mode):
+    """The variants on the KDA kernel that checks every row position for
+    pivot rows (a head with more than 8 pivot rows, so 16-bit fields at two
+    positions or more), in lockstep with the oracle."""
+    from tests.test_gpu_parity import Setup, lockstep
+    cfg = W.with_overrides(W.CONFIGS[2], batch=3, heads=2)
+    r_ = np.random.default_rng(7)
+    bits = r_.choice([3, 4, 5, 6, 7, 8], size=(2, 128)).astype(np.uint8)
+    bits[0, r_.choice(128, 20, replace=False)] = 16
+    assert W.position_widths(bits[0])[2] == 16  # a third 16-bit position
+    cmp, worst = lockstep(Setup(cfg, bits=bits, mode=mode), steps=3)
+    print(f"mode {mode}, 20 pivot rows: {cmp.diff}/{cmp.codes} codes differ, worst readout {worst:.2e}")
