@@ -188,17 +188,8 @@ def perturbed_copy(ref, bits, heads, seed):
     return P
 
 
-def test_free_running_drift_config0():
-    """Free-running rollout, 64 steps.  Requantising every step is chaotic: one
-    rounding decision that differs (the fp32 sums run in a different order on
-    the GPU) decorrelates that item's quantisation noise within a step, so
-    per-step readout and code tolerances apply only in lockstep (above).  Here
-    the drift against each side's own unquantised fp32 recursion must agree
-    with the oracle's to within 1e-3 relative or, when larger, three times the
-    spread of the oracle's drift across rollouts whose items each start one
-    code step apart."""
-    cfg = W.CONFIGS[0]
-    su = Setup(cfg)
+def drift_check(cfg, rho=None, steps=None):
+    su = Setup(cfg, rho=rho)
     n = cfg.items
     S0 = oracle.initial_state(cfg)
     su.ref.pack(S0.reshape(n, 128, 128))
@@ -206,7 +197,7 @@ def test_free_running_drift_config0():
     others = [perturbed_copy(su.ref, su.bits, cfg.heads, seed) for seed in range(3)]
     Sf_or = S0.reshape(n, 128, 128).copy()
     Sf_gpu = torch.from_numpy(S0).cuda()
-    for t in range(cfg.steps):
+    for t in range(cfg.steps if steps is None else steps):
         x = W.step_inputs(cfg, t)
         d = to_dev(x)
         out = su.gpu.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
@@ -215,7 +206,7 @@ def test_free_running_drift_config0():
         o_ref = su.ref.step(*args)
         for P in others:
             P.step(*args)
-        oracle.fp32_step(Sf_or, *args)
+        oracle.fp32_step(Sf_or, *args, kda=su.kda)
         if t == 0:  # the first step starts from identical bytes
             assert rel_l2(out.cpu().numpy().reshape(n, -1), o_ref) <= 1e-4
         if (t + 1) % 16 == 0:
@@ -227,6 +218,27 @@ def test_free_running_drift_config0():
             tol = max(1e-3 * D_or, 3 * spread)
             print(f"step {t}: drift gpu {D_gpu:.6f} oracle {D_or:.6f} spread {spread:.2e}")
             assert abs(D_gpu - D_or) <= tol, f"step {t}: drift {D_gpu:.6e} vs oracle {D_or:.6e} (tol {tol:.2e})"
+
+
+def test_free_running_drift_config0():
+    """Free-running rollout, 64 steps.  Requantising every step is chaotic: one
+    rounding decision that differs (the fp32 sums run in a different order on
+    the GPU) decorrelates that item's quantisation noise within a step, so
+    per-step readout and code tolerances apply only in lockstep (above).  Here
+    the drift against each side's own unquantised fp32 recursion must agree
+    with the oracle's to within 1e-3 relative or, when larger, three times the
+    spread of the oracle's drift across rollouts whose items each start one
+    code step apart."""
+    drift_check(W.CONFIGS[0])
+
+
+def test_free_running_drift_kda():
+    """The same drift rule on KDA heads (row-wise widths, pivot rows, per-row
+    gates), 64 steps.  Impact weights 1: with the workload's widely spread
+    stand-in weights the requantised state diverges in the oracle and on the
+    GPU alike, which leaves no drift to compare."""
+    cfg = W.with_overrides(W.CONFIGS[2], batch=2, heads=2)
+    drift_check(cfg, rho=np.ones((2, 128), np.float32), steps=64)
 
 
 @pytest.mark.parametrize("ci", [0, 2])
