@@ -139,3 +139,24 @@ def test_calibration_host_steps_validate(S):
 
 def test_scale_mode_rejects_unknown(S):
     assert S.lib.stepq_pool_set_scale_mode(None, 0) == S.ERR_INVALID_ARG
+
+
+def test_layout_agrees_across_implementations(S):
+    """Item sizes of random mixed-width heads (pivot rows included) agree
+    between the library, the oracle and the workload's format arithmetic:
+    the storage-row order and per-position field widths are written three
+    times, independently."""
+    import oracle
+    r = np.random.default_rng(21)
+    for trial in range(12):
+        H = int(r.integers(1, 6))
+        choices = r.choice([2, 3, 4, 5, 6, 7, 8, 16], size=int(r.integers(1, 5)), replace=False)
+        bits = r.choice(choices, size=(H, 128)).astype(np.uint8)
+        if trial % 3 == 0:
+            bits[0] = bits[0, 0]  # one head of a single width (key order)
+        rho = np.ones((H, 128), np.float32)
+        per_head = [oracle.item_bytes(bits[h]) for h in range(H)]
+        _, total = W.item_offsets(bits, 128, 3)
+        assert total == 3 * sum(per_head), trial
+        d, keep = S.make_desc(S.KDA, 3, H, bits, rho)
+        assert S.lib.stepq_state_bytes(C.byref(d)) == total, trial
