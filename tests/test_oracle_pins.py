@@ -483,3 +483,30 @@ def test_fp32_recursion_close_to_fp64():
         o64 = oracle.fp64_step(S64, q, k, v, a, b, kda=True)
     assert np.linalg.norm(S32 - S64) / np.linalg.norm(S64) < 1e-5
     assert np.linalg.norm(o32 - o64) / np.linalg.norm(o64) < 1e-5
+
+
+def test_golden_pack_streams_mixed_widths():
+    """Hand-derived streams of a mixed-width head (tests/golden/pack_streams_mixed.txt):
+    pins the storage-row order and the per-position field widths."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "pack_streams_mixed.txt")
+    want = None
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if line:
+            want = [int(x, 16) for x in line.split()]
+    bits = np.array([4] * 64 + [2] * 64, np.uint8)
+    code = np.zeros((128, 128), np.int32)
+    key = np.arange(128)
+    code[:64] = ((key[:64] // 8) % 7 - 3)[:, None]
+    code[64:] = 1
+    item = oracle.pack_item(bits, np.ones(128), np.ones(128), code, np.zeros((128, 128)))
+    words = item[1024:].view("<u4")
+    Wh = len(want)
+    assert words.size == 8 * 32 * Wh
+    for s_ in range(8):
+        slab = words[s_ * 32 * Wh:(s_ + 1) * 32 * Wh].reshape(Wh, 32)
+        for l in range(32):
+            assert list(slab[:, l]) == want, (s_, l)
+    back = oracle.unpack_item(bits, item, 128, 128)
+    np.testing.assert_array_equal(back["code"], code)
