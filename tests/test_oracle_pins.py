@@ -510,3 +510,31 @@ def test_golden_pack_streams_mixed_widths():
             assert list(slab[:, l]) == want, (s_, l)
     back = oracle.unpack_item(bits, item, 128, 128)
     np.testing.assert_array_equal(back["code"], code)
+
+
+def test_golden_pack_streams_pivot_position():
+    """Hand-derived streams of a head with one pivot row
+    (tests/golden/pack_streams_pivot.txt): binary16 fields and 16-bit codes
+    sharing the leading position."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "pack_streams_pivot.txt")
+    want = {}
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if line:
+            g, hx = [x.strip() for x in line.split("|")]
+            want[g] = [int(x, 16) for x in hx.split()]
+    bits = np.full(128, 8, np.uint8); bits[5] = 16
+    code = np.ones((128, 128), np.int32); code[5] = 0
+    piv = np.zeros((128, 128), np.float32); piv[5] = 1.0
+    item = oracle.pack_item(bits, np.ones(128), np.ones(128), code, piv)
+    Wh = len(want["0"])
+    words = item[1024:].view("<u4")
+    assert words.size == 8 * 32 * Wh
+    for s_ in range(8):
+        slab = words[s_ * 32 * Wh:(s_ + 1) * 32 * Wh].reshape(Wh, 32)
+        for l in range(32):
+            assert list(slab[:, l]) == want["0" if l % 8 == 0 else "other"], (s_, l)
+    back = oracle.unpack_item(bits, item, 128, 128)
+    np.testing.assert_array_equal(back["code"], code)
+    np.testing.assert_array_equal(back["piv"], piv)
