@@ -27,7 +27,8 @@
  *     readout o = S^T q on the updated, unquantised state;
  *   - stored form S_ij = r_i * c_j * code_ij, symmetric codes in [-Q_b, Q_b],
  *     Q_b = 2^(b-1) - 1, kept offset-binary (u = code + 2^(b-1), never 0);
- *   - row scale r_i = rms_i * rho_i^(-1/2) / Q_(b_i) (rms_i -> 1 if zero);
+ *   - row scale r_i = rms_i * max(rho_i, rho_max / 4)^(-1/2) / Q_(b_i)
+ *     (rms_i -> 1 if zero; rho_max the largest weight of the state's quantised rows);
  *   - column scale: init c_j = max_i |S_ij| / (r_i Q_(b_i)) (-> 1 if zero),
  *     then ls_iters rounds of impact-weighted least squares for fixed codes,
  *     weights rho_i r_i^2 on p_ij = S_ij / r_i;

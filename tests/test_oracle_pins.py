@@ -246,8 +246,15 @@ def test_row_scale_direction_and_invariances():
     base = oracle.fit_quantise(S, bits, rho)
     S2 = S.copy(); S2[3] *= 3.0
     assert oracle.fit_quantise(S2, bits, rho)["r"][3] > base["r"][3]
-    rho2 = rho.copy(); rho2[5] *= 4.0
-    assert oracle.fit_quantise(S, bits, rho2)["r"][5] < base["r"][5]
+    # four times the largest weight halves that row's scale (exactly: powers of 4)
+    top = int(np.argmax(rho))
+    rho2 = rho.copy(); rho2[top] *= 4.0
+    assert oracle.fit_quantise(S, bits, rho2)["r"][top] == base["r"][top] / 2
+    # a row already at the impact floor keeps its scale when its weight falls
+    low = int(np.argmin(rho))
+    assert rho[low] < rho.max() / 4
+    rho3 = rho.copy(); rho3[low] *= 0.5
+    np.testing.assert_array_equal(oracle.fit_quantise(S, bits, rho3)["r"], base["r"])
     # common factor 16 on the weights: r halves, c doubles, codes unchanged (exact)
     st = oracle.fit_quantise(S, bits, rho * 16)
     np.testing.assert_array_equal(st["code"], base["code"])
@@ -258,6 +265,28 @@ def test_row_scale_direction_and_invariances():
     np.testing.assert_array_equal(st3["code"], base["code"])
     np.testing.assert_array_equal(st3["r"], base["r"] * 8)
     np.testing.assert_array_equal(st3["c"], base["c"])
+
+
+def test_row_scale_hand_worked():
+    """Row scales worked by hand on rows whose root mean square, mean absolute
+    value and maximum all differ, with the impact floor binding on two rows
+    and a pivot row's weight ignored ("Methodology in Plain English": the
+    scale grows with the row's magnitude and shrinks with its impact score;
+    the magnitude is the row's RMS, the measure "Main Findings" uses).
+        row 0 = [1, -1, 2, 4]: RMS sqrt(22/4), mean |.| 2, max 4; rho 16 (the largest) -> s = 1/4
+        row 1 = [0, 3, 0, -4]: RMS 5/2, mean |.| 7/4, max 4; rho 1 < 16/4 -> s = 4^-1/2 = 1/2
+        row 2 = [2, 2, 2, 2]:  RMS 2; rho 1/2 -> floored, s = 1/2
+        row 3: a pivot row with rho 1000, outside the fit and the floor
+    r_i = RMS_i s_i / Q_i with Q = 7, 7, 31 (widths 4, 4, 6)."""
+    S = np.array([[1, -1, 2, 4], [0, 3, 0, -4], [2, 2, 2, 2], [9, 9, 9, 9]], np.float64)
+    bits = np.array([4, 4, 6, 16], np.uint8)
+    rho = np.array([16, 1, 0.5, 1000], np.float32)
+    st = oracle.fit_quantise(S, bits, rho, dtype=np.float64)
+    expect = [np.sqrt(5.5) * 0.25 / 7, 2.5 * 0.5 / 7, 2.0 * 0.5 / 31, 0.0]
+    np.testing.assert_allclose(st["r"], expect, rtol=1e-15, atol=0)
+    # the same rows in fp32: the scales round once per operation
+    st32 = oracle.fit_quantise(S, bits, rho)
+    np.testing.assert_allclose(st32["r"], expect, rtol=2e-7, atol=0)
 
 
 def test_higher_impact_rows_reconstruct_better():
