@@ -85,7 +85,11 @@ typedef struct {
      * an FP16 pivot row.  Gated-DeltaNet requires one width per head. */
     const uint8_t *bits;
     /* host [heads * dk]: calibrated row-impact weight of key row i of head h,
-     * finite and > 0 (pivot rows: ignored).  Fixed for all requests. */
+     * finite and > 0 (pivot rows: ignored).  Fixed for all requests.  It
+     * enters the row scale as max(rho_i, rho_max / 4)^(-1/2), rho_max the
+     * largest weight among the head's quantised rows (a row is coarsened by
+     * at most a factor 2 against the head's highest-impact row), and the
+     * column-scale fit as the weight of the row's squared error. */
     const float *rho;
 } stepq_desc;
 
@@ -186,7 +190,8 @@ STEPQ_API stepq_status stepq_pool_set_active(stepq_pool *pool, const int *active
  * Fit and quantise full-precision states into the pool (the initial state of
  * every item, or a restore from a checkpoint).  S: device fp32
  * [batch, heads, dk, dv].  Per item: row scales from the row's root-mean-square
- * magnitude and impact weight, column scales by least squares, codes by
+ * magnitude and impact weight (r_i = rms_i max(rho_i, rho_max / 4)^(-1/2) /
+ * Q_i), column scales by least squares, codes by
  * round-half-even with clamping -- the same fit the decode step performs after
  * its update (ai.info summary, "Methodology in Plain English").
  */
@@ -268,6 +273,12 @@ STEPQ_API stepq_status stepq_pool_check(stepq_pool *pool);
  * call rebuilds them on the host and uploads them on the stream before its
  * launch.  No device or host memory is allocated on the success path (an
  * error message may be formatted into the library's per-thread error string).
+ *
+ * The upload is a cudaMemcpyAsync from a static, pageable host image, and CUDA
+ * starts a copy from pageable host memory only after the work queued earlier
+ * on the stream has finished: each call therefore blocks the calling thread
+ * until the stream has drained up to it, then returns with its own kernel
+ * queued (unlike the pool entry points, which return without waiting).
  *
  * desc: as for stepq_pool_create, with heads <= 64 and tables that fit the
  * scratch (about 10 000 items at 32 heads, 7 500 at 64); larger descriptors

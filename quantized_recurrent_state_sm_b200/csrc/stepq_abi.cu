@@ -113,6 +113,13 @@ int fill_rows(const stepq_desc *d, int h, stepq::HeadRec &R)
     const uint8_t *bits = d->bits + (size_t)h * kDK;
     int key_of[kDK];
     storage_rows(bits, key_of);
+    // impact floor of the row-scale factor: a quarter of the largest weight
+    // among the head's quantised rows, so that no row's step is coarsened by
+    // more than a factor 2 against the head's highest-impact row
+    double rho_max = 0.0;
+    for (int i = 0; i < kDK; i++)
+        if (bits[i] != STEPQ_PIVOT_BITS) rho_max = std::max(rho_max, (double)d->rho[(size_t)h * kDK + i]);
+    const double rho_floor = rho_max / 4.0;
     int npiv = 0, same = 1;
     for (int s = 0; s < kDK; s++) {
         const int i = key_of[s], b = bits[i];
@@ -125,7 +132,7 @@ int fill_rows(const stepq_desc *d, int h, stepq::HeadRec &R)
             R.rho[s] = 0.f;
             R.rq[s] = 0.f;
         } else {
-            R.s[s] = (float)(1.0 / std::sqrt((double)d->rho[(size_t)h * kDK + i]));
+            R.s[s] = (float)(1.0 / std::sqrt(std::max((double)d->rho[(size_t)h * kDK + i], rho_floor)));
             R.rho[s] = d->rho[(size_t)h * kDK + i];
             R.rq[s] = (float)(1.0 / (double)((1 << (b - 1)) - 1));
         }

@@ -31,7 +31,7 @@ constexpr int kHeadMixed = 2;     // some rows pivots
 // Per-head record (host-built, staged with every item): the fit constants and
 // the tile layout of the head's items.
 struct HeadRec {
-    float s[kDK];                // fp32(rho_i^-1/2), rounded once from fp64 (0 on pivot rows), by storage row
+    float s[kDK];                // fp32(max(rho_i, rho_max / 4)^-1/2), rounded once from fp64 (0 on pivot rows), by storage row
     float rho[kDK];              // row-impact weights (0 on pivot rows)
     float rq[kDK];               // fp32(1 / Q_i), Q_i = 2^(b_i - 1) - 1 (0 on pivot rows)
     // per storage row (key order for a one-width head; otherwise the key rows

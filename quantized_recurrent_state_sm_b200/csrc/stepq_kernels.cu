@@ -21,7 +21,9 @@
 //   gate         S'   = diag(alpha) S
 //   update       S    = S' + (beta k)(v - S'^T k)^T
 //   readout      o    = S^T q
-//   refit        r_i  = rms_i rho_i^-1/2 / Q_i ; p = S / r ;
+//   refit        r_i  = rms_i s_i / Q_i, s_i = max(rho_i, rho_max / 4)^-1/2 (no row
+//                coarsened by more than a factor 2 against the highest-impact row);
+//                p = S / r ;
 //                c_j  = max_i |p_ij| / Q_i, then least squares for fixed codes
 //   requantise   code = clamp(rne(p / c)); pack; store.
 //
@@ -1594,9 +1596,19 @@ __global__ void __launch_bounds__(kThreads) k_calib_error(CalibArgs c)
     RowFactors &rf = sm.u.rf[0];
     const int item = blockIdx.x, h = item % c.heads, tid = threadIdx.x;
     float s_i = 0.f, rho_i = 0.f;
+    __shared__ float rho_wmax[kThreads / 32];
+    if (tid < kDK) rho_i = c.rho[h * kDK + tid];
+    {  // the head's largest impact weight (every row is quantised here); weights are positive floats
+        const unsigned m = __reduce_max_sync(kFull, __float_as_uint(rho_i));
+        if ((tid & 31) == 0) rho_wmax[tid >> 5] = __uint_as_float(m);
+        __syncthreads();
+    }
     if (tid < kDK) {
-        rho_i = c.rho[h * kDK + tid];
-        s_i = (float)(1.0 / sqrt((double)rho_i));  // fp32(rho^-1/2) from fp64, as the host tables
+        float rmax = rho_wmax[0];
+#pragma unroll
+        for (int x = 1; x < kDK / 32; x++) rmax = fmaxf(rmax, rho_wmax[x]);
+        // fp32(max(rho, rho_max / 4)^-1/2) from fp64, as the host tables
+        s_i = (float)(1.0 / sqrt(fmax((double)rho_i, (double)rmax / 4.0)));
     }
     for (int x = 0; x < c.n_widths; x++) {
         const int b = c.widths[x];

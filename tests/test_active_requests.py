@@ -1,6 +1,9 @@
-"""Decode over an active subset of the pool's requests (stepq_pool_set_active):
-the active requests' items come out exactly as in a full step over the same
-states, and the inactive requests' states stay untouched."""
+"""Decode over an active subset of the pool's requests (stepq_pool_set_active),
+the slot-indexed pool of a serving runtime: the active requests' items match
+the oracle's pool over exactly those slots (lockstep, the parity rules of the
+full step), the inactive requests' input rows are never read, their output
+rows never written and their states left untouched; the subset step also
+equals the full step bit for bit on the active items."""
 import numpy as np
 import pytest
 import torch
@@ -13,6 +16,37 @@ pytestmark = pytest.mark.gpu
 def _pool(stepq, cfg):
     bits, rho = W.bit_table(cfg), W.rho(cfg)
     return stepq.PackedStatePool(cfg.variant, cfg.batch, cfg.heads, bits, rho, cfg.ls_iters)
+
+
+@pytest.mark.parametrize("ci", [1, 2, 4])
+def test_active_subset_matches_oracle(ci):
+    from tests.test_gpu_parity import Setup, lockstep
+    cfg = W.with_overrides(W.CONFIGS[ci], batch=6)
+    active = [4, 0, 3]
+    inactive = [1, 2, 5]
+    su = Setup(cfg, requests=active)  # the oracle follows exactly the active slots
+    g = torch.Generator(device="cuda").manual_seed(ci)
+    su.gpu.pack(torch.randn((cfg.batch, cfg.heads, 128, 128), device="cuda", generator=g) * 0.2)
+    su.gpu.set_active(active)
+    offs, total = W.item_offsets(su.bits, 128, cfg.batch)
+    per_req = int(np.asarray(offs).reshape(cfg.batch, cfg.heads)[1, 0])
+
+    def step(gpu, d):
+        before = gpu.state.clone()
+        xp = {k: v.clone() for k, v in d.items()}
+        for k in xp:
+            xp[k][inactive] = float("nan")  # never read
+        out = torch.full((cfg.batch, cfg.heads, 128), -7.0, device="cuda")
+        gpu.decode_step(xp["q"], xp["k"], xp["v"], xp["alpha"], xp["beta"], out)
+        torch.cuda.synchronize()
+        assert bool((out[inactive] == -7.0).all())  # never written
+        for b in inactive:
+            seg = slice(b * per_req, (b + 1) * per_req)
+            assert torch.equal(gpu.state[seg], before[seg]), b
+        return out
+
+    cmp, worst = lockstep(su, steps=3, t0=50, step=step)
+    print(f"config {ci}, active {active}: {cmp.diff}/{cmp.codes} codes differ, worst readout {worst:.2e}")
 
 
 @pytest.mark.parametrize("ci", [1, 2])

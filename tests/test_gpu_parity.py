@@ -169,78 +169,6 @@ def test_kda_position_layouts():
     lockstep(Setup(cfg, bits=bits), steps=4)
 
 
-def perturbed_copy(ref, bits, heads, seed):
-    """The oracle pool with one code of every item moved by one step: a rollout
-    whose rounding noise is decorrelated from the original in every item."""
-    P = oracle.SlotPool(ref.slot_head, ref.bits, ref.rho, ls_iters=ref.ls_iters, kda=ref.kda)
-    P.pool[:] = ref.pool
-    r = np.random.default_rng(seed)
-    for s in range(P.n):
-        bh = bits[ref.slot_head[s]]
-        it = oracle.unpack_item(bh, P.item(s), 128, 128)
-        rows = np.flatnonzero(bh != 16)
-        if rows.size == 0:
-            continue
-        i, j = int(r.choice(rows)), int(r.integers(128))
-        Q = (1 << (int(bh[i]) - 1)) - 1
-        it["code"][i, j] += 1 if it["code"][i, j] < Q else -1
-        P.set_item(s, oracle.pack_item(bh, it["r"], it["c"], it["code"], it["piv"]))
-    return P
-
-
-def drift_check(cfg, rho=None, steps=None):
-    su = Setup(cfg, rho=rho)
-    n = cfg.items
-    S0 = oracle.initial_state(cfg)
-    su.ref.pack(S0.reshape(n, 128, 128))
-    su.push_oracle_bytes()
-    others = [perturbed_copy(su.ref, su.bits, cfg.heads, seed) for seed in range(3)]
-    Sf_or = S0.reshape(n, 128, 128).copy()
-    Sf_gpu = torch.from_numpy(S0).cuda()
-    for t in range(cfg.steps if steps is None else steps):
-        x = W.step_inputs(cfg, t)
-        d = to_dev(x)
-        out = su.gpu.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
-        stepq.fp32_step(cfg.variant, Sf_gpu, d["q"], d["k"], d["v"], d["alpha"], d["beta"])
-        args = su.slot_inputs(x)
-        o_ref = su.ref.step(*args)
-        for P in others:
-            P.step(*args)
-        oracle.fp32_step(Sf_or, *args, kda=su.kda)
-        if t == 0:  # the first step starts from identical bytes
-            assert rel_l2(out.cpu().numpy().reshape(n, -1), o_ref) <= 1e-4
-        if (t + 1) % 16 == 0:
-            Sg = Sf_gpu.cpu().numpy().reshape(n, 128, 128)
-            assert rel_l2(Sg, Sf_or) < 1e-5  # the two fp32 references agree
-            D_gpu = rel_l2(su.gpu.unpack().cpu().numpy().reshape(n, 128, 128), Sg)
-            D_or = rel_l2(su.ref.unpack(), Sf_or)
-            spread = max(abs(rel_l2(P.unpack(), Sf_or) - D_or) for P in others)
-            tol = max(1e-3 * D_or, 3 * spread)
-            print(f"step {t}: drift gpu {D_gpu:.6f} oracle {D_or:.6f} spread {spread:.2e}")
-            assert abs(D_gpu - D_or) <= tol, f"step {t}: drift {D_gpu:.6e} vs oracle {D_or:.6e} (tol {tol:.2e})"
-
-
-def test_free_running_drift_config0():
-    """Free-running rollout, 64 steps.  Requantising every step is chaotic: one
-    rounding decision that differs (the fp32 sums run in a different order on
-    the GPU) decorrelates that item's quantisation noise within a step, so
-    per-step readout and code tolerances apply only in lockstep (above).  Here
-    the drift against each side's own unquantised fp32 recursion must agree
-    with the oracle's to within 1e-3 relative or, when larger, three times the
-    spread of the oracle's drift across rollouts whose items each start one
-    code step apart."""
-    drift_check(W.CONFIGS[0])
-
-
-def test_free_running_drift_kda():
-    """The same drift rule on KDA heads (row-wise widths, pivot rows, per-row
-    gates), 64 steps.  Impact weights 1: with the workload's widely spread
-    stand-in weights the requantised state diverges in the oracle and on the
-    GPU alike, which leaves no drift to compare."""
-    cfg = W.with_overrides(W.CONFIGS[2], batch=2, heads=2)
-    drift_check(cfg, rho=np.ones((2, 128), np.float32), steps=64)
-
-
 @pytest.mark.parametrize("ci", [0, 2])
 def test_fp32_baseline_matches_oracle(ci):
     cfg = W.with_overrides(W.CONFIGS[ci], batch=2)

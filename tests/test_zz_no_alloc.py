@@ -39,10 +39,11 @@ def test_noalloc_matches_pool_on_two_calls(S, ci, batch):
                                        x["beta"], ls_iters=cfg.ls_iters)
         torch.cuda.synchronize()
         pool.check()
-        a, b = o_free.double(), o_pool.double()
-        assert float((a - b).norm() / b.norm()) <= 1e-4, f"readout differs at call {t}"
+        # the same kernel on the same bytes and inputs, in the same item order:
+        # identical results, bit for bit
+        assert torch.equal(o_free, o_pool), f"readout differs at call {t}"
         diff = int((states != pool.state).sum())
-        assert diff <= 1e-4 * states.numel(), f"{diff} packed bytes differ at call {t}"
+        assert diff == 0, f"{diff} packed bytes differ at call {t}"
 
 
 @pytest.mark.gpu
