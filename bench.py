@@ -818,6 +818,10 @@ def main():
         del S_tmp
     pool.pack(S)
     torch.cuda.synchronize()
+    if args.profile:  # keep a profiler's device-memory save and restore small
+        del S
+        S = None
+        torch.cuda.empty_cache()
 
     def step(i):
         d = ring[i % RING]

@@ -133,6 +133,27 @@ STEPQ_API size_t stepq_pool_bytes(const stepq_desc *desc);
 STEPQ_API size_t stepq_state_bytes(const stepq_desc *desc);
 
 /*
+ * Where a pool buffer's regions lie (byte offsets from its start), for
+ * inspection and tests; the pages describe no counterpart.  The packed states
+ * come first, then the library's tables: the per-head records, the item
+ * offsets within a request and the item sizes per head, the device status
+ * word, the item order and the staging records (one per item, 16 bytes:
+ * item, item bytes | head << 16, item offset / 1024, request).  Every region
+ * is followed by a guard region of guard_bytes bytes (guards[0] after the
+ * states, then one after each table in that order) that pool creation fills
+ * with a fixed pattern and stepq_pool_check_guards compares.
+ * STEPQ_ERR_INVALID_ARG / STEPQ_ERR_UNSUPPORTED for an invalid descriptor.
+ */
+typedef struct {
+    size_t states, state_bytes;
+    size_t head_records, head_offsets, item_sizes, status_word, item_order, staging_records;
+    size_t guards[7];
+    size_t guard_bytes;
+    size_t total; /* == stepq_pool_bytes(desc) */
+} stepq_pool_regions;
+STEPQ_API stepq_status stepq_pool_layout(const stepq_desc *desc, stepq_pool_regions *out);
+
+/*
  * Create a pool over a caller-owned device buffer of at least
  * stepq_pool_bytes(desc) bytes (16-byte aligned).  Copies the descriptor and
  * the host tables, writes the derived per-head tables into the tail of the
@@ -258,6 +279,27 @@ STEPQ_API stepq_status stepq_fp32_step(const stepq_desc *desc, float *S, const f
  * word).
  */
 STEPQ_API stepq_status stepq_pool_check(stepq_pool *pool);
+
+/*
+ * Memory-safety aid (no counterpart on the pages): synchronise the pool's
+ * stream and compare the guard regions that follow every region of the pool
+ * buffer (see stepq_pool_layout) with the pattern pool creation wrote.  A
+ * kernel write beyond the packed states or a table shows up here.  Returns
+ * STEPQ_OK, or STEPQ_ERR_STATE naming the first changed guard word in
+ * stepq_last_error(); STEPQ_ERR_CUDA if the copy back fails.  Host memory
+ * only on the stack; the guards are not rewritten.
+ *
+ * A library built with STEPQ_CHECK=1 (libstepq_check.so, loaded by the Python
+ * binding when the environment variable STEPQ_CHECK is 1) also validates, in a
+ * kernel launched before every kernel that reads the pool's tables, each head
+ * record and staging record against the layout: item and head in range, the
+ * item's size equal to its head's, its offset equal to request x request bytes
+ * + the head's offset and inside the packed states, the order table equal to
+ * the staging records.  A violation sets the status word (reported by
+ * stepq_pool_check) and the dependent kernels return without touching memory;
+ * while the word is set, later launches do nothing.
+ */
+STEPQ_API stepq_status stepq_pool_check_guards(stepq_pool *pool);
 
 /*
  * The fused decode step of stepq_decode_step without a pool, allocating

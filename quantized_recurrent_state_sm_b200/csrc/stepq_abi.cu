@@ -39,6 +39,8 @@ struct stepq_pool {
     std::vector<long long> item_bytes;   // per head
     std::vector<long long> head_off;     // per head
     std::vector<int> active_tables;      // host copy of the uploaded order and staging records
+    size_t guard[7] = {};                // offsets of the guard regions (kGuardRegions)
+    size_t total = 0;                    // bytes of the pool's regions, guards included
 };
 
 namespace {
@@ -149,10 +151,23 @@ int fill_rows(const stepq_desc *d, int h, stepq::HeadRec &R)
     return npiv;
 }
 
+// Guard words: a 64-byte region after every region of a pool buffer, filled
+// at creation with a fixed pattern and compared by stepq_pool_check_guards.
+constexpr size_t kGuardBytes = 64;
+constexpr int kGuardRegions = 7;
+const char *const kGuardAfter[kGuardRegions] = {"packed states", "head records", "head offsets", "item sizes",
+                                                "status word", "item order", "staging records"};
+
+uint32_t guard_word(int g, int k)
+{
+    return 0x5A17C0DEu ^ (uint32_t)g * 0x9E3779B9u ^ (uint32_t)k * 0x85EBCA6Bu;
+}
+
 struct Layout {
     size_t state = 0;
     size_t off_rec = 0, off_head_off = 0, off_head_bytes = 0, off_order = 0, off_stage = 0, off_status = 0,
            total = 0;
+    size_t guard[kGuardRegions] = {};
     long long req_bytes = 0;
     std::vector<long long> item_bytes;  // per head
     std::vector<int> slab_words;        // per head: 32-bit words per stream
@@ -205,13 +220,21 @@ stepq_status check_desc(const stepq_desc *d, bool need_tables, Layout *L)
         }
         L->req_bytes = req;
         L->state = (size_t)req * (size_t)d->batch;
-        size_t o = align_up(L->state, 256);
-        L->off_rec = o;        o = align_up(o + sizeof(stepq::HeadRec) * (size_t)H, 256);
+        // each region is followed by a guard region
+        size_t o = align_up(L->state, 16);
+        L->guard[0] = o;       o = align_up(o + kGuardBytes, 256);
+        L->off_rec = o;        o = align_up(o + sizeof(stepq::HeadRec) * (size_t)H, 16);
+        L->guard[1] = o;       o = align_up(o + kGuardBytes, 16);
         L->off_head_off = o;   o = align_up(o + 8 * (size_t)H, 16);
+        L->guard[2] = o;       o = align_up(o + kGuardBytes, 16);
         L->off_head_bytes = o; o = align_up(o + 4 * (size_t)H, 16);
+        L->guard[3] = o;       o = align_up(o + kGuardBytes, 16);
         L->off_status = o;     o = align_up(o + 16, 16);
+        L->guard[4] = o;       o = align_up(o + kGuardBytes, 16);
         L->off_order = o;      o = align_up(o + 4 * (size_t)H * d->batch, 16);
+        L->guard[5] = o;       o = align_up(o + kGuardBytes, 16);
         L->off_stage = o;      o = align_up(o + 16 * (size_t)H * d->batch, 16);
+        L->guard[6] = o;       o = align_up(o + kGuardBytes, 16);
         L->total = o;
     }
     return STEPQ_OK;
@@ -270,6 +293,8 @@ stepq::StepArgs base_args(const stepq_pool *p)
     a.n_pivot_items = p->n_pivot_items;
     a.max_n16 = p->max_n16;
     a.scale_mode = p->scale_mode;
+    a.batch = p->desc.batch;
+    a.state_bytes = (long long)p->state_bytes;
     return a;
 }
 
@@ -348,6 +373,26 @@ size_t stepq_state_bytes(const stepq_desc *desc)
     return check_desc(desc, true, &L) == STEPQ_OK ? L.state : 0;
 }
 
+stepq_status stepq_pool_layout(const stepq_desc *desc, stepq_pool_regions *out)
+{
+    if (!out) return fail(STEPQ_ERR_INVALID_ARG, "out is NULL");
+    Layout L;
+    stepq_status st = check_desc(desc, true, &L);
+    if (st != STEPQ_OK) return st;
+    out->states = 0;
+    out->state_bytes = L.state;
+    out->head_records = L.off_rec;
+    out->head_offsets = L.off_head_off;
+    out->item_sizes = L.off_head_bytes;
+    out->status_word = L.off_status;
+    out->item_order = L.off_order;
+    out->staging_records = L.off_stage;
+    for (int g = 0; g < kGuardRegions; g++) out->guards[g] = L.guard[g];
+    out->guard_bytes = kGuardBytes;
+    out->total = L.total;
+    return STEPQ_OK;
+}
+
 stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t bytes, void *cuda_stream,
                                stepq_pool **out)
 {
@@ -361,8 +406,12 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
 
     const int H = desc->heads, B = desc->batch;
     const size_t HD = (size_t)H * kDK;
-    std::vector<uint8_t> host(L.total - L.off_rec, 0);
-    auto at = [&](size_t off) { return host.data() + (off - L.off_rec); };
+    std::vector<uint8_t> host(L.total - L.guard[0], 0);
+    auto at = [&](size_t off) { return host.data() + (off - L.guard[0]); };
+    for (int g = 0; g < kGuardRegions; g++) {
+        uint32_t *gw = reinterpret_cast<uint32_t *>(at(L.guard[g]));
+        for (int k = 0; k < (int)(kGuardBytes / 4); k++) gw[k] = guard_word(g, k);
+    }
     stepq::HeadRec *rec = reinterpret_cast<stepq::HeadRec *>(at(L.off_rec));
     long long *head_off = reinterpret_cast<long long *>(at(L.off_head_off));
     int *head_bytes = reinterpret_cast<int *>(at(L.off_head_bytes));
@@ -415,7 +464,7 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(cuda_stream);
     uint8_t *dev = static_cast<uint8_t *>(dev_buf);
-    cudaError_t e = cudaMemcpyAsync(dev + L.off_rec, host.data(), host.size(), cudaMemcpyHostToDevice, s);
+    cudaError_t e = cudaMemcpyAsync(dev + L.guard[0], host.data(), host.size(), cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return cuda_fail(e, "table upload");
     e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "table upload sync");
@@ -429,6 +478,8 @@ stepq_status stepq_pool_create(const stepq_desc *desc, void *dev_buf, size_t byt
     p->dev = dev;
     p->bytes = bytes;
     p->state_bytes = L.state;
+    for (int g = 0; g < kGuardRegions; g++) p->guard[g] = L.guard[g];
+    p->total = L.total;
     p->req_bytes = L.req_bytes;
     p->stream = s;
     p->t.rowrec = reinterpret_cast<const stepq::HeadRec *>(dev + L.off_rec);
@@ -668,9 +719,31 @@ stepq_status stepq_pool_check(stepq_pool *pool)
     if (code != 0) {
         const int zero = 0;
         cudaMemcpy(pool->t.status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        if (code == stepq::kStatusBadTable)
+            return fail(STEPQ_ERR_CUDA, "the checking build found a staging record or head record that does not "
+                                        "match the pool's layout (device status %d); no item was updated", code);
         return fail(STEPQ_ERR_CUDA, "a kernel gave up waiting for a staged copy (device status %d); "
                                     "the affected items were not updated", code);
     }
+    return STEPQ_OK;
+}
+
+stepq_status stepq_pool_check_guards(stepq_pool *pool)
+{
+    stepq_status st = check_pool(pool);
+    if (st != STEPQ_OK) return st;
+    cudaError_t e = cudaStreamSynchronize(pool->stream);
+    if (e != cudaSuccess) return cuda_fail(e, "stepq_pool_check_guards: stream");
+    uint32_t w[kGuardBytes / 4];
+    for (int g = 0; g < kGuardRegions; g++) {
+        e = cudaMemcpy(w, pool->dev + pool->guard[g], kGuardBytes, cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e, "stepq_pool_check_guards: read back");
+        for (int k = 0; k < (int)(kGuardBytes / 4); k++)
+            if (w[k] != guard_word(g, k))
+                return fail(STEPQ_ERR_STATE, "guard word %d after the %s changed: 0x%08x, expected 0x%08x", k,
+                            kGuardAfter[g], w[k], guard_word(g, k));
+    }
+    g_err.clear();
     return STEPQ_OK;
 }
 
@@ -1130,6 +1203,8 @@ stepq_status stepq_decode_step_noalloc(const stepq_desc *desc, void *states, siz
     a.t.status = reinterpret_cast<int *>(dsc + off_status);
     a.req_bytes = req;
     a.heads = H;
+    a.batch = B;
+    a.state_bytes = req * (long long)B;
     a.n_items = (int)n;
     a.ls_iters = desc->ls_iters;
     a.kda = kda;

@@ -81,6 +81,8 @@ struct StepArgs {
     int n_pivot_items;  // items of all-pivot heads, placed first in the order
     int max_n16;        // the most leading 16-bit field positions of any other head
     int scale_mode;     // kScaleDual (the method) or an ablation variant
+    int batch;                // requests of the pool (the layout's, also for an active subset)
+    long long state_bytes;    // bytes of the packed states (the checking build validates against it)
     const float *q, *k, *v, *alpha, *beta;
     float *out;
     const float *S_in;  // pack
@@ -90,6 +92,7 @@ struct StepArgs {
 // Device status codes.
 constexpr int kStatusWaitTimeout = 1;
 constexpr int kStatusBadHead = 2;
+constexpr int kStatusBadTable = 3;  // the checking build (STEPQ_CHECK) found an inconsistent table entry
 
 cudaError_t launch_decode_step(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_pack(const StepArgs &a, cudaStream_t s);

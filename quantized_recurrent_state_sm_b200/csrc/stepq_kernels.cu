@@ -762,6 +762,61 @@ __device__ __forceinline__ FitResult fit_and_store(ItemSmem &sm, RowFactors &rf,
     return abort_after ? kFitAbortAfter : kFitDone;
 }
 
+#ifndef STEPQ_CHECK
+#define STEPQ_CHECK 0
+#endif
+
+#if STEPQ_CHECK
+// Checking build: every head record against the head tables and the layout
+// (threads n < heads), every staging record n < n_pos against the order table,
+// the head tables and the packed states' extent.  Any mismatch sets the status
+// word; the kernels that read the tables then return without touching memory.
+__global__ void __launch_bounds__(256) k_check_tables(StepArgs a, int n_pos)
+{
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    bool bad = false;
+    if (n < a.heads) {
+        const HeadRec &R = a.t.rowrec[n];
+        const long long off = a.t.head_off[n];
+        const int hb = a.t.head_bytes[n], W = R.slab_words;
+        bad |= R.head_off != off || R.head_bytes != hb || off < 0 || off + hb > a.req_bytes;
+        bad |= hb != kHeaderBytes + 4 * W * kStreams * kSlabs;
+        if (R.head_kind == kHeadAllPivot) {
+            bad |= W != 2 * kRowsPerGroup;
+        } else {
+            int sum_f = 0;
+            for (int p = 0; p < kRowsPerGroup; p++) sum_f += R.pos_bits[p];
+            bad |= (R.head_b > 0) ? (W != 2 * R.head_b) : (W != (4 * sum_f + 31) / 32);
+        }
+    }
+    if (n < n_pos) {
+        const int4 st = a.t.stage[n];
+        const int item = st.x, h = (int)((uint32_t)st.y >> 16), bytes = st.y & 0xFFFF;
+        const long long off = (long long)(uint32_t)st.z << 10;
+        bad |= item < 0 || (long long)item >= (long long)a.batch * a.heads || h >= a.heads || h != item % a.heads ||
+               st.w != item / a.heads;
+        if (!bad) {
+            bad |= a.t.order[n] != item || bytes != a.t.head_bytes[h];
+            bad |= off != (long long)st.w * a.req_bytes + a.t.head_off[h] || off + bytes > a.state_bytes;
+            bad |= (n < a.n_pivot_items) != (a.t.rowrec[h].head_kind == kHeadAllPivot);
+        }
+    }
+    if (bad) atomicExch(a.t.status, kStatusBadTable);
+}
+
+// CTA-uniform: whether the status word is set (the kernel then returns).
+__device__ __forceinline__ bool tables_rejected(const StepArgs &a)
+{
+    return __syncthreads_or(threadIdx.x == 0 && *reinterpret_cast<volatile int *>(a.t.status) != 0);
+}
+#define STEPQ_RETURN_IF_REJECTED(a) \
+    if (tables_rejected(a)) return
+#else
+#define STEPQ_RETURN_IF_REJECTED(a) \
+    do {                            \
+    } while (0)
+#endif
+
 // ---------------------------------------------------------------------------
 // The fused decode step: persistent CTAs walk the item order.  Items of heads
 // whose rows are all FP16 pivots come first in the order and are processed
@@ -1128,6 +1183,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode(StepArgs a)
 {
     extern __shared__ __align__(128) uint8_t ring[];
     __shared__ ItemSmem sm;
+    STEPQ_RETURN_IF_REJECTED(a);
     const int tid = threadIdx.x;
     const int G = gridDim.x;
     if (tid == 0) {
@@ -1253,6 +1309,7 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads) k_pack(StepArgs a)
 {
     __shared__ ItemSmem sm;
+    STEPQ_RETURN_IF_REJECTED(a);
     RowFactors &rf = sm.u.rf[0];
     const int item = blockIdx.x;
     const int rq = item / a.heads, h = item - rq * a.heads;
@@ -1308,6 +1365,7 @@ __device__ __forceinline__ void unpack_body(const RowFactors &rf, const HeadRec 
 __global__ void __launch_bounds__(kThreads) k_unpack(StepArgs a)
 {
     __shared__ RowFactors rf;
+    STEPQ_RETURN_IF_REJECTED(a);
     const int item = blockIdx.x;
     const int rq = item / a.heads, h = item - rq * a.heads;
     const HeadRec *rec = a.t.rowrec + h;
@@ -1417,6 +1475,7 @@ __device__ __forceinline__ void split_update_body(const RowFactors &rf, const He
 __global__ void __launch_bounds__(kThreads) k_split_update(StepArgs a)
 {
     __shared__ RowFactors rf;
+    STEPQ_RETURN_IF_REJECTED(a);
     const int item = blockIdx.x;
     const int rq = item / a.heads, h = item - rq * a.heads;
     const HeadRec *rec = a.t.rowrec + h;
@@ -1676,9 +1735,22 @@ cudaError_t launch_calib_reduce(const CalibArgs &c, cudaStream_t s)
     return cudaGetLastError();
 }
 
+// Checking build: validate the tables the next launch reads (n_pos staging
+// records; the head records always).
+static inline void check_tables(const StepArgs &a, int n_pos, cudaStream_t s)
+{
+#if STEPQ_CHECK
+    const int n = n_pos > a.heads ? n_pos : a.heads;
+    k_check_tables<<<(n + 255) / 256, 256, 0, s>>>(a, n_pos);
+#else
+    (void)a, (void)n_pos, (void)s;
+#endif
+}
+
 cudaError_t launch_decode_step(const StepArgs &a, cudaStream_t s)
 {
     if (a.n_items == 0) return cudaSuccess;
+    check_tables(a, a.n_items, s);
     switch (a.scale_mode) {  // the variants fit without least squares: one instantiation each
         case kScaleRow: return launch_decode_m<false, kScaleRow>(a, s);
         case kScaleCol: return launch_decode_m<false, kScaleCol>(a, s);
@@ -1703,6 +1775,7 @@ int decode_ctas_per_sm(int nslots, int slot_bytes)
 cudaError_t launch_pack(const StepArgs &a, cudaStream_t s)
 {
     if (a.n_items == 0) return cudaSuccess;
+    check_tables(a, 0, s);
     switch (a.scale_mode) {
         case kScaleRow: k_pack<kScaleRow><<<a.n_items, kThreads, 0, s>>>(a); break;
         case kScaleCol: k_pack<kScaleCol><<<a.n_items, kThreads, 0, s>>>(a); break;
@@ -1715,6 +1788,7 @@ cudaError_t launch_pack(const StepArgs &a, cudaStream_t s)
 cudaError_t launch_split_update(const StepArgs &a, cudaStream_t s)
 {
     if (a.n_items == 0) return cudaSuccess;
+    check_tables(a, 0, s);
     k_split_update<<<a.n_items, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
@@ -1722,6 +1796,7 @@ cudaError_t launch_split_update(const StepArgs &a, cudaStream_t s)
 cudaError_t launch_unpack(const StepArgs &a, cudaStream_t s)
 {
     if (a.n_items == 0) return cudaSuccess;
+    check_tables(a, 0, s);
     k_unpack<<<a.n_items, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }

@@ -15,7 +15,10 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libstepq.so")
+# STEPQ_CHECK=1 in the environment selects the checking build (the kernels
+# validate the pool's tables before touching memory; include/stepq.h).
+CHECK_BUILD = os.environ.get("STEPQ_CHECK", "0") == "1"
+LIB_PATH = os.path.join(_HERE, "libstepq_check.so" if CHECK_BUILD else "libstepq.so")
 
 GDN, KDA = 0, 1
 SCALE_DUAL, SCALE_ROW, SCALE_COL, SCALE_HEAD = 0, 1, 2, 3
@@ -36,6 +39,13 @@ class Desc(C.Structure):
                 ("dv", C.c_int), ("ls_iters", C.c_int), ("bits", C.c_void_p), ("rho", C.c_void_p)]
 
 
+class Regions(C.Structure):
+    _fields_ = [("states", C.c_size_t), ("state_bytes", C.c_size_t), ("head_records", C.c_size_t),
+                ("head_offsets", C.c_size_t), ("item_sizes", C.c_size_t), ("status_word", C.c_size_t),
+                ("item_order", C.c_size_t), ("staging_records", C.c_size_t), ("guards", C.c_size_t * 7),
+                ("guard_bytes", C.c_size_t), ("total", C.c_size_t)]
+
+
 class CalibDesc(C.Structure):
     _fields_ = [("variant", C.c_int), ("batch", C.c_int), ("heads", C.c_int), ("dk", C.c_int),
                 ("dv", C.c_int), ("steps", C.c_int), ("sample_every", C.c_int), ("ls_iters", C.c_int),
@@ -43,7 +53,7 @@ class CalibDesc(C.Structure):
                 ("pivot_frac", C.c_double)]
 
 
-EXPORTS = ("stepq_pool_bytes", "stepq_state_bytes", "stepq_pool_create", "stepq_pool_destroy",
+EXPORTS = ("stepq_pool_bytes", "stepq_state_bytes", "stepq_pool_layout", "stepq_pool_check_guards", "stepq_pool_create", "stepq_pool_destroy",
            "stepq_pool_set_stream", "stepq_pack", "stepq_unpack", "stepq_decode_step",
            "stepq_fp32_step", "stepq_pool_check", "stepq_status_string", "stepq_last_error",
            "stepq_decode_step_noalloc", "stepq_decode_step_split", "stepq_pool_set_active",
@@ -63,6 +73,8 @@ def _load():
     L.stepq_pool_destroy.argtypes = [P]
     L.stepq_pool_set_stream.argtypes = [P, P]
     L.stepq_pool_check.argtypes = [P]
+    L.stepq_pool_check_guards.argtypes = [P]
+    L.stepq_pool_layout.argtypes = [D, C.POINTER(Regions)]
     L.stepq_pack.argtypes = [P, P]
     L.stepq_unpack.argtypes = [P, P]
     L.stepq_decode_step.argtypes = [P, P, P, P, P, P, P]
@@ -235,6 +247,20 @@ class PackedStatePool:
         """Synchronise the pool's stream and raise if a kernel reported an error."""
         self._sync_stream()
         _check(lib.stepq_pool_check(self._h))
+
+    def check_guards(self):
+        """Raise if a guard word after any region of the pool buffer changed."""
+        self._sync_stream()
+        _check(lib.stepq_pool_check_guards(self._h))
+
+    @property
+    def regions(self) -> dict:
+        """Byte offsets of the buffer's regions (stepq_pool_layout)."""
+        r = Regions()
+        _check(lib.stepq_pool_layout(C.byref(self._desc), C.byref(r)))
+        out = {f: getattr(r, f) for f, _ in Regions._fields_ if f != "guards"}
+        out["guards"] = list(r.guards)
+        return out
 
     def close(self):
         if getattr(self, "_h", None):

@@ -160,3 +160,28 @@ def test_layout_agrees_across_implementations(S):
         assert total == 3 * sum(per_head), trial
         d, keep = S.make_desc(S.KDA, 3, H, bits, rho)
         assert S.lib.stepq_state_bytes(C.byref(d)) == total, trial
+
+
+def test_pool_layout_regions_and_guards(S):
+    """stepq_pool_layout: the packed states first, then each table, every
+    region followed by its guard region, in order and without overlap; the
+    total is stepq_pool_bytes and the states' extent stepq_state_bytes."""
+    for ci in range(5):
+        cfg = W.with_overrides(W.CONFIGS[ci], batch=3)
+        bits, rho = W.bit_table(cfg), W.rho(cfg)
+        d, keep = S.make_desc(cfg.variant, cfg.batch, cfg.heads, bits, rho)
+        r = S.Regions()
+        assert S.lib.stepq_pool_layout(C.byref(d), C.byref(r)) == S.OK
+        H, n = cfg.heads, cfg.items
+        assert r.states == 0 and r.state_bytes == S.lib.stepq_state_bytes(C.byref(d))
+        assert r.total == S.lib.stepq_pool_bytes(C.byref(d))
+        g = list(r.guards)
+        sizes = [r.state_bytes, None, 8 * H, 4 * H, 4, 4 * n, 16 * n]
+        starts = [r.states, r.head_records, r.head_offsets, r.item_sizes, r.status_word, r.item_order,
+                  r.staging_records]
+        for k in range(7):
+            if sizes[k] is not None:
+                assert starts[k] + sizes[k] <= g[k], (ci, k)
+            assert g[k] % 16 == 0 and g[k] + r.guard_bytes <= (starts[k + 1] if k < 6 else r.total), (ci, k)
+        assert starts[1] % 256 == 0 and all(x % 16 == 0 for x in starts)
+    assert S.lib.stepq_pool_layout(None, C.byref(r)) == S.ERR_INVALID_ARG

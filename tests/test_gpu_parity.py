@@ -68,10 +68,11 @@ class Setup:
         return self.bits[self.slots[s] % self.cfg.heads]
 
 
-def lockstep(setup, steps, t0=0, full_inputs=True, step=None):
+def lockstep(setup, steps, t0=0, full_inputs=True, step=None, S0=None):
     cfg = setup.cfg
     cmp = PoolComparison()
-    S0 = oracle.initial_state(cfg, setup.req)
+    if S0 is None:
+        S0 = oracle.initial_state(cfg, setup.req)
     setup.ref.pack(S0.reshape(-1, 128, 128))
     worst = 0.0
     for t in range(t0, t0 + steps):
@@ -142,6 +143,38 @@ def test_lockstep_config3_full_size_sampled():
     cfg = W.CONFIGS[3]
     cmp, worst = lockstep(Setup(cfg, W.parity_requests(cfg)), steps=2, t0=500)
     print(f"config 3: {cmp.diff}/{cmp.codes} codes differ, worst readout {worst:.2e}")
+
+
+def long_rollout_state(cfg, requests, steps):
+    """The oracle's unquantised fp32 recursion from the initial state over the
+    first `steps` steps, for the given requests: [R, H, dk, dv]."""
+    S = oracle.initial_state(cfg, requests)
+    R, H = S.shape[:2]
+    Sf = np.ascontiguousarray(S.reshape(R * H, 128, 128))
+    kda = cfg.variant == W.KDA
+    for t in range(steps):
+        x = W.step_inputs(cfg, t, requests)
+        oracle.fp32_step(Sf, x["q"].reshape(R * H, -1), x["k"].reshape(R * H, -1), x["v"].reshape(R * H, -1),
+                         x["alpha"].reshape(R * H, -1) if kda else x["alpha"].reshape(-1), x["beta"].reshape(-1),
+                         kda=kda)
+    return Sf.reshape(R, H, 128, 128)
+
+
+@pytest.mark.parametrize("ci", [3, 4])
+def test_lockstep_from_long_rollout_state(ci):
+    """Lockstep from the state of each configuration's full-length unquantised
+    rollout (1024 steps for config 3, 2048 for config 4, where the 30x key and
+    value channels have grown their outlier rows and columns), 8 steps, on the
+    full batch with the oracle on requests {0, 1, B/2, B-1}: the parity rules
+    hold at the magnitudes and clip rates of a long rollout."""
+    cfg = W.CONFIGS[ci]
+    req = W.parity_requests(cfg)
+    S_T = long_rollout_state(cfg, req, cfg.steps)
+    su = Setup(cfg, req)
+    cmp, worst = lockstep(su, steps=8, t0=cfg.steps, S0=S_T)
+    rms = np.sqrt(np.mean(S_T.astype(np.float64) ** 2, axis=3))  # row RMS, [R, H, dk]
+    print(f"config {ci} after {cfg.steps} steps: row RMS max/median {np.median(rms.max(-1) / np.median(rms, -1)):.1f}; "
+          f"{cmp.diff}/{cmp.codes} codes differ, worst readout {worst:.2e}")
 
 
 def test_every_width_and_pivot_rows_kda():
