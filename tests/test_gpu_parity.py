@@ -23,7 +23,7 @@ else:  # pragma: no cover
 
 
 def to_dev(x):
-    return {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in x.items()}
+    return {k: torch.from_numpy(np.array(v, copy=True)).cuda() for k, v in x.items()}
 
 
 class Setup:
@@ -287,9 +287,30 @@ def test_invalid_arguments_are_rejected_on_the_host():
     torch.cuda.synchronize()  # the context is still healthy
 
 
-@pytest.mark.parametrize("ci,ls", [(1, 2), (2, 0), (2, 3)])
+@pytest.mark.parametrize("ci,ls", [(1, 0), (1, 2), (3, 3), (2, 0), (2, 3)])
 def test_least_squares_round_counts(ci, ls):
     """0 rounds (maximum-based column scales), and several rounds (later
     rounds clip to the row's range)."""
     cfg = W.with_overrides(W.CONFIGS[ci], batch=2, ls_iters=ls)
     lockstep(Setup(cfg), steps=2, t0=7)
+
+
+def test_every_width_gdn():
+    """Gated-DeltaNet heads of every width 2..8 (one instantiation of the
+    fused kernel per width) and an all-pivot head in one pool, lockstep."""
+    widths = [2, 3, 4, 5, 6, 7, 8, 16]
+    cfg = W.with_overrides(W.CONFIGS[1], batch=3, heads=len(widths))
+    bits = np.repeat(np.array(widths, np.uint8)[:, None], 128, axis=1)
+    cmp, worst = lockstep(Setup(cfg, bits=bits), steps=4, t0=3)
+    print(f"widths {widths}: {cmp.diff}/{cmp.codes} codes differ, worst readout {worst:.2e}")
+
+
+@pytest.mark.parametrize("ci,batch,heads", [(0, 1, 1), (1, 5, 3), (2, 1, 1), (2, 7, 5), (4, 3, 33)])
+def test_odd_shapes(ci, batch, heads):
+    """One request of one head, and item counts that fill the persistent grid
+    unevenly (the configuration's generators at that head count; no pivot
+    head where a 16-bit unit would not fit the bit budget of so few heads)."""
+    cfg = W.with_overrides(W.CONFIGS[ci], batch=batch, heads=heads)
+    if cfg.variant == W.GDN and heads < 8:
+        cfg = W.with_overrides(cfg, pivot_frac=0.0)
+    lockstep(Setup(cfg), steps=3, t0=11)
