@@ -140,7 +140,7 @@ def drift(request):
 
 
 def test_drift_within_stated_tolerance(drift):
-    """The benchmark spec's criterion, |D_gpu - D_or| <= 1e-3 D_or at every checkpoint,
+    """The stated drift tolerance, |D_gpu - D_or| <= 1e-3 D_or at every checkpoint,
     wherever the oracle meets it against itself.  Where two equally valid
     oracle rollouts of the sample (one code of every item nudged by one step
     at the start) already differ by more than 1e-3 at some checkpoint, no
