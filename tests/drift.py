@@ -44,7 +44,7 @@ def _group(args):
     heads = np.asarray(heads)
     pool = oracle.SlotPool(heads, bits, rho, ls_iters=cfg.ls_iters, kda=kda)
     pool.pool[:] = s0_bytes
-    S = pool.unpack()  # the fp32 recursion starts from the same state as the GPU's, S0
+    # the fp32 recursion starts from the same full-precision state as the GPU's, S0
     Sf = np.ascontiguousarray(oracle.initial_state(cfg, [req])[0][heads])
     pools = [pool]
     if perturb:
@@ -52,7 +52,6 @@ def _group(args):
         P.pool[:] = pool.pool
         _perturb(P, bits, seed=1000 * req + int(heads[0]))
         pools.append(P)
-    del S
     rows = []
     for t in range(steps):
         x = W.step_inputs(cfg, t, [req])
