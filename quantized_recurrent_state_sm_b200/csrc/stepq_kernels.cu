@@ -1627,17 +1627,18 @@ __global__ void __launch_bounds__(kDK) k_calib_accumulate(CalibArgs c)
     }
 }
 
+// One candidate width of the calibration's per-row errors; the thread's 64
+// state values come from its own block of the shared-memory copy (`own`,
+// value rr at own[rr * kThreads]: a warp's lanes read consecutive 16-byte
+// chunks).
 template <int B, bool MULTI>
 __device__ __forceinline__ void calib_width(ItemSmem &sm, RowFactors &rf, const HeadRec *rec, const CalibArgs &c,
-                                            int item, int x)
+                                            int item, int x, const float4 *own)
 {
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31, rg = l & 7, cg = l >> 3;
-    const int col0 = 16 * w + 4 * cg;
     X2 X;
-    const float *src = c.S + (long long)item * kDK * kDV;
 #pragma unroll
     for (int rr = 0; rr < kRowsPerGroup; rr++) {
-        const float4 v = ld4(src + (kRowsPerGroup * rg + rr) * kDV + col0);
+        const float4 v = own[rr * kThreads];
         X[rr][0] = f2(v.x, v.y);
         X[rr][1] = f2(v.z, v.w);
     }
@@ -1647,13 +1648,29 @@ __device__ __forceinline__ void calib_width(ItemSmem &sm, RowFactors &rf, const 
                                                   c.ls_iters, true, true, NoMid{}, c.err + o * kDK);
 }
 
+// The state is copied once per CTA into shared memory (each thread its own 16
+// rows x 4 columns, 256 bytes, by asynchronous copies; 64 KiB of dynamic
+// shared memory per CTA), so that the candidate widths after the first reload
+// it from there instead of from L2.
 template <bool MULTI>
 __global__ void __launch_bounds__(kThreads) k_calib_error(CalibArgs c)
 {
+    extern __shared__ __align__(16) float4 state_copy[];
     __shared__ ItemSmem sm;
     __shared__ HeadRec rec;
     RowFactors &rf = sm.u.rf[0];
     const int item = blockIdx.x, h = item % c.heads, tid = threadIdx.x;
+    float4 *own = state_copy + tid;
+    {
+        const int w = tid >> 5, l = tid & 31, rg = l & 7, cg = l >> 3;
+        const float *src = c.S + (long long)item * kDK * kDV + (kRowsPerGroup * rg) * kDV + 16 * w + 4 * cg;
+#pragma unroll
+        for (int rr = 0; rr < kRowsPerGroup; rr++)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(own + rr * kThreads)),
+                         "l"(src + rr * kDV)
+                         : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
     float s_i = 0.f, rho_i = 0.f;
     __shared__ float rho_wmax[kThreads / 32];
     if (tid < kDK) rho_i = c.rho[h * kDK + tid];
@@ -1687,16 +1704,18 @@ __global__ void __launch_bounds__(kThreads) k_calib_error(CalibArgs c)
             rec.n16 = 0;
         }
         __syncthreads();
+        if (x == 0) asm volatile("cp.async.wait_all;" ::: "memory");  // the thread's own copy has landed
         switch (b) {
-            case 2: calib_width<2, MULTI>(sm, rf, &rec, c, item, x); break;
-            case 3: calib_width<3, MULTI>(sm, rf, &rec, c, item, x); break;
-            case 4: calib_width<4, MULTI>(sm, rf, &rec, c, item, x); break;
-            case 5: calib_width<5, MULTI>(sm, rf, &rec, c, item, x); break;
-            case 6: calib_width<6, MULTI>(sm, rf, &rec, c, item, x); break;
-            case 7: calib_width<7, MULTI>(sm, rf, &rec, c, item, x); break;
-            default: calib_width<8, MULTI>(sm, rf, &rec, c, item, x); break;  // widths are validated on the host
+            case 2: calib_width<2, MULTI>(sm, rf, &rec, c, item, x, own); break;
+            case 3: calib_width<3, MULTI>(sm, rf, &rec, c, item, x, own); break;
+            case 4: calib_width<4, MULTI>(sm, rf, &rec, c, item, x, own); break;
+            case 5: calib_width<5, MULTI>(sm, rf, &rec, c, item, x, own); break;
+            case 6: calib_width<6, MULTI>(sm, rf, &rec, c, item, x, own); break;
+            case 7: calib_width<7, MULTI>(sm, rf, &rec, c, item, x, own); break;
+            default: calib_width<8, MULTI>(sm, rf, &rec, c, item, x, own); break;  // widths are validated on the host
         }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // (no width: the copy lands before the CTA ends)
 }
 
 __global__ void __launch_bounds__(kDK) k_calib_reduce(CalibArgs c)
@@ -1721,10 +1740,15 @@ cudaError_t launch_calib_error(const CalibArgs &c, cudaStream_t s)
 {
     const long long n = (long long)c.batch * c.heads;
     if (n == 0 || c.n_widths == 0) return cudaSuccess;
+    constexpr int dyn = kThreads * kRowsPerGroup * (int)sizeof(float4);  // the state copy, 64 KiB
+    cudaError_t e = cudaFuncSetAttribute(k_calib_error<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_calib_error<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    if (e != cudaSuccess) return e;
     if (c.ls_iters <= 1)
-        k_calib_error<false><<<(unsigned)n, kThreads, 0, s>>>(c);
+        k_calib_error<false><<<(unsigned)n, kThreads, dyn, s>>>(c);
     else
-        k_calib_error<true><<<(unsigned)n, kThreads, 0, s>>>(c);
+        k_calib_error<true><<<(unsigned)n, kThreads, dyn, s>>>(c);
     return cudaGetLastError();
 }
 
