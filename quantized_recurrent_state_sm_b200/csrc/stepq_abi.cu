@@ -145,6 +145,7 @@ int fill_rows(const stepq_desc *d, int h, stepq::HeadRec &R)
     R.n16 = 0;
     for (int p = 0; p < stepq::kRowsPerGroup; p++) {
         R.pos_bits[p] = (uint8_t)F[p];
+        R.pos_off[p] = (uint16_t)(p == 0 ? 0 : R.pos_off[p - 1] + 4 * F[p - 1]);
         R.n16 += F[p] == STEPQ_PIVOT_BITS;
     }
     R.pad = 0;

@@ -43,6 +43,9 @@ struct HeadRec {
     // lays out its fields alike.  Positions of 16-bit fields (pivot rows)
     // come first: n16 of them.
     uint8_t pos_bits[kRowsPerGroup];
+    // bit offset of row position p in every stream: 4 x the sum of the
+    // widths of the positions before it (a per-head constant)
+    uint16_t pos_off[kRowsPerGroup];
     long long head_off;          // byte offset of the head's item inside a request
     int head_b;                  // common row width, 0 if the rows differ
     int head_kind;               // kHeadQuant / kHeadAllPivot / kHeadMixed

@@ -145,8 +145,7 @@ struct alignas(16) RowFactors {
 // Thread p < 16: position p of the head's table (row-wise widths).
 __device__ __forceinline__ void make_pos(RowFactors &rf, const HeadRec *rec, int p)
 {
-    int O = 0;
-    for (int q = 0; q < p; q++) O += 4 * rec->pos_bits[q];
+    const int O = rec->pos_off[p];
     const int F = rec->pos_bits[p], W = rec->slab_words, m = O >> 5, sh = O & 31;
     PosRec r;
     r.w0 = m * kStreams;
@@ -785,7 +784,10 @@ __global__ void __launch_bounds__(256) k_check_tables(StepArgs a, int n_pos)
             bad |= W != 2 * kRowsPerGroup;
         } else {
             int sum_f = 0;
-            for (int p = 0; p < kRowsPerGroup; p++) sum_f += R.pos_bits[p];
+            for (int p = 0; p < kRowsPerGroup; p++) {
+                bad |= R.pos_off[p] != 4 * sum_f;
+                sum_f += R.pos_bits[p];
+            }
             bad |= (R.head_b > 0) ? (W != 2 * R.head_b) : (W != (4 * sum_f + 31) / 32);
         }
     }
