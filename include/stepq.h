@@ -333,8 +333,7 @@ STEPQ_API stepq_status stepq_pool_check_guards(stepq_pool *pool);
  * Calls share the one scratch array per device: two calls in flight at the
  * same time (on different streams or threads) race on it, so order them on
  * one stream.  The first call on a device looks up the scratch address
- * (cudaGetSymbolAddress) and should come before any stream capture.  The
- * status word the kernel writes when a staged copy never lands is cleared by
+ * (cudaGetSymbolAddress).  The status word the kernel writes when a staged copy never lands is cleared by
  * the next call and not reported here; use a pool and stepq_pool_check where
  * that report is needed.
  */
