@@ -118,9 +118,25 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
-        self.idx = gpu_index
+    def __init__(self, device):
+        self.idx = self.smi_id(device)
         self.proc = None
+
+    @staticmethod
+    def smi_id(device):
+        """nvidia-smi's name for CUDA device `device` (its UUID), so that the
+        samples follow the device this process runs on under any
+        CUDA_VISIBLE_DEVICES mapping; the ordinal if the UUID is unavailable."""
+        try:
+            import torch
+            ident = f"GPU-{torch.cuda.get_device_properties(device).uuid}"
+            r = subprocess.run(["nvidia-smi", f"--id={ident}", "--query-gpu=index", "--format=csv,noheader"],
+                               capture_output=True, text=True, timeout=20)
+            if r.returncode == 0 and r.stdout.strip():
+                return ident
+        except Exception:
+            pass
+        return str(device)
 
     def __enter__(self):
         try:
@@ -163,7 +179,7 @@ class ClockSampler:
 SOAK_S = 0.5  # seconds of the same, untimed steps before and after the timed region
 
 
-def loaded_window(step, stream, n_steps, sampler_index, soak_s=SOAK_S, barrier=None):
+def loaded_window(step, stream, n_steps, device, soak_s=SOAK_S, barrier=None):
     """Time exactly n_steps calls of step(i) with CUDA events on `stream`,
     bracketed by a device synchronize (and `barrier`, every rank's) on both
     sides, inside a window in which the GPU runs the same steps, untimed, for
@@ -182,7 +198,7 @@ def loaded_window(step, stream, n_steps, sampler_index, soak_s=SOAK_S, barrier=N
     per = max(c0.elapsed_time(c1) / 5, 1e-3)
     n_soak = int(min(200000, max(1, soak_s * 1e3 / per))) if soak_s > 0 else 0
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(sampler_index) as clocks:
+    with ClockSampler(device) as clocks:
         time.sleep(0.1)  # the sampler is up
         for i in range(n_soak):
             step(i)
@@ -723,7 +739,7 @@ def run_all_configs(args):
 
         for i in range(3):
             fstep(i)
-        fp32_ms, _ = loaded_window(fstep, stream, args.steps, 0, soak_s=0.1)
+        fp32_ms, _ = loaded_window(fstep, stream, args.steps, torch.cuda.current_device(), soak_s=0.1)
         fp32_ms /= args.steps
         del S_tmp
         pool.pack(S)
@@ -734,7 +750,7 @@ def run_all_configs(args):
 
         for i in range(max(3, args.warmup)):
             step(i)
-        ms, clocks = loaded_window(step, stream, args.steps, 0, soak_s=0.25)
+        ms, clocks = loaded_window(step, stream, args.steps, torch.cuda.current_device(), soak_s=0.25)
         ms_per_step = ms / args.steps
         finite = bool(torch.isfinite(out).all())
         pool.check()
