@@ -160,13 +160,14 @@ def long_rollout_state(cfg, requests, steps):
     return Sf.reshape(R, H, 128, 128)
 
 
-@pytest.mark.parametrize("ci", [3, 4])
+@pytest.mark.parametrize("ci", [0, 1, 2, 3, 4])
 def test_lockstep_from_long_rollout_state(ci):
     """Lockstep from the state of each configuration's full-length unquantised
-    rollout (1024 steps for config 3, 2048 for config 4, where the 30x key and
-    value channels have grown their outlier rows and columns), 8 steps, on the
-    full batch with the oracle on requests {0, 1, B/2, B-1}: the parity rules
-    hold at the magnitudes and clip rates of a long rollout."""
+    rollout (64 steps for config 0, 256 for configs 1 and 2, 1024 for config
+    3, 2048 for config 4, where the 30x key and value channels have grown
+    their outlier rows and columns), 8 steps, on the full batch with the
+    oracle on requests {0, 1, B/2, B-1}: the parity rules hold at the
+    magnitudes and clip rates of a long rollout."""
     cfg = W.CONFIGS[ci]
     req = W.parity_requests(cfg)
     S_T = long_rollout_state(cfg, req, cfg.steps)
