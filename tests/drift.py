@@ -101,3 +101,40 @@ def oracle_drift(ci, requests, bits, rho, s0_items, steps, every=64, perturb=Tru
         errp = np.sum([[r[3] for r in g] for g in res], axis=0)
         D_p = np.sqrt(errp / ref)
     return T, D_or, D_p
+
+
+def _group_bytes(args):
+    """One request's heads `heads` over steps 0 .. steps-1 of the packed
+    recursion from the packed S0: the final packed bytes of each item."""
+    ci, overrides, req, heads, steps, bits, rho, s0_bytes = args
+    import oracle
+    from quantized_recurrent_state_sm_b200 import workload as W
+    cfg = W.with_overrides(W.CONFIGS[ci], **overrides) if overrides else W.CONFIGS[ci]
+    kda = cfg.variant == W.KDA
+    heads = np.asarray(heads)
+    pool = oracle.SlotPool(heads, bits, rho, ls_iters=cfg.ls_iters, kda=kda)
+    pool.pool[:] = s0_bytes
+    for t in range(steps):
+        x = W.step_inputs(cfg, t, [req])
+        pool.step(x["q"][0][heads], x["k"][0][heads], x["v"][0][heads], x["alpha"][0][heads],
+                  x["beta"][0][heads])
+    return [(req, int(h), pool.item(s).copy()) for s, h in enumerate(heads)]
+
+
+def oracle_rollout_bytes(ci, requests, bits, rho, s0_items, steps, overrides=None, workers=None):
+    """The oracle's packed recursion over requests x all heads from the packed
+    bytes s0_items[(req, h)]: {(req, h): packed bytes after `steps` steps}."""
+    from quantized_recurrent_state_sm_b200 import workload as W
+    cfg = W.with_overrides(W.CONFIGS[ci], **overrides) if overrides else W.CONFIGS[ci]
+    H = cfg.heads
+    workers = workers or max(1, min(32, os.cpu_count() or 1))
+    per = max(1, -(-H // max(1, -(-workers // len(requests)))))
+    jobs = []
+    for req in requests:
+        for h0 in range(0, H, per):
+            hs = list(range(h0, min(H, h0 + per)))
+            s0 = np.concatenate([s0_items[(req, h)] for h in hs])
+            jobs.append((ci, overrides, int(req), hs, steps, bits, rho, s0))
+    with mp.get_context("spawn").Pool(min(workers, len(jobs))) as pool:
+        res = pool.map(_group_bytes, jobs)
+    return {(r, h): b for group in res for (r, h, b) in group}

@@ -68,12 +68,19 @@ class Setup:
         return self.bits[self.slots[s] % self.cfg.heads]
 
 
-def lockstep(setup, steps, t0=0, full_inputs=True, step=None, S0=None):
+def lockstep(setup, steps, t0=0, full_inputs=True, step=None, S0=None, ref_bytes=None):
+    """`steps` steps from step t0 with the oracle's bytes pushed before each;
+    the oracle's pool starts from S0 packed (default: the initial state) or
+    from ref_bytes[(request, head)]."""
     cfg = setup.cfg
     cmp = PoolComparison()
-    if S0 is None:
-        S0 = oracle.initial_state(cfg, setup.req)
-    setup.ref.pack(S0.reshape(-1, 128, 128))
+    if ref_bytes is not None:
+        for s, slot in enumerate(setup.slots):
+            setup.ref.set_item(s, ref_bytes[(int(slot // cfg.heads), int(slot % cfg.heads))])
+    else:
+        if S0 is None:
+            S0 = oracle.initial_state(cfg, setup.req)
+        setup.ref.pack(S0.reshape(-1, 128, 128))
     worst = 0.0
     for t in range(t0, t0 + steps):
         setup.push_oracle_bytes()
@@ -176,6 +183,28 @@ def test_lockstep_from_long_rollout_state(ci):
     rms = np.sqrt(np.mean(S_T.astype(np.float64) ** 2, axis=3))  # row RMS, [R, H, dk]
     print(f"config {ci} after {cfg.steps} steps: row RMS max/median {np.median(rms.max(-1) / np.median(rms, -1)):.1f}; "
           f"{cmp.diff}/{cmp.codes} codes differ, worst readout {worst:.2e}")
+
+
+@pytest.mark.parametrize("ci", [0, 1, 2, 3, 4])
+def test_lockstep_from_packed_rollout_state(ci):
+    """Lockstep from the oracle's own packed state after each configuration's
+    full-length requantised rollout (every step fitted, rounded and packed, so
+    the codes carry the accumulated requantisation structure), 8 steps, on the
+    full batch with the oracle on requests {0, 1, B/2, B-1}."""
+    from tests.drift import oracle_rollout_bytes
+    cfg = W.CONFIGS[ci]
+    req = W.parity_requests(cfg)
+    bits, rho = W.bit_table(cfg), W.rho(cfg)
+    S0 = oracle.initial_state(cfg, req)
+    s0 = {}
+    for a, r in enumerate(req):
+        for h in range(cfg.heads):
+            f = oracle.fit_quantise(S0[a, h], bits[h], rho[h], cfg.ls_iters)
+            s0[(int(r), h)] = oracle.pack_item(bits[h], f["r"], f["c"], f["code"], f["piv"])
+    final = oracle_rollout_bytes(ci, [int(r) for r in req], bits, rho, s0, cfg.steps)
+    cmp, worst = lockstep(Setup(cfg, req), steps=8, t0=cfg.steps, ref_bytes=final)
+    print(f"config {ci} from the packed state after {cfg.steps} steps: {cmp.diff}/{cmp.codes} codes differ, "
+          f"worst readout {worst:.2e}")
 
 
 def test_every_width_and_pivot_rows_kda():
