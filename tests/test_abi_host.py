@@ -78,6 +78,22 @@ def test_descriptor_validation(S):
     d.bits = None
     assert S.lib.stepq_pool_bytes(C.byref(d)) == 0
     assert S.lib.stepq_pool_bytes(None) == 0
+    # the limits: batch x heads up to 2^24 items, heads up to 65535 (the
+    # staging records hold a head in 16 bits)
+    top = (1 << 24) // cfg.heads
+    d, keep = S.make_desc(cfg.variant, top, cfg.heads, bits, rho)
+    states = S.lib.stepq_state_bytes(C.byref(d))
+    assert states == top * int(W.head_item_bytes(bits, cfg.dv).sum())  # ~0.2 TB: 64-bit sizes
+    assert S.lib.stepq_pool_bytes(C.byref(d)) > states
+    n, msg = nbytes(batch=top + 1)
+    assert n == 0 and "exceeds" in msg
+    H = 65536
+    hb = np.full((H, 128), 6, np.uint8)
+    hr = np.ones((H, 128), np.float32)
+    d, keep = S.make_desc(cfg.variant, 1, H, hb, hr)
+    assert S.lib.stepq_pool_bytes(C.byref(d)) == 0 and "65535" in S.lib.stepq_last_error().decode()
+    d, keep = S.make_desc(cfg.variant, 1, H - 1, hb[:H - 1], hr[:H - 1])
+    assert S.lib.stepq_pool_bytes(C.byref(d)) > 0
 
 
 def test_null_and_dead_handles(S):
