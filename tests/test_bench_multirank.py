@@ -54,3 +54,18 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(3.5, 1, "cpu") == 3.5
     assert bench.whole_job_rate(1, 100, 10, 1.0) == pytest.approx(1e6)
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    """Under torchrun the reference arm (the oracle on the host cores) runs
+    and prints on rank 0 alone; every other rank exits 0 without work."""
+    import types
+
+    import bench
+    from quantized_recurrent_state_sm_b200 import workload as W
+    monkeypatch.setenv("RANK", "1")
+    called = []
+    monkeypatch.setattr(bench, "cpu_oracle_rate", lambda *a, **k: called.append(a) or (1.0, {}))
+    args = types.SimpleNamespace(steps=3, warmup=3, gpus=2, cpu_seconds=1.0)
+    assert bench.run_reference(args, W.CONFIGS[3]) == 0
+    assert not called and capsys.readouterr().out == ""
