@@ -54,3 +54,38 @@ def test_inconsistent_staging_record_is_rejected():
     pool.check()  # the status word was cleared; the restored tables pass
     pool.check_guards()
     assert not torch.equal(pool.state, before)
+
+
+def test_inconsistent_position_offset_is_rejected():
+    """A KDA head record whose stored bit offset of a row position disagrees
+    with the position widths is rejected before any kernel reads a stream."""
+    cfg = W.with_overrides(W.CONFIGS[2], batch=2)
+    bits = W.bit_table(cfg)
+    pool = stepq.PackedStatePool(cfg.variant, cfg.batch, cfg.heads, bits, W.rho(cfg))
+    pool.pack(torch.from_numpy(oracle.initial_state(cfg)).cuda())
+    x = {k: torch.from_numpy(v).cuda() for k, v in W.step_inputs(cfg, 0).items()}
+    F = W.position_widths(bits[0])
+    offs = np.concatenate([[0], np.cumsum(4 * F[:-1])]).astype("<u2")
+    r0 = pool.regions["head_records"]
+    head0 = pool.buffer[r0:r0 + 4096].cpu().numpy().tobytes()  # the first head's record lies in here
+    at = head0.find(offs.tobytes())
+    assert at >= 0 and head0.find(offs.tobytes(), at + 1) < 0  # the offsets, found once
+    at = r0 + at + 2 * 5  # position 5
+    saved = pool.buffer[at:at + 2].clone()
+    bad = offs.copy()
+    bad[5] += 4
+    pool.buffer[at:at + 2] = torch.from_numpy(bad[5:6].view(np.uint8).copy()).cuda()
+    before = pool.state.clone()
+    out = torch.full((cfg.batch, cfg.heads, 128), -3.0, device="cuda")
+    pool.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], out)
+    torch.cuda.synchronize()
+    try:
+        pool.check()
+        raise AssertionError("the inconsistent position offset was not reported")
+    except stepq.StepqError as e:
+        assert "checking build" in str(e)
+    assert torch.equal(pool.state, before) and bool((out == -3.0).all())
+    pool.buffer[at:at + 2] = saved
+    pool.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], out)
+    pool.check()
+    pool.check_guards()
