@@ -281,6 +281,22 @@ STEPQ_API stepq_status stepq_fp32_step(const stepq_desc *desc, float *S, const f
 STEPQ_API stepq_status stepq_pool_check(stepq_pool *pool);
 
 /*
+ * Failure-detection self-test (no counterpart on the pages): one CTA runs the
+ * bounded barrier wait the decode kernel uses for its staged copies, on a
+ * barrier that needs one arrival.  With arrive != 0 the thread arrives first
+ * and the wait completes; with arrive == 0 nothing arrives and the wait gives
+ * up after limit_cycles SM clock cycles, as a wait for a copy that never lands
+ * would.  result: device int[2], written with result[0] = 0 (completed) or 1
+ * (gave up: the decode kernel's timeout status) and result[1] = cycles spent
+ * waiting (saturated at 2^31 - 1).  limit_cycles in [0, 2^34] (up to about 8 s
+ * at the B200's clock), else STEPQ_ERR_INVALID_ARG.  Asynchronous on
+ * cuda_stream (cudaStream_t or NULL); nothing else is touched, so the context
+ * stays usable after a wait that gave up.
+ */
+STEPQ_API stepq_status stepq_selftest_bounded_wait(int *result, long long limit_cycles, int arrive,
+                                                   void *cuda_stream);
+
+/*
  * Memory-safety aid (no counterpart on the pages): synchronise the pool's
  * stream and compare the guard regions that follow every region of the pool
  * buffer (see stepq_pool_layout) with the pattern pool creation wrote.  A

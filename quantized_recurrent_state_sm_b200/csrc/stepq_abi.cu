@@ -729,6 +729,18 @@ stepq_status stepq_pool_check(stepq_pool *pool)
     return STEPQ_OK;
 }
 
+stepq_status stepq_selftest_bounded_wait(int *result, long long limit_cycles, int arrive, void *cuda_stream)
+{
+    if (!result) return fail(STEPQ_ERR_INVALID_ARG, "stepq_selftest_bounded_wait: result is NULL");
+    if (limit_cycles < 0 || limit_cycles > (1LL << 34))
+        return fail(STEPQ_ERR_INVALID_ARG, "stepq_selftest_bounded_wait: limit_cycles %lld outside [0, 2^34]",
+                    limit_cycles);
+    cudaError_t e = stepq::launch_wait_selftest(result, limit_cycles, arrive ? 1 : 0,
+                                                static_cast<cudaStream_t>(cuda_stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stepq_selftest_bounded_wait launch");
+    return STEPQ_OK;
+}
+
 stepq_status stepq_pool_check_guards(stepq_pool *pool)
 {
     stepq_status st = check_pool(pool);

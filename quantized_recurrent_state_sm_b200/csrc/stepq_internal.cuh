@@ -103,6 +103,9 @@ cudaError_t launch_unpack(const StepArgs &a, cudaStream_t s);
 // The pages' split pipeline, first half: reconstruct, update, read out; the
 // updated unquantised state goes to a.S_in (a work buffer), for launch_pack.
 cudaError_t launch_split_update(const StepArgs &a, cudaStream_t s);
+// Self-test of the bounded barrier wait the kernels use (one CTA): result[0] =
+// 0 or kStatusWaitTimeout, result[1] = cycles waited (saturated).
+cudaError_t launch_wait_selftest(int *result, long long limit, int arrive, cudaStream_t s);
 // Calibration kernels (the offline step that makes a pool's tables).
 constexpr int kCalibMaxWidths = 8;
 struct CalibArgs {

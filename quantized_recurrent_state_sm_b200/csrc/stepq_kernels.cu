@@ -1178,6 +1178,25 @@ __device__ __forceinline__ void abort_drain(ItemSmem &sm, const StepArgs &a, uin
     __syncthreads();
 }
 
+// Self-test of the bounded wait (one CTA, thread 0): a barrier that needs one
+// arrival, which thread 0 makes first when `arrive` is set; otherwise nothing
+// arrives and the wait gives up after `limit` cycles, as a wait for a staged
+// copy that never lands does in the decode kernel.  result[0]: 0 or
+// kStatusWaitTimeout; result[1]: cycles spent in the wait (saturated).
+__global__ void k_wait_selftest(int *result, long long limit, int arrive)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    if (arrive) mbar_arrive(&bar);
+    const long long t0 = clock64();
+    const bool ok = mbar_wait_bounded(&bar, 0u, limit);
+    const long long dt = clock64() - t0;
+    result[0] = ok ? 0 : kStatusWaitTimeout;
+    result[1] = (int)min(dt, 2147483647LL);
+}
+
 // NP (row-wise widths): the leading positions checked for 16-bit fields; 1
 // when no head of the pool has more than one, else all 16.
 template <bool KDA, bool MULTI, int NP, int MODE>
@@ -1824,6 +1843,12 @@ cudaError_t launch_unpack(const StepArgs &a, cudaStream_t s)
     if (a.n_items == 0) return cudaSuccess;
     check_tables(a, 0, s);
     k_unpack<<<a.n_items, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(int *result, long long limit, int arrive, cudaStream_t s)
+{
+    k_wait_selftest<<<1, 32, 0, s>>>(result, limit, arrive);
     return cudaGetLastError();
 }
 

@@ -55,7 +55,7 @@ class CalibDesc(C.Structure):
 
 EXPORTS = ("stepq_pool_bytes", "stepq_state_bytes", "stepq_pool_layout", "stepq_pool_check_guards", "stepq_pool_create", "stepq_pool_destroy",
            "stepq_pool_set_stream", "stepq_pack", "stepq_unpack", "stepq_decode_step",
-           "stepq_fp32_step", "stepq_pool_check", "stepq_status_string", "stepq_last_error",
+           "stepq_fp32_step", "stepq_pool_check", "stepq_status_string", "stepq_last_error", "stepq_selftest_bounded_wait",
            "stepq_decode_step_noalloc", "stepq_decode_step_split", "stepq_pool_set_active",
            "stepq_pool_set_scale_mode", "stepq_calib_scratch_bytes", "stepq_calibrate", "stepq_calib_accumulate", "stepq_calib_row_error",
            "stepq_calib_reduce", "stepq_calib_rho", "stepq_calib_bits")
@@ -75,6 +75,7 @@ def _load():
     L.stepq_pool_check.argtypes = [P]
     L.stepq_pool_check_guards.argtypes = [P]
     L.stepq_pool_layout.argtypes = [D, C.POINTER(Regions)]
+    L.stepq_selftest_bounded_wait.argtypes = [P, C.c_longlong, C.c_int, P]
     L.stepq_pack.argtypes = [P, P]
     L.stepq_unpack.argtypes = [P, P]
     L.stepq_decode_step.argtypes = [P, P, P, P, P, P, P]
@@ -91,7 +92,8 @@ def _load():
     L.stepq_calib_reduce.argtypes = [i, i, i, P, P, P]
     L.stepq_calib_rho.argtypes = [i, dbl, P, P]
     L.stepq_calib_bits.argtypes = [i, i, dbl, P, P, P, i, P, dbl, dbl, P]
-    for fn in ("stepq_pool_create", "stepq_pool_destroy", "stepq_pool_set_stream", "stepq_pool_check", "stepq_pack",
+    for fn in ("stepq_pool_create", "stepq_pool_destroy", "stepq_pool_set_stream", "stepq_pool_check",
+               "stepq_selftest_bounded_wait", "stepq_pack",
                "stepq_unpack", "stepq_decode_step", "stepq_fp32_step", "stepq_decode_step_noalloc",
                "stepq_decode_step_split", "stepq_pool_set_active", "stepq_pool_set_scale_mode", "stepq_calibrate", "stepq_calib_accumulate",
                "stepq_calib_row_error", "stepq_calib_reduce", "stepq_calib_rho", "stepq_calib_bits"):
@@ -311,6 +313,17 @@ def decode_step_noalloc(variant: int, bits, rho, states: torch.Tensor, q, k, v, 
                                          _dev(beta, "beta", (B, H)), _dev(out, "out", (B, H, DV)),
                                          _stream_ptr()))
     return out
+
+
+def selftest_bounded_wait(limit_cycles: int, arrive: bool, device=None) -> tuple[int, int]:
+    """Run the kernels' bounded barrier wait once (include/stepq.h,
+    stepq_selftest_bounded_wait): (0 or 1 = gave up, cycles waited)."""
+    res = torch.full((2,), -1, dtype=torch.int32, device=device or "cuda")
+    _check(lib.stepq_selftest_bounded_wait(C.c_void_p(res.data_ptr()), int(limit_cycles), int(bool(arrive)),
+                                           _stream_ptr()))
+    torch.cuda.current_stream().synchronize()
+    r = res.cpu().tolist()
+    return r[0], r[1]
 
 
 # ---- calibration -------------------------------------------------------------

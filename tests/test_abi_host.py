@@ -201,3 +201,11 @@ def test_pool_layout_regions_and_guards(S):
             assert g[k] % 16 == 0 and g[k] + r.guard_bytes <= (starts[k + 1] if k < 6 else r.total), (ci, k)
         assert starts[1] % 256 == 0 and all(x % 16 == 0 for x in starts)
     assert S.lib.stepq_pool_layout(None, C.byref(r)) == S.ERR_INVALID_ARG
+
+
+def test_selftest_bounded_wait_arguments(S):
+    """Argument checks of the wait self-test happen on the host."""
+    assert S.lib.stepq_selftest_bounded_wait(None, 1000, 0, None) == S.ERR_INVALID_ARG
+    assert S.lib.stepq_selftest_bounded_wait(C.c_void_p(16), -1, 0, None) == S.ERR_INVALID_ARG
+    assert S.lib.stepq_selftest_bounded_wait(C.c_void_p(16), (1 << 34) + 1, 0, None) == S.ERR_INVALID_ARG
+    assert "limit_cycles" in S.lib.stepq_last_error().decode()
