@@ -9,7 +9,7 @@ from tests.test_gpu_parity import Setup, lockstep
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("ci,batch", [(0, 4), (1, 2), (2, 2), (4, 2)])
+@pytest.mark.parametrize("ci,batch", [(0, 4), (1, 2), (2, 2), (3, 2), (4, 2)])
 def test_split_pipeline_lockstep(ci, batch):
     cfg = W.with_overrides(W.CONFIGS[ci], batch=batch)
     setup = Setup(cfg)
