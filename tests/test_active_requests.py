@@ -18,7 +18,7 @@ def _pool(stepq, cfg):
     return stepq.PackedStatePool(cfg.variant, cfg.batch, cfg.heads, bits, rho, cfg.ls_iters)
 
 
-@pytest.mark.parametrize("ci", [1, 2, 4])
+@pytest.mark.parametrize("ci", [1, 2, 3, 4])
 def test_active_subset_matches_oracle(ci):
     from tests.test_gpu_parity import Setup, lockstep
     cfg = W.with_overrides(W.CONFIGS[ci], batch=6)
