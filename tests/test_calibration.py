@@ -245,7 +245,7 @@ def test_gpu_calib_accumulate(ci):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("ci,ls", [(1, 1), (2, 1), (3, 2)])
+@pytest.mark.parametrize("ci,ls", [(1, 1), (2, 1), (3, 2), (4, 1)])
 def test_gpu_calib_row_error(ci, ls):
     """Per-row errors, r' and c of every candidate width against the oracle.
     r': relative 2e-5 (fp32 fits whose sums run in another order, and the
@@ -288,7 +288,7 @@ def test_gpu_calib_row_error(ci, ls):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("ci", [1, 2])
+@pytest.mark.parametrize("ci", [1, 2, 4])
 def test_gpu_calibrate_end_to_end(ci):
     """stepq_calibrate: rho identical to the oracle's (same exact sums); the
     widths equal the oracle's allocation of the GPU's own error sums (taken
