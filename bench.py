@@ -911,7 +911,7 @@ def main():
         if split is not None:
             split["fused_speedup"] = split["ms_per_step"] / ms_per_step
             line["split_pipeline"] = split
-        if not (args.no_cpu_baseline or args.profile):
+        if world == 1 and not (args.no_cpu_baseline or args.profile):  # the host baseline at N = 1 only
             rate, meta = cpu_oracle_rate(cfg, args.cpu_seconds)
             line["cpu_baseline"] = dict(value=rate, unit=UNIT, **meta)
             rate1, meta1 = cpu_oracle_rate(cfg, max(1.0, args.cpu_seconds / 2), cores=1)
